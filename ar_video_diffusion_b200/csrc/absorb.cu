@@ -1,0 +1,328 @@
+// Layer Absorb: the closed-form ridge solve
+//   dW = (G + lambda I)^-1 R W,   lambda = lambda_abs + lambda_rel tr(G) / D,
+// ("Towards Memory-Efficient Autoregressive Video Generation via
+// Instance-Specific Parametric Absorption", gist.science technical summary,
+// section 2 stage 2 "Layer Absorb"), then W_new = W + dW (stage 3).
+//
+// fp32 throughout, all on the device, stream ordered:
+//   1. trace(G) -> lambda (one block, fp64 sum);  M = G + lambda I;
+//   2. S = R W  (written straight into dW, which the solves then update in place);
+//   3. right-looking blocked Cholesky M = L L^T with 64 x 64 panels: the
+//      diagonal block is factored in shared memory by one CTA (which also
+//      forms its inverse), the panel below is multiplied by that inverse, and
+//      the trailing lower triangle gets a rank-64 update;
+//   4. L Y = S, then L^T X = Y, block by block with the stored diagonal
+//      inverses and rank-64 updates of the remaining rows;
+//   5. W_new = W + dW, rounded to W's dtype.
+// The fp32 GEMM used by steps 2-4 (and by the fp32 activation path of the
+// statistics and the projection) is a 64 x 64-tile CUDA-core kernel with
+// arbitrary strides, so transposed operands are read in place.
+#include <cstring>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace ispa {
+namespace simt {
+
+constexpr int kT = 64;   // tile edge
+constexpr int kTK = 16;  // K slice per shared-memory stage
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// C[m, n] = beta * C[m, n] + alpha * sum_k A(m, k) B(k, n) with
+// A(m, k) = A[m * a_rs + k * a_cs], B(k, n) = B[k * b_rs + n * b_cs].
+// lower_only: tiles strictly above the block diagonal are skipped.
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) gemm_f32_kernel(int M, int N, int K, float alpha, const TA* __restrict__ A,
+                                                       int64_t a_rs, int64_t a_cs, const TB* __restrict__ B,
+                                                       int64_t b_rs, int64_t b_cs, float beta, float* C,
+                                                       int64_t ldc, int lower_only) {
+  const int tm = blockIdx.y, tn = blockIdx.x;
+  if (lower_only && tn > tm) return;
+  __shared__ float As[kTK][kT + 4];
+  __shared__ float Bs[kTK][kT + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  const int m0 = tm * kT, n0 = tn * kT;
+  float acc[4][4] = {};
+  const bool a_k_fast = a_cs == 1;
+  const bool b_n_fast = b_cs == 1;
+  for (int k0 = 0; k0 < K; k0 += kTK) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + 256 * i;
+      int mm, kk;
+      if (a_k_fast) {
+        kk = idx % kTK;
+        mm = idx / kTK;
+      } else {
+        mm = idx % kT;
+        kk = idx / kT;
+      }
+      const int gm = m0 + mm, gk = k0 + kk;
+      As[kk][mm] = (gm < M && gk < K) ? to_f32(A[gm * a_rs + gk * a_cs]) : 0.f;
+      int nn, kb;
+      if (b_n_fast) {
+        nn = idx % kT;
+        kb = idx / kT;
+      } else {
+        kb = idx % kTK;
+        nn = idx / kTK;
+      }
+      const int gn = n0 + nn, gkb = k0 + kb;
+      Bs[kb][nn] = (gn < N && gkb < K) ? to_f32(B[gkb * b_rs + gn * b_cs]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kTK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gm = m0 + ty + 16 * i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx + 16 * j;
+      if (gn >= N) continue;
+      float* c = C + gm * ldc + gn;
+      *c = (beta == 0.f ? 0.f : beta * *c) + alpha * acc[i][j];
+    }
+  }
+}
+
+template <typename TA, typename TB>
+void gemm_f32(cudaStream_t st, int M, int N, int K, float alpha, const TA* A, int64_t a_rs, int64_t a_cs, const TB* B,
+              int64_t b_rs, int64_t b_cs, float beta, float* C, int64_t ldc, bool lower_only = false) {
+  if (M <= 0 || N <= 0) return;
+  dim3 grid((N + kT - 1) / kT, (M + kT - 1) / kT);
+  gemm_f32_kernel<TA, TB><<<grid, 256, 0, st>>>(M, N, K, alpha, A, a_rs, a_cs, B, b_rs, b_cs, beta, C, ldc,
+                                                lower_only ? 1 : 0);
+}
+
+// ---------------------------------------------------------------- absorb
+__global__ void trace_lambda_kernel(const float* __restrict__ G, int D, double lam_abs, double lam_rel,
+                                    double* __restrict__ lam_out) {
+  __shared__ double part[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) s += (double)G[(int64_t)i * D + i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) part[threadIdx.x] += part[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *lam_out = lam_abs + lam_rel * part[0] / D;
+}
+
+__global__ void shift_kernel(const float* __restrict__ G, float* __restrict__ M, int D,
+                             const double* __restrict__ lam) {
+  const float l = (float)*lam;
+  const int64_t total = (int64_t)D * D / 4;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    float4 g = reinterpret_cast<const float4*>(G)[e];
+    const int64_t i = (e * 4) / D, j0 = (e * 4) % D;
+    if (i >= j0 && i < j0 + 4) (&g.x)[i - j0] += l;
+    reinterpret_cast<float4*>(M)[e] = g;
+  }
+}
+
+// Factor the 64 x 64 diagonal block k of M in place (lower triangle) and
+// write the inverse of its Cholesky factor to Linv (64 x 64, row-major).
+__global__ void __launch_bounds__(256) potrf_diag_kernel(float* M, int D, int k, float* Linv, int32_t* status) {
+  __shared__ float A[kT][kT + 1];
+  __shared__ float X[kT][kT + 1];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  float* blk = M + (int64_t)k * kT * D + (int64_t)k * kT;
+  for (int e = tid; e < kT * kT; e += 256) A[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
+  if (tid == 0) bad = -1;
+  __syncthreads();
+  for (int j = 0; j < kT; ++j) {
+    if (tid == 0) {
+      float d = A[j][j];
+      if (!(d > 0.f) || !isfinite(d)) {
+        if (bad < 0) bad = j;
+        d = 1.f;
+      }
+      A[j][j] = sqrtf(d);
+    }
+    __syncthreads();
+    const float inv = 1.0f / A[j][j];
+    for (int i = j + 1 + tid; i < kT; i += 256) A[i][j] *= inv;
+    __syncthreads();
+    const int n = kT - 1 - j;
+    for (int e = tid; e < n * n; e += 256) {
+      const int i = j + 1 + e / n, c = j + 1 + e % n;
+      if (c <= i) A[i][c] -= A[i][j] * A[c][j];
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && bad >= 0 && status) {
+    if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = k * kT + bad;
+  }
+  // inverse of the lower-triangular factor, one column per thread
+  if (tid < kT) {
+    const int c = tid;
+    for (int i = 0; i < kT; ++i) {
+      if (i < c) {
+        X[i][c] = 0.f;
+        continue;
+      }
+      float s = (i == c) ? 1.f : 0.f;
+      for (int t = c; t < i; ++t) s -= A[i][t] * X[t][c];
+      X[i][c] = s / A[i][i];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < kT * kT; e += 256) {
+    const int i = e / kT, c = e % kT;
+    if (c <= i) blk[(int64_t)i * D + c] = A[i][c];
+    Linv[e] = X[i][c];
+  }
+}
+
+// Panel below diagonal block k: M[r, k] <- M[r, k] Linv_k^T, one 64-row block per CTA.
+__global__ void __launch_bounds__(256) panel_kernel(float* M, int D, int k, const float* __restrict__ Linv) {
+  __shared__ float Li[kT][kT + 1];
+  __shared__ float P[kT][kT + 1];
+  const int r = k + 1 + blockIdx.x;
+  float* blk = M + (int64_t)r * kT * D + (int64_t)k * kT;
+  for (int e = threadIdx.x; e < kT * kT; e += 256) {
+    Li[e / kT][e % kT] = Linv[e];
+    P[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kT * kT; e += 256) {
+    const int i = e / kT, c = e % kT;
+    float s = 0.f;
+    for (int t = 0; t <= c; ++t) s = fmaf(P[i][t], Li[c][t], s);
+    blk[(int64_t)i * D + c] = s;
+  }
+}
+
+// X[k-block rows, :] <- Linv_k X  (transpose_l = 0) or Linv_k^T X (1), in place;
+// one 64-column slab per CTA.
+__global__ void __launch_bounds__(256) diag_apply_kernel(float* X, int D, int k, const float* __restrict__ Linv,
+                                                         int transpose_l) {
+  __shared__ float Li[kT][kT + 1];
+  __shared__ float T[kT][kT + 1];
+  float* blk = X + (int64_t)k * kT * D + (int64_t)blockIdx.x * kT;
+  for (int e = threadIdx.x; e < kT * kT; e += 256) {
+    Li[e / kT][e % kT] = Linv[e];
+    T[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kT * kT; e += 256) {
+    const int i = e / kT, c = e % kT;
+    float s = 0.f;
+    if (!transpose_l) {
+      for (int t = 0; t <= i; ++t) s = fmaf(Li[i][t], T[t][c], s);
+    } else {
+      for (int t = i; t < kT; ++t) s = fmaf(Li[t][i], T[t][c], s);
+    }
+    blk[(int64_t)i * D + c] = s;
+  }
+}
+
+template <typename TW>
+__global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ dW, TW* __restrict__ Wn, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float v = to_f32(W[e]) + dW[e];
+    if constexpr (sizeof(TW) == 2)
+      Wn[e] = __float2bfloat16_rn(v);
+    else
+      Wn[e] = v;
+  }
+}
+
+}  // namespace simt
+
+size_t absorb_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
+
+ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D64,
+                                  double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
+                                  int32_t* status, cudaStream_t st) {
+  using namespace simt;
+  const int D = (int)D64;
+  const int nb = D / kT;
+  float* M = static_cast<float*>(workspace);
+  float* Linv = M + (int64_t)D * D;
+  double* lam = reinterpret_cast<double*>(Linv + (int64_t)D * kT);
+
+  trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
+  const int sms = num_sms();
+  shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
+  // S = R W, written into dW
+  if (w_dt == ISPA_DT_BF16)
+    gemm_f32(st, D, D, D, 1.f, R, D, 1, static_cast<const __nv_bfloat16*>(W), D, 1, 0.f, dW, D);
+  else
+    gemm_f32(st, D, D, D, 1.f, R, D, 1, static_cast<const float*>(W), D, 1, 0.f, dW, D);
+  // Cholesky
+  for (int k = 0; k < nb; ++k) {
+    float* Lk = Linv + (int64_t)k * kT * kT;
+    potrf_diag_kernel<<<1, 256, 0, st>>>(M, D, k, Lk, status);
+    const int rest = nb - k - 1;
+    if (rest > 0) {
+      panel_kernel<<<rest, 256, 0, st>>>(M, D, k, Lk);
+      const int off = (k + 1) * kT;
+      const float* P = M + (int64_t)off * D + (int64_t)k * kT;
+      gemm_f32(st, D - off, D - off, kT, -1.f, P, D, 1, P, 1, D, 1.f, M + (int64_t)off * D + off, D, true);
+    }
+  }
+  // forward: L Y = S
+  for (int k = 0; k < nb; ++k) {
+    diag_apply_kernel<<<nb, 256, 0, st>>>(dW, D, k, Linv + (int64_t)k * kT * kT, 0);
+    const int off = (k + 1) * kT;
+    if (off < D)
+      gemm_f32(st, D - off, D, kT, -1.f, M + (int64_t)off * D + (int64_t)k * kT, D, 1, dW + (int64_t)k * kT * D, D,
+               1, 1.f, dW + (int64_t)off * D, D);
+  }
+  // backward: L^T X = Y
+  for (int k = nb - 1; k >= 0; --k) {
+    diag_apply_kernel<<<nb, 256, 0, st>>>(dW, D, k, Linv + (int64_t)k * kT * kT, 1);
+    const int rows = k * kT;
+    if (rows > 0)
+      gemm_f32(st, rows, D, kT, -1.f, M + (int64_t)k * kT * D, 1, D, dW + (int64_t)k * kT * D, D, 1, 1.f, dW, D);
+  }
+  if (w_new) {
+    const int64_t n = (int64_t)D * D;
+    if (w_dt == ISPA_DT_BF16)
+      wnew_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), dW,
+                                           static_cast<__nv_bfloat16*>(w_new), n);
+    else
+      wnew_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(W), dW, static_cast<float*>(w_new), n);
+  }
+  return check_launch("absorb_solve");
+}
+
+// fp32 activation path of the statistics: [G | R] (+)= A_loc^T [A_loc | delta].
+ispa_status_t gram_f32(const float* a_loc, const float* a_delta, int64_t n_rows, int64_t D, int64_t row_stride,
+                       float* G, float* R, bool overwrite, cudaStream_t st) {
+  using namespace simt;
+  const float beta = overwrite ? 0.f : 1.f;
+  gemm_f32(st, (int)D, (int)D, (int)n_rows, 1.f, a_loc, 1, row_stride, a_loc, row_stride, 1, beta, G, D);
+  gemm_f32(st, (int)D, (int)D, (int)n_rows, 1.f, a_loc, 1, row_stride, a_delta, row_stride, 1, beta, R, D);
+  return check_launch("gram_f32");
+}
+
+// fp32 activation path of the projection: y = a w.
+ispa_status_t project_f32(const float* a, int64_t n_rows, int64_t d_in, int64_t d_out, int64_t a_stride,
+                          const float* w, float* y, cudaStream_t st) {
+  simt::gemm_f32(st, (int)n_rows, (int)d_out, (int)d_in, 1.f, a, a_stride, 1, w, d_out, 1, 0.f, y, d_out);
+  return check_launch("project_f32");
+}
+
+}  // namespace ispa

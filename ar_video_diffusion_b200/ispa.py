@@ -1,0 +1,299 @@
+"""Python binding of libispa (ctypes), same names as the C ABI in include/ispa.h.
+
+Argument marshalling only: tensors are passed as raw device pointers with their
+sizes and strides, the caller's current CUDA stream is forwarded, and non-OK
+status codes raise ``IspaError``.  Every step of the computation runs in the
+CUDA kernels of libispa.so; there is no fallback of any kind -- importing the
+functions works without a GPU, but calling a device entry point without the
+built library or without a GPU raises.
+
+Thin convenience wrappers (``dual_attention``, ``gram_accumulate``,
+``absorb_solve``, ``local_attention_project``, ``project``, ``lse_merge``)
+allocate the outputs with torch and call the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libispa.so")
+
+ISPA_OK = 0
+STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTED", 3: "ISPA_ERR_CUDA",
+                4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT", 6: "ISPA_ERR_WORKSPACE"}
+DT_BF16, DT_F32 = 0, 1
+MAX_SEGMENTS = 8
+
+# every symbol declared in include/ispa.h
+EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "ispa_absorb_workspace_bytes",
+            "ispa_absorb_solve", "ispa_project", "ispa_local_attention_project", "ispa_chunk_token_ranges",
+            "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
+            "ispa_version")
+
+
+class IspaError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}: {detail}")
+
+
+class KVSegment(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n_tokens", ctypes.c_int64),
+                ("row_stride", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libispa.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m ar_video_diffusion_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        i32, i64, f32, f64, vp, sz = c.c_int32, c.c_int64, c.c_float, c.c_double, c.c_void_p, c.c_size_t
+        seg_p = c.POINTER(KVSegment)
+        sig = {
+            "ispa_dual_attention": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, seg_p, i32, vp, vp, vp, vp,
+                                          vp, vp, vp]),
+            "ispa_lse_merge": (i32, [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]),
+            "ispa_gram_accumulate": (i32, [vp, vp, i64, i64, i64, i32, vp, vp, i32, vp]),
+            "ispa_absorb_workspace_bytes": (sz, [i64]),
+            "ispa_absorb_solve": (i32, [vp, vp, vp, i32, i64, f64, f64, vp, vp, vp, sz, vp, vp]),
+            "ispa_project": (i32, [vp, i64, i64, i64, i64, i32, vp, vp, vp]),
+            "ispa_local_attention_project": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp, vp,
+                                                   vp]),
+            "ispa_chunk_token_ranges": (i32, [i64, i64, i64, i64, c.POINTER(i64)]),
+            "ispa_kv_bytes": (i64, [i64, i32, c.c_uint64, i32, i64, i64, i64, i32, i64]),
+            "ispa_selftest_wait_timeout": (i32, [c.c_uint32, vp, vp]),
+            "ispa_status_string": (c.c_char_p, [i32]),
+            "ispa_last_error": (c.c_char_p, []),
+            "ispa_version": (i32, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != ISPA_OK:
+        raise IspaError(code, where, lib().ispa_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DT_BF16
+    if t.dtype == torch.float32:
+        return DT_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(t: Optional[torch.Tensor], name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t.data_ptr()
+
+
+def _row_stride(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D row-major matrix")
+    return t.stride(0)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _segments(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]]):
+    arr = (KVSegment * max(1, len(pairs)))()
+    for i, (k, v) in enumerate(pairs):
+        if k.shape != v.shape or k.stride() != v.stride():
+            raise ValueError("k and v of a segment must have the same shape and strides")
+        arr[i] = KVSegment(_dev(k, "k") if k.numel() else None, _dev(v, "v") if v.numel() else None,
+                           k.shape[0], _row_stride(k, "k") if k.shape[0] else k.shape[1])
+    return arr, len(pairs)
+
+
+# ------------------------------------------------------------ raw C entry points
+def ispa_dual_attention(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local, hist, n_hist,
+                        a_loc, a_full, a_delta, lse_loc, lse_full, dev_status, stream):
+    _check(lib().ispa_dual_attention(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local, hist,
+                                     n_hist, a_loc, a_full, a_delta, lse_loc, lse_full, dev_status, stream),
+           "ispa_dual_attention")
+
+
+def ispa_lse_merge(o_loc, lse_loc, o_hist, lse_hist, n_q, n_heads, head_dim, dt, a_full, a_delta, lse_full, stream):
+    _check(lib().ispa_lse_merge(o_loc, lse_loc, o_hist, lse_hist, n_q, n_heads, head_dim, dt, a_full, a_delta,
+                                lse_full, stream), "ispa_lse_merge")
+
+
+def ispa_gram_accumulate(a_loc, a_delta, n_rows, d_model, row_stride, dt, G, R, zero_first, stream):
+    _check(lib().ispa_gram_accumulate(a_loc, a_delta, n_rows, d_model, row_stride, dt, G, R, zero_first, stream),
+           "ispa_gram_accumulate")
+
+
+def ispa_absorb_workspace_bytes(d_model: int) -> int:
+    return lib().ispa_absorb_workspace_bytes(d_model)
+
+
+def ispa_absorb_solve(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, workspace, workspace_bytes,
+                      dev_status, stream):
+    _check(lib().ispa_absorb_solve(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, workspace,
+                                   workspace_bytes, dev_status, stream), "ispa_absorb_solve")
+
+
+def ispa_project(a, n_rows, d_in, d_out, a_stride, dt, w, y, stream):
+    _check(lib().ispa_project(a, n_rows, d_in, d_out, a_stride, dt, w, y, stream), "ispa_project")
+
+
+def ispa_local_attention_project(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local, w_new, y,
+                                 a_loc_out, dev_status, stream):
+    _check(lib().ispa_local_attention_project(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local,
+                                              n_local, w_new, y, a_loc_out, dev_status, stream),
+           "ispa_local_attention_project")
+
+
+def ispa_chunk_token_ranges(chunk: int, frame_tokens: int, chunk_frames: int, sink_frames: int = 1):
+    out = (ctypes.c_int64 * 6)()
+    _check(lib().ispa_chunk_token_ranges(chunk, frame_tokens, chunk_frames, sink_frames, out),
+           "ispa_chunk_token_ranges")
+    return {"sink": (out[0], out[1]), "hist": (out[2], out[3]), "cur": (out[4], out[5])}
+
+
+def ispa_kv_bytes(chunk, n_layers, l_layer_mask, transitioned, frame_tokens, chunk_frames, d_model, elem_bytes,
+                  sink_frames=1) -> int:
+    r = lib().ispa_kv_bytes(chunk, n_layers, l_layer_mask, int(bool(transitioned)), frame_tokens, chunk_frames,
+                            d_model, elem_bytes, sink_frames)
+    if r < 0:
+        raise IspaError(1, "ispa_kv_bytes", "invalid arguments")
+    return r
+
+
+def ispa_selftest_wait_timeout(timeout_us, dev_status, stream):
+    _check(lib().ispa_selftest_wait_timeout(timeout_us, dev_status, stream), "ispa_selftest_wait_timeout")
+
+
+def ispa_status_string(code: int) -> str:
+    return lib().ispa_status_string(code).decode()
+
+
+def ispa_version() -> int:
+    return lib().ispa_version()
+
+
+# ------------------------------------------------------- torch-level wrappers
+def new_status(device="cuda") -> torch.Tensor:
+    """Zeroed two-int32 device status word (code, detail)."""
+    return torch.zeros(2, dtype=torch.int32, device=device)
+
+
+def raise_on_status(status: torch.Tensor, where: str):
+    code, detail = (int(x) for x in status.cpu().tolist())
+    if code != 0:
+        raise IspaError(code, where, f"device status detail {detail}")
+
+
+def dual_attention(q: torch.Tensor, local: Sequence[Tuple[torch.Tensor, torch.Tensor]],
+                   hist: Sequence[Tuple[torch.Tensor, torch.Tensor]], n_heads: int, softmax_scale: float = 0.0,
+                   dual: bool = True, out: Optional[dict] = None, status: Optional[torch.Tensor] = None,
+                   stream=None) -> dict:
+    """Decomposable Attention of one chunk; returns a dict of output tensors.
+
+    dual=True: a_loc, a_full, a_delta, lse_loc, lse_full.  dual=False: one
+    pass over local + hist giving a_full and lse_full.
+    """
+    n_q, D = q.shape
+    head_dim = D // n_heads
+    dev = q.device
+    if out is None:
+        out = {"a_full": torch.empty(n_q, D, dtype=q.dtype, device=dev),
+               "lse_full": torch.empty(n_heads, n_q, dtype=torch.float32, device=dev)}
+        if dual:
+            out["a_loc"] = torch.empty(n_q, D, dtype=q.dtype, device=dev)
+            out["a_delta"] = torch.empty(n_q, D, dtype=q.dtype, device=dev)
+            out["lse_loc"] = torch.empty(n_heads, n_q, dtype=torch.float32, device=dev)
+    ls, nl = _segments(local)
+    hs, nh = _segments(hist)
+    ispa_dual_attention(_dev(q, "q"), n_q, _row_stride(q, "q"), n_heads, head_dim, _dtype_code(q), softmax_scale,
+                        ls, nl, hs, nh, _dev(out.get("a_loc"), "a_loc"), _dev(out["a_full"], "a_full"),
+                        _dev(out.get("a_delta"), "a_delta"), _dev(out.get("lse_loc"), "lse_loc"),
+                        _dev(out.get("lse_full"), "lse_full"), _dev(status, "status"), _stream(stream))
+    return out
+
+
+def lse_merge(o_loc, lse_loc, o_hist, lse_hist, n_heads: int, out: Optional[dict] = None, stream=None) -> dict:
+    n_q, D = o_loc.shape
+    if out is None:
+        out = {"a_full": torch.empty_like(o_loc), "a_delta": torch.empty_like(o_loc),
+               "lse_full": torch.empty_like(lse_loc)}
+    ispa_lse_merge(_dev(o_loc, "o_loc"), _dev(lse_loc, "lse_loc"), _dev(o_hist, "o_hist"), _dev(lse_hist, "lse_hist"),
+                   n_q, n_heads, D // n_heads, _dtype_code(o_loc), _dev(out["a_full"], "a_full"),
+                   _dev(out.get("a_delta"), "a_delta"), _dev(out.get("lse_full"), "lse_full"), _stream(stream))
+    return out
+
+
+def gram_accumulate(a_loc: torch.Tensor, a_delta: torch.Tensor, G: torch.Tensor, R: torch.Tensor,
+                    zero_first: bool = False, stream=None):
+    n, D = a_loc.shape
+    ispa_gram_accumulate(_dev(a_loc, "a_loc"), _dev(a_delta, "a_delta"), n, D, _row_stride(a_loc, "a_loc"),
+                         _dtype_code(a_loc), _dev(G, "G"), _dev(R, "R"), int(zero_first), _stream(stream))
+
+
+def absorb_workspace(d_model: int, device="cuda") -> torch.Tensor:
+    nbytes = ispa_absorb_workspace_bytes(d_model)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def absorb_solve(G: torch.Tensor, R: torch.Tensor, W: torch.Tensor, lambda_rel: float = 1e-2,
+                 lambda_abs: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                 status: Optional[torch.Tensor] = None, delta_w: Optional[torch.Tensor] = None,
+                 w_new: Optional[torch.Tensor] = None, stream=None):
+    D = G.shape[0]
+    if workspace is None:
+        workspace = absorb_workspace(D, G.device)
+    if delta_w is None:
+        delta_w = torch.empty(D, D, dtype=torch.float32, device=G.device)
+    if w_new is None:
+        w_new = torch.empty_like(W)
+    ispa_absorb_solve(_dev(G, "G"), _dev(R, "R"), _dev(W, "W"), _dtype_code(W), D, lambda_abs, lambda_rel,
+                      _dev(delta_w, "delta_w"), _dev(w_new, "w_new"), _dev(workspace, "workspace"),
+                      workspace.numel(), _dev(status, "status"), _stream(stream))
+    return delta_w, w_new
+
+
+def project(a: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    n, d_in = a.shape
+    d_out = w.shape[1]
+    if y is None:
+        y = torch.empty(n, d_out, dtype=a.dtype, device=a.device)
+    ispa_project(_dev(a, "a"), n, d_in, d_out, _row_stride(a, "a"), _dtype_code(a), _dev(w, "w"), _dev(y, "y"),
+                 _stream(stream))
+    return y
+
+
+def local_attention_project(q: torch.Tensor, local: Sequence[Tuple[torch.Tensor, torch.Tensor]], w_new: torch.Tensor,
+                            n_heads: int, softmax_scale: float = 0.0, y: Optional[torch.Tensor] = None,
+                            a_loc: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                            stream=None):
+    n_q, D = q.shape
+    if y is None:
+        y = torch.empty(n_q, D, dtype=q.dtype, device=q.device)
+    if a_loc is None:
+        a_loc = torch.empty(n_q, D, dtype=q.dtype, device=q.device)
+    ls, nl = _segments(local)
+    ispa_local_attention_project(_dev(q, "q"), n_q, _row_stride(q, "q"), n_heads, D // n_heads, _dtype_code(q),
+                                 softmax_scale, ls, nl, _dev(w_new, "w_new"), _dev(y, "y"), _dev(a_loc, "a_loc"),
+                                 _dev(status, "status"), _stream(stream))
+    return y, a_loc

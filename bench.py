@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the ISPA hot path on B200 (one JSON line on rank 0).
+
+One step = one pass of the whole hot path for one Wan-1.3B-shaped layer
+(12 heads x 128, 4680 chunk queries, 1560 sink + 18720 history keys, bf16):
+  dual-stream attention (local + history branches, fused LSE merge)
+  -> warm-up output projection y = A_full W
+  -> Gram / cross-covariance accumulation G += A_loc^T A_loc, R += A_loc^T delta
+  -> absorb solve dW = (G + lambda I)^-1 R W and W_new = W + dW
+  -> L-layer chunk: local-only attention + projection with W_new
+  -> F-layer chunk: single-pass attention over all keys + projection with W.
+The headline value is the dual-stream attention throughput (algorithmic
+FLOPs 4 n_q n_k d H over the kernel's CUDA-event time); absorb ms/layer and
+the L-/F-layer chunk latencies are reported beside it.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With --gpus N > 1 (launched under torchrun) every rank runs the same layer
+(replicas: the single-layer path has no data exchange), value = all ranks'
+FLOPs / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from ar_video_diffusion_b200 import synth  # noqa: E402
+
+METRIC = "dual-stream attn TFLOP/s (% BF16 peak); absorb ms/layer; chunk latency"
+WORKLOAD = "wan1.3b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_flops(w) -> float:
+    n_k = w.n_sink + w.n_q + w.n_hist
+    return 4.0 * w.n_q * n_k * w.head_dim * w.n_heads
+
+
+def gram_flops(w, rows) -> float:
+    D = w.d_model
+    return rows * D * (D + 1) + 2.0 * rows * D * D
+
+
+def absorb_launches(D: int) -> int:
+    nb = D // 64
+    return 7 * nb  # trace, shift, R W, W_new + 3nb-2 Cholesky + 2(2nb-1) solves
+
+
+def cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.file.flush()
+        self.file.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, device):
+    from ar_video_diffusion_b200 import ispa
+
+    w = synth.WORKLOADS[WORKLOAD]
+    H, d, D = w.n_heads, w.head_dim, w.d_model
+    x = synth.single_layer_inputs(w, 1)
+    Wh = synth.weight(w, 0)
+
+    def t(a):
+        return torch.from_numpy(a).to(torch.bfloat16).to(device)
+
+    q, ks, vs, kc, vc, kh, vh = (t(x[k]) for k in ("q", "k_sink", "v_sink", "k_cur", "v_cur", "k_hist", "v_hist"))
+    W = t(Wh)
+    local = [(ks, vs), (kc, vc)]
+    hist = [(kh, vh)]
+    bf = dict(dtype=torch.bfloat16, device=device)
+    f32 = dict(dtype=torch.float32, device=device)
+    dual_out = {"a_loc": torch.empty(w.n_q, D, **bf), "a_full": torch.empty(w.n_q, D, **bf),
+                "a_delta": torch.empty(w.n_q, D, **bf), "lse_loc": torch.empty(H, w.n_q, **f32),
+                "lse_full": torch.empty(H, w.n_q, **f32)}
+    f_out = {"a_full": torch.empty(w.n_q, D, **bf), "lse_full": torch.empty(H, w.n_q, **f32)}
+    y_warm = torch.empty(w.n_q, D, **bf)
+    y_l, a_l = torch.empty(w.n_q, D, **bf), torch.empty(w.n_q, D, **bf)
+    y_f = torch.empty(w.n_q, D, **bf)
+    G, R = torch.empty(D, D, **f32), torch.empty(D, D, **f32)
+    dW, Wn = torch.empty(D, D, **f32), torch.empty(D, D, **bf)
+    ws = ispa.absorb_workspace(D, device)
+    status = ispa.new_status(device)
+    stream = torch.cuda.current_stream(device)
+
+    # statistics start from one chunk so the first solve already sees SPD data
+    ispa.dual_attention(q, local, hist, H, out=dual_out, status=status)
+    ispa.gram_accumulate(dual_out["a_loc"], dual_out["a_delta"], G, R, zero_first=True)
+
+    n_ev = 8
+    def step(evs):
+        evs[0].record(stream)
+        ispa.dual_attention(q, local, hist, H, out=dual_out, status=status)
+        evs[1].record(stream)
+        ispa.project(dual_out["a_full"], W, y_warm)
+        evs[2].record(stream)
+        ispa.gram_accumulate(dual_out["a_loc"], dual_out["a_delta"], G, R)
+        evs[3].record(stream)
+        ispa.absorb_solve(G, R, W, lambda_rel=1e-2, workspace=ws, status=status, delta_w=dW, w_new=Wn)
+        evs[4].record(stream)
+        ispa.local_attention_project(q, local, Wn, H, y=y_l, a_loc=a_l, status=status)
+        evs[5].record(stream)
+        ispa.dual_attention(q, local, hist, H, dual=False, out=f_out, status=status)
+        evs[6].record(stream)
+        ispa.project(f_out["a_full"], W, y_f)
+        evs[7].record(stream)
+
+    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        step(all_evs[i])
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.warmup, args.warmup + args.steps):
+        step(all_evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    code = int(status[0].item())
+    if code != 0:
+        raise RuntimeError(f"device status {ispa.STATUS_NAMES.get(code, code)} during the benchmark")
+
+    total_ms = t_start.elapsed_time(t_end)
+    parts = np.array([[all_evs[i][j].elapsed_time(all_evs[i][j + 1]) for j in range(n_ev - 1)]
+                      for i in range(args.warmup, args.warmup + args.steps)])
+    mean = parts.mean(axis=0)  # ms per component
+    t_dual = float(parts[:, 0].sum())
+    # max over ranks of the time that defines `value`, and of the step time
+    vals = torch.tensor([t_dual, total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    t_dual_max, total_max = (float(v) for v in vals.tolist())
+    F = attn_flops(w)
+    value = world * F * args.steps / (t_dual_max * 1e-3) / 1e12
+
+    # e2e through the public API with host buffers: pinned H2D of the chunk's
+    # new inputs (queries and the current chunk's K, V; the sink/history cache
+    # is device-resident state), the dual attention, D2H of A_full and LSE_full
+    hq = torch.from_numpy(x["q"]).to(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(x["k_cur"]).to(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(x["v_cur"]).to(torch.bfloat16).pin_memory()
+    out_a = torch.empty(w.n_q, D, dtype=torch.bfloat16).pin_memory()
+    out_l = torch.empty(H, w.n_q, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(kc), torch.empty_like(vc)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ispa.dual_attention(dq, [(ks, vs), (dk, dv)], hist, H, out=dual_out, status=status)
+        out_a.copy_(dual_out["a_full"], non_blocking=True)
+        out_l.copy_(dual_out["lse_full"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * F * args.steps / (float(e2e_ms.item()) * 1e-3) / 1e12
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = out_a.numel() * 2 + out_l.numel() * 4
+
+    # standalone LSE merge over rotating buffer sets larger than L2
+    merge_gbs = merge_bench(ispa, w, device)
+
+    pk, src = peaks()
+    tc_peak = pk["bf16_tflops"]
+    achieved = F / (t_dual / args.steps * 1e-3) / 1e12
+    traffic = load_traffic("dual_attention_kernel")
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded PCG64; Wan-1.3B latent shapes; random-init W)",
+        "config": {"workload": "wan1.3b single layer: 12 heads x 128, 4680 chunk queries, 1560 sink + 4680 "
+                               "current + 18720 history keys; warm-up statistics over one chunk per step; "
+                               "absorb D=1536",
+                   "l2": "inputs larger than L2 (153 MB of K/V read per attention pass)",
+                   "parallelism": f"replicas x{world}"},
+        "absorb_ms_per_layer": round(float(mean[3]), 4),
+        "chunk_latency_ms": {"l_layer": round(float(mean[4]), 4),
+                             "f_layer": round(float(mean[5] + mean[6]), 4),
+                             "warmup_f_layer": round(float(mean[0] + mean[1] + mean[2]), 4)},
+        "components_ms": {"dual_attention": round(float(mean[0]), 4), "warmup_projection": round(float(mean[1]), 4),
+                          "gram_accumulate": round(float(mean[2]), 4), "absorb_solve": round(float(mean[3]), 4),
+                          "local_attention_project": round(float(mean[4]), 4),
+                          "full_attention": round(float(mean[5]), 4), "f_projection": round(float(mean[6]), 4)},
+        "components_rate": {
+            "dual_attention_tflops": round(achieved, 2),
+            "full_attention_tflops": round(F / (mean[5] * 1e-3) / 1e12, 2),
+            "gram_tflops": round(gram_flops(w, w.n_q) / (mean[2] * 1e-3) / 1e12, 2),
+            "projection_tflops": round(2.0 * w.n_q * D * D / (mean[1] * 1e-3) / 1e12, 2),
+            "lse_merge_gbs": round(merge_gbs, 1)},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tc_peak, 4), "traffic": traffic,
+                     "kernel": "dual_attention_kernel<128,3>", "peak_source": f"{src} bf16 burst",
+                     "frac_of_spec_2250": round(achieved / 2250.0, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+        "gpu_launches": args.steps * (7 + absorb_launches(D)),
+    }
+    return res
+
+
+def merge_bench(ispa, w, device, sets=4, iters=20) -> float:
+    H, D, n = w.n_heads, w.d_model, w.n_q
+    g = torch.Generator(device=device).manual_seed(0)
+    bufs = []
+    for _ in range(sets):
+        bufs.append({"o_loc": torch.randn(n, D, device=device, generator=g).to(torch.bfloat16),
+                     "o_hist": torch.randn(n, D, device=device, generator=g).to(torch.bfloat16),
+                     "l_loc": torch.randn(H, n, device=device, generator=g),
+                     "l_hist": torch.randn(H, n, device=device, generator=g),
+                     "out": {"a_full": torch.empty(n, D, dtype=torch.bfloat16, device=device),
+                             "a_delta": torch.empty(n, D, dtype=torch.bfloat16, device=device),
+                             "lse_full": torch.empty(H, n, device=device)}})
+    for b in bufs:
+        ispa.lse_merge(b["o_loc"], b["l_loc"], b["o_hist"], b["l_hist"], H, out=b["out"])
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(iters):
+        b = bufs[i % sets]
+        ispa.lse_merge(b["o_loc"], b["l_loc"], b["o_hist"], b["l_hist"], H, out=b["out"])
+    e1.record()
+    torch.cuda.synchronize(device)
+    nbytes = n * D * 2 * 4 + H * n * 4 * 3
+    return nbytes * iters / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        return json.load(f).get(kernel)
+
+
+# --------------------------------------------------------- CPU baseline
+def oracle_sample(rows: int):
+    """fp64 oracle dual-stream pass over `rows` query rows of the workload."""
+    from oracle import ispa_oracle as orc
+    w = synth.WORKLOADS[WORKLOAD]
+    x = synth.single_layer_inputs(w, 1)
+    loc = [(x["k_sink"], x["v_sink"]), (x["k_cur"], x["v_cur"])]
+    his = [(x["k_hist"], x["v_hist"])]
+    flops = attn_flops(w) * rows / w.n_q
+
+    def run():
+        orc.dual_stream(x["q"][:rows], loc, his, w.n_heads)
+    return run, flops
+
+
+def cpu_baseline(rows=256):
+    run, flops = oracle_sample(rows)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, {rows} of 4680 query rows of the wan1.3b chunk (local, history and "
+                      f"single-pass full attention), {dt:.2f} s"}
+
+
+def run_reference(args):
+    rows = 64
+    run, flops = oracle_sample(rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    v = flops * args.steps / dt / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded PCG64; Wan-1.3B latent shapes)",
+            "config": {"workload": "wan1.3b single layer dual-stream attention; each step a bounded sample of "
+                                   f"{rows} query rows", "parallelism": "none (host cores)"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+                             "sample": f"{rows} of 4680 query rows per step"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    from ar_video_diffusion_b200 import build as ispa_build
+    if rank == 0:
+        ispa_build.build()
+    if world > 1:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        torch.distributed.barrier()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for the GPU arm")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    res = run_ours(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,92 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/ispa.h declares, rejects bad arguments on the host before any launch,
+and its host bookkeeping matches the oracle bit for bit."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ar_video_diffusion_b200 import build as ispa_build
+from ar_video_diffusion_b200 import ispa
+from oracle import ispa_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    ispa_build.build()
+    return ispa.lib()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "ispa.h")).read()
+    return sorted(set(re.findall(r"ISPA_API\s+[\w\s\*]+?\b(ispa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_hot_path_entry_points():
+    names = _declared_symbols()
+    for n in ("ispa_dual_attention", "ispa_gram_accumulate", "ispa_absorb_solve", "ispa_local_attention_project"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared_symbols()
+    assert names, "no declarations found"
+    for n in names:
+        assert hasattr(L, n), f"{n} not exported"
+    assert set(names) == set(ispa.EXPORTED)
+
+
+def test_version_and_status_strings(L):
+    assert ispa.ispa_version() >= 100
+    assert ispa.ispa_status_string(0) == "ok"
+    assert "positive definite" in ispa.ispa_status_string(4)
+
+
+def test_host_validation_rejects_before_launch(L):
+    # NULL q -> invalid argument, no CUDA call needed
+    r = L.ispa_dual_attention(None, 10, 128, 1, 128, 0, 0.0, None, 0, None, 0, None, None, None, None, None, None,
+                              None)
+    assert r == 1 and "q is NULL" in L.ispa_last_error().decode()
+    # unsupported head_dim
+    r = L.ispa_dual_attention(ctypes.c_void_p(256), 10, 96, 1, 96, 0, 0.0, None, 0, None, 0, None, None, None, None,
+                              None, None, None)
+    assert r == 2
+    # unsupported dtype
+    r = L.ispa_gram_accumulate(None, None, 4, 128, 128, 7, None, None, 0, None)
+    assert r == 2
+    # workspace too small
+    r = L.ispa_absorb_solve(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 128, 0.0, 0.01,
+                            ctypes.c_void_p(256), None, ctypes.c_void_p(256), 16, None, None)
+    assert r == 6
+    # d_model not a multiple of 64
+    r = L.ispa_absorb_solve(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), 0, 100, 0.0, 0.01,
+                            ctypes.c_void_p(256), None, ctypes.c_void_p(256), 1 << 20, None, None)
+    assert r == 2
+    # misaligned projection input
+    r = L.ispa_project(ctypes.c_void_p(258), 4, 128, 128, 128, 0, ctypes.c_void_p(256), ctypes.c_void_p(256), None)
+    assert r == 1
+
+
+def test_workspace_size_formula(L):
+    for D in (64, 128, 1536, 5120):
+        assert ispa.ispa_absorb_workspace_bytes(D) >= 4 * D * D + 4 * 64 * D + 8
+
+
+@pytest.mark.parametrize("chunk", [0, 1, 2, 7, 23])
+def test_chunk_token_ranges_bit_exact(L, chunk):
+    for F, cf, sf in [(1560, 3, 1), (16, 4, 1), (7, 2, 2)]:
+        got = ispa.ispa_chunk_token_ranges(chunk, F, cf, sf)
+        assert got == orc.chunk_token_ranges(chunk, F, cf, sf)
+
+
+def test_kv_bytes_bit_exact(L):
+    mask = orc.layer_mask(30, range(0, 30, 2))
+    for chunk in range(24):
+        for trans in (False, True):
+            for m in (0, mask, (1 << 30) - 1):
+                assert ispa.ispa_kv_bytes(chunk, 30, m, trans, 1560, 3, 1536, 2) == \
+                    orc.kv_bytes(chunk, 30, m, trans, 1560, 3, 1536, 2)
+    assert ispa.ispa_kv_bytes(23, 30, mask, True, 1560, 3, 1536, 2) == 15 * 112320 * 6144 + 15 * 6240 * 6144
