@@ -30,8 +30,8 @@ MAX_SEGMENTS = 8
 
 # every symbol declared in include/ispa.h
 EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "ispa_absorb_workspace_bytes",
-            "ispa_absorb_solve", "ispa_project", "ispa_local_attention_project", "ispa_chunk_token_ranges",
-            "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
+            "ispa_absorb_solve", "ispa_absorb_solve_noalloc", "ispa_project", "ispa_local_attention_project",
+            "ispa_chunk_token_ranges", "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
             "ispa_version")
 
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "ispa_gram_accumulate": (i32, [vp, vp, i64, i64, i64, i32, vp, vp, i32, vp]),
             "ispa_absorb_workspace_bytes": (sz, [i64]),
             "ispa_absorb_solve": (i32, [vp, vp, vp, i32, i64, f64, f64, vp, vp, vp, sz, vp, vp]),
+            "ispa_absorb_solve_noalloc": (i32, [vp, vp, vp, i32, i64, f64, f64, vp, vp, vp, vp]),
             "ispa_project": (i32, [vp, i64, i64, i64, i64, i32, vp, vp, vp]),
             "ispa_local_attention_project": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp, vp,
                                                    vp]),
@@ -152,6 +153,11 @@ def ispa_absorb_solve(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w
                       dev_status, stream):
     _check(lib().ispa_absorb_solve(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, workspace,
                                    workspace_bytes, dev_status, stream), "ispa_absorb_solve")
+
+
+def ispa_absorb_solve_noalloc(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, dev_status, stream):
+    _check(lib().ispa_absorb_solve_noalloc(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new,
+                                           dev_status, stream), "ispa_absorb_solve_noalloc")
 
 
 def ispa_project(a, n_rows, d_in, d_out, a_stride, dt, w, y, stream):

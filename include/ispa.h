@@ -155,6 +155,32 @@ ISPA_API ispa_status_t ispa_absorb_solve(const float* G, const float* R, const v
                                 size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * ispa_absorb_solve_noalloc -- the same solve as ispa_absorb_solve, for callers
+ * that cannot allocate device memory.  The ISPA method has no counterpart of
+ * this call; it exists for deployment: code running inside a host callback or
+ * an allocator hook, a plugin that receives device pointers but no allocator,
+ * or a serving process whose device memory is fixed before it starts cannot
+ * call cudaMalloc, so it cannot provide the workspace ispa_absorb_solve needs.
+ * Here the working matrices live in a device array owned by the library
+ * (4 d^2 + 256 d + 256 bytes for d = 2048, about 17.3 MB), which every GPU that
+ * loads libispa holds until the process exits.  The caller still passes G, R,
+ * W and the outputs, exactly as for ispa_absorb_solve.
+ *   - d_model must be a multiple of 64 and at most 2048; larger sizes return
+ *     ISPA_ERR_UNSUPPORTED without launching.
+ *   - No allocation of any kind happens, and nothing needs clearing: each call
+ *     writes every working value before reading it.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array: calls whose executions overlap
+ *     on the GPU (different streams without ordering between them) race and
+ *     give undefined results.  Calls on one stream are safe.
+ */
+ISPA_API ispa_status_t ispa_absorb_solve_noalloc(const float* G, const float* R, const void* W, ispa_dtype_t w_dt,
+                                                 int64_t d_model, double lambda_abs, double lambda_rel,
+                                                 float* delta_w, void* w_new, int32_t* dev_status, void* stream);
+
+/*
  * ispa_project -- y = a @ w for one layer's output projection (the warm-up and
  * F-layer output, and the second half of ispa_local_attention_project).
  * a [n_rows, d_in] (row stride a_stride elements), w [d_in, d_out] row-major,
