@@ -134,22 +134,38 @@ __global__ void shift_kernel(const float* __restrict__ G, float* __restrict__ M,
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     float4 g = reinterpret_cast<const float4*>(G)[e];
     const int64_t i = (e * 4) / D, j0 = (e * 4) % D;
-    if (i >= j0 && i < j0 + 4) (&g.x)[i - j0] += l;
+    const int64_t off = i - j0;  // position of the diagonal inside this float4, if any
+    g.x += off == 0 ? l : 0.f;
+    g.y += off == 1 ? l : 0.f;
+    g.z += off == 2 ? l : 0.f;
+    g.w += off == 3 ? l : 0.f;
     reinterpret_cast<float4*>(M)[e] = g;
   }
 }
 
 // Factor the 64 x 64 diagonal block k of M in place (lower triangle) and
 // write the inverse of its Cholesky factor to Linv (64 x 64, row-major).
+// Column-by-column: at step j the pivot is square-rooted, column j of L is
+// scaled, the trailing lower triangle gets the rank-1 update, and the same
+// elimination is applied to X (initially I), which ends as L^-1.  Thread t owns
+// column t % 64 of rows t / 64 + 4 a, a = 0..15.
 __global__ void __launch_bounds__(256) potrf_diag_kernel(float* M, int D, int k, float* Linv, int32_t* status) {
   __shared__ float A[kT][kT + 1];
   __shared__ float X[kT][kT + 1];
+  __shared__ float s_inv;
   __shared__ int bad;
   const int tid = threadIdx.x;
+  const int c = tid & 63, r0 = tid >> 6;
   float* blk = M + (int64_t)k * kT * D + (int64_t)k * kT;
-  for (int e = tid; e < kT * kT; e += 256) A[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
+#pragma unroll
+  for (int a = 0; a < 16; ++a) {
+    const int i = r0 + 4 * a;
+    A[i][c] = blk[(int64_t)i * D + c];
+    X[i][c] = (i == c) ? 1.f : 0.f;
+  }
   if (tid == 0) bad = -1;
   __syncthreads();
+#pragma unroll 1
   for (int j = 0; j < kT; ++j) {
     if (tid == 0) {
       float d = A[j][j];
@@ -157,40 +173,62 @@ __global__ void __launch_bounds__(256) potrf_diag_kernel(float* M, int D, int k,
         if (bad < 0) bad = j;
         d = 1.f;
       }
-      A[j][j] = sqrtf(d);
+      const float sq = sqrtf(d);
+      A[j][j] = sq;
+      s_inv = 1.0f / sq;
     }
     __syncthreads();
-    const float inv = 1.0f / A[j][j];
-    for (int i = j + 1 + tid; i < kT; i += 256) A[i][j] *= inv;
+    const float inv = s_inv;
+    if (tid < kT) {
+      if (tid > j) A[tid][j] *= inv;
+      X[j][tid] *= inv;
+    }
     __syncthreads();
-    const int n = kT - 1 - j;
-    for (int e = tid; e < n * n; e += 256) {
-      const int i = j + 1 + e / n, c = j + 1 + e % n;
-      if (c <= i) A[i][c] -= A[i][j] * A[c][j];
+    const float acj = A[c][j];
+    const float xjc = X[j][c];
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+      const int i = r0 + 4 * a;
+      if (i > j) {
+        const float aij = A[i][j];
+        if (c > j && c <= i) A[i][c] -= aij * acj;
+        X[i][c] -= aij * xjc;
+      }
     }
     __syncthreads();
   }
   if (tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = k * kT + bad;
   }
-  // inverse of the lower-triangular factor, one column per thread
-  if (tid < kT) {
-    const int c = tid;
-    for (int i = 0; i < kT; ++i) {
-      if (i < c) {
-        X[i][c] = 0.f;
-        continue;
-      }
-      float s = (i == c) ? 1.f : 0.f;
-      for (int t = c; t < i; ++t) s -= A[i][t] * X[t][c];
-      X[i][c] = s / A[i][i];
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < kT * kT; e += 256) {
-    const int i = e / kT, c = e % kT;
+#pragma unroll
+  for (int a = 0; a < 16; ++a) {
+    const int i = r0 + 4 * a;
     if (c <= i) blk[(int64_t)i * D + c] = A[i][c];
-    Linv[e] = X[i][c];
+    Linv[i * kT + c] = X[i][c];
+  }
+}
+
+// 64 x 64 x 64 product out = P Q (with P or Q read transposed), register
+// tiled: thread (ty, tx) of 16 x 16 owns rows ty + 16 a, columns tx + 16 b.
+// pt: P is given transposed (P(i, t) = Ps[t][i]); qt: Q(t, c) = Qs[c][t].
+__device__ __forceinline__ void mm64(const float (*Ps)[kT + 1], const float (*Qs)[kT + 1], bool pt, bool qt,
+                                     float (&acc)[4][4]) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 8
+  for (int t = 0; t < kT; ++t) {
+    float pa[4], qb[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) pa[a] = pt ? Ps[t][ty + 16 * a] : Ps[ty + 16 * a][t];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) qb[b] = qt ? Qs[tx + 16 * b][t] : Qs[t][tx + 16 * b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(pa[a], qb[b], acc[a][b]);
   }
 }
 
@@ -205,12 +243,13 @@ __global__ void __launch_bounds__(256) panel_kernel(float* M, int D, int k, cons
     P[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kT * kT; e += 256) {
-    const int i = e / kT, c = e % kT;
-    float s = 0.f;
-    for (int t = 0; t <= c; ++t) s = fmaf(P[i][t], Li[c][t], s);
-    blk[(int64_t)i * D + c] = s;
-  }
+  float acc[4][4];
+  mm64(P, Li, false, true, acc);
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) blk[(int64_t)(ty + 16 * a) * D + tx + 16 * b] = acc[a][b];
 }
 
 // X[k-block rows, :] <- Linv_k X  (transpose_l = 0) or Linv_k^T X (1), in place;
@@ -225,16 +264,14 @@ __global__ void __launch_bounds__(256) diag_apply_kernel(float* X, int D, int k,
     T[e / kT][e % kT] = blk[(int64_t)(e / kT) * D + e % kT];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kT * kT; e += 256) {
-    const int i = e / kT, c = e % kT;
-    float s = 0.f;
-    if (!transpose_l) {
-      for (int t = 0; t <= i; ++t) s = fmaf(Li[i][t], T[t][c], s);
-    } else {
-      for (int t = i; t < kT; ++t) s = fmaf(Li[t][i], T[t][c], s);
-    }
-    blk[(int64_t)i * D + c] = s;
-  }
+  float acc[4][4];
+  mm64(Li, T, transpose_l != 0, false, acc);
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) blk[(int64_t)(ty + 16 * a) * D + tx + 16 * b] = acc[a][b];
 }
 
 template <typename TW>

@@ -4,7 +4,9 @@
 
 #include <cstdarg>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "internal.h"
 
@@ -81,11 +83,22 @@ bool encode_map_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint
 }
 
 ispa_status_t set_smem(const void* kernel, int bytes) {
+  // The attribute is per device; set it once per (kernel, device) so later
+  // calls (including calls made while a stream is being captured) skip it.
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(kernel, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return ISPA_OK;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(%d bytes of shared memory): %s", bytes, cudaGetErrorString(e));
     return ISPA_ERR_CUDA;
   }
+  done[key] = bytes;
   return ISPA_OK;
 }
 

@@ -194,3 +194,47 @@ def random_case(seed: int, n_q: int, n_heads: int, head_dim: int, seg_tokens: Li
         v = g.standard_normal((n, D), dtype=np.float32)
         segs.append((_store(k, dtype), _store(v, dtype)))
     return {"q": q, "segments": segs}
+
+
+# ----------------------------------------------------------------------------
+# Device-side generator for the streaming rollout: the same recipe (noise plus
+# a rank-4 per-frame key component, W ~ N(0, 1/D)) drawn with torch's CUDA RNG
+# so that thousands of frames are produced in milliseconds.  Each tensor is
+# seeded from the same (seed, layer, key, tensor_id) tuple as the host recipe;
+# the values differ from the host generator's but are fixed by the seed.
+def _seed_int(seed: int, layer: int, key: int, tensor_id: int) -> int:
+    s = np.random.SeedSequence([seed, layer, key, tensor_id]).generate_state(2, dtype=np.uint32)
+    return (int(s[0]) << 31) ^ int(s[1])
+
+
+def _randn_device(shape, seed_int: int, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed_int)
+    return torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+
+
+def frame_kv_device(w: Workload, layer: int, frame: int, device):
+    """K and V of one latent frame on `device`, bf16 [frame_tokens, D]."""
+    import torch
+    F, H, d = w.frame_tokens, w.n_heads, w.head_dim
+    noise = _randn_device((F, H * d), _seed_int(w.seed, layer, frame, _T_K_NOISE), device)
+    coef = _randn_device((F, RANK), _seed_int(w.seed, layer, frame, _T_K_COEF), device)
+    basis = _randn_device((H, RANK, d), _seed_int(w.seed, layer, frame, _T_K_BASIS), device)
+    shared = (coef @ basis.reshape(H, RANK, d).permute(1, 0, 2).reshape(RANK, H * d))
+    k = noise + RANK_SCALE * shared
+    v = _randn_device((F, H * d), _seed_int(w.seed, layer, frame, _T_V), device)
+    return k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def chunk_q_device(w: Workload, layer: int, chunk: int, device):
+    import torch
+    q = _randn_device((w.n_q, w.d_model), _seed_int(w.seed, layer, chunk, _T_Q), device)
+    return q.to(torch.bfloat16)
+
+
+def weight_device(w: Workload, layer: int, device):
+    import torch
+    D = w.d_model
+    W = _randn_device((D, D), _seed_int(w.seed, layer, 0, _T_W), device) / float(np.sqrt(D))
+    return W.to(torch.bfloat16)

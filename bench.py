@@ -155,28 +155,42 @@ def run_ours(args, rank, world, device):
     ispa.dual_attention(q, local, hist, H, out=dual_out, status=status)
     ispa.gram_accumulate(dual_out["a_loc"], dual_out["a_delta"], G, R, zero_first=True)
 
-    n_ev = 8
-    def step(evs):
-        evs[0].record(stream)
-        ispa.dual_attention(q, local, hist, H, out=dual_out, status=status)
-        evs[1].record(stream)
-        ispa.project(dual_out["a_full"], W, y_warm)
-        evs[2].record(stream)
-        ispa.gram_accumulate(dual_out["a_loc"], dual_out["a_delta"], G, R)
-        evs[3].record(stream)
-        ispa.absorb_solve(G, R, W, lambda_rel=1e-2, workspace=ws, status=status, delta_w=dW, w_new=Wn)
-        evs[4].record(stream)
-        ispa.local_attention_project(q, local, Wn, H, y=y_l, a_loc=a_l, status=status)
-        evs[5].record(stream)
-        ispa.dual_attention(q, local, hist, H, dual=False, out=f_out, status=status)
-        evs[6].record(stream)
-        ispa.project(f_out["a_full"], W, y_f)
-        evs[7].record(stream)
+    comps = [
+        ("dual_attention", lambda: ispa.dual_attention(q, local, hist, H, out=dual_out, status=status)),
+        ("warmup_projection", lambda: ispa.project(dual_out["a_full"], W, y_warm)),
+        ("gram_accumulate", lambda: ispa.gram_accumulate(dual_out["a_loc"], dual_out["a_delta"], G, R)),
+        ("absorb_solve", lambda: ispa.absorb_solve(G, R, W, lambda_rel=1e-2, workspace=ws, status=status,
+                                                   delta_w=dW, w_new=Wn)),
+        ("local_attention_project", lambda: ispa.local_attention_project(q, local, Wn, H, y=y_l, a_loc=a_l,
+                                                                         status=status)),
+        ("full_attention", lambda: ispa.dual_attention(q, local, hist, H, dual=False, out=f_out, status=status)),
+        ("f_projection", lambda: ispa.project(f_out["a_full"], W, y_f)),
+    ]
 
-    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.warmup + args.steps)]
-    for i in range(args.warmup):
-        step(all_evs[i])
+    def step():
+        for _, fn in comps:
+            fn()
+
+    # eager warm-up, then the launches of a step are captured into CUDA graphs
+    # (one graph for the whole step, one per component) so that the timings
+    # below hold device time only, without host launch gaps
+    for _ in range(args.warmup):
+        step()
     torch.cuda.synchronize(device)
+    side = torch.cuda.Stream(device)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=side, capture_error_mode="relaxed"):
+        step()
+    g_comp = []
+    for name, fn in comps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+            fn()
+        g_comp.append((name, g))
+    for _ in range(args.warmup):
+        g_step.replay()
+    torch.cuda.synchronize(device)
+
     if world > 1:
         torch.distributed.barrier()
     clocks = ClockSampler(device.index if device.index is not None else 0)
@@ -188,22 +202,32 @@ def run_ours(args, rank, world, device):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.warmup, args.warmup + args.steps):
-        step(all_evs[i])
+    for _ in range(args.steps):
+        g_step.replay()
     t_end.record(stream)
     torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
+    # per-component device time: K back-to-back replays of a graph holding
+    # only that component's launches
+    comp_ms = {}
+    for name, g in g_comp:
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        comp_ms[name] = e0.elapsed_time(e1) / args.steps
     clk = clocks.stop()
     code = int(status[0].item())
     if code != 0:
         raise RuntimeError(f"device status {ispa.STATUS_NAMES.get(code, code)} during the benchmark")
 
     total_ms = t_start.elapsed_time(t_end)
-    parts = np.array([[all_evs[i][j].elapsed_time(all_evs[i][j + 1]) for j in range(n_ev - 1)]
-                      for i in range(args.warmup, args.warmup + args.steps)])
-    mean = parts.mean(axis=0)  # ms per component
-    t_dual = float(parts[:, 0].sum())
+    mean = [comp_ms[n] for n, _ in comps]  # ms per component
+    t_dual = comp_ms["dual_attention"] * args.steps
     # max over ranks of the time that defines `value`, and of the step time
     vals = torch.tensor([t_dual, total_ms], dtype=torch.float64, device=device)
     if world > 1:
@@ -249,6 +273,8 @@ def run_ours(args, rank, world, device):
     # standalone LSE merge over rotating buffer sets larger than L2
     merge_gbs = merge_bench(ispa, w, device)
 
+    rollout = None if args.no_rollout else run_rollout(device)
+
     pk, src = peaks()
     tc_peak = pk["bf16_tflops"]
     achieved = F / (t_dual / args.steps * 1e-3) / 1e12
@@ -270,6 +296,8 @@ def run_ours(args, rank, world, device):
                                "current + 18720 history keys; warm-up statistics over one chunk per step; "
                                "absorb D=1536",
                    "l2": "inputs larger than L2 (153 MB of K/V read per attention pass)",
+                   "timing": "CUDA-graph replays: a step graph for ms_per_step, one graph per component for the "
+                             "breakdown and the value",
                    "parallelism": f"replicas x{world}"},
         "absorb_ms_per_layer": round(float(mean[3]), 4),
         "chunk_latency_ms": {"l_layer": round(float(mean[4]), 4),
@@ -293,7 +321,93 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": d2h},
         "clocks": clk,
         "gpu_launches": args.steps * (7 + absorb_launches(D)),
+        "rollout": rollout,
     }
+    return res
+
+
+def run_profile_case(op: str, reps: int, device):
+    """One op of the hot path on the wan1.3b shapes, `reps` times back to back."""
+    from ar_video_diffusion_b200 import ispa
+    w = synth.WORKLOADS[WORKLOAD]
+    H, D, n = w.n_heads, w.d_model, w.n_q
+    x = synth.single_layer_inputs(w, 1)
+
+    def t(a):
+        return torch.from_numpy(a).to(torch.bfloat16).to(device)
+
+    q, ks, vs, kc, vc, kh, vh = (t(x[k]) for k in ("q", "k_sink", "v_sink", "k_cur", "v_cur", "k_hist", "v_hist"))
+    W = t(synth.weight(w, 0))
+    local, hist = [(ks, vs), (kc, vc)], [(kh, vh)]
+    status = ispa.new_status(device)
+    # set-up launches are issued only for the ops that need them, so that an
+    # ncu capture with "-s 1" skips exactly the first launch of the loop below
+    out = G = R = o_hist = None
+    if op in ("gram", "absorb", "project", "merge"):
+        out = ispa.dual_attention(q, local, hist, H, status=status)
+    if op in ("gram", "absorb"):
+        G, R = torch.empty(D, D, device=device), torch.empty(D, D, device=device)
+        ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=True)
+    if op == "merge":
+        o_hist = ispa.dual_attention(q, [], hist, H, dual=False, status=status)
+    if op == "dual":
+        out = {"a_loc": torch.empty(n, D, dtype=torch.bfloat16, device=device),
+               "a_full": torch.empty(n, D, dtype=torch.bfloat16, device=device),
+               "a_delta": torch.empty(n, D, dtype=torch.bfloat16, device=device),
+               "lse_loc": torch.empty(H, n, device=device), "lse_full": torch.empty(H, n, device=device)}
+    torch.cuda.synchronize(device)
+    for _ in range(reps):
+        if op == "dual":
+            ispa.dual_attention(q, local, hist, H, out=out, status=status)
+        elif op == "full":
+            ispa.dual_attention(q, local, hist, H, dual=False, status=status)
+        elif op == "local":
+            ispa.local_attention_project(q, local, W, H, status=status)
+        elif op == "gram":
+            ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R)
+        elif op == "project":
+            ispa.project(out["a_full"], W)
+        elif op == "merge":
+            ispa.lse_merge(out["a_loc"], out["lse_loc"], o_hist["a_full"], o_hist["lse_full"], H)
+        elif op == "absorb":
+            ispa.absorb_solve(G, R, W, status=status)
+    torch.cuda.synchronize(device)
+    if int(status[0].item()) != 0:
+        raise RuntimeError(f"device status {int(status[0].item())}")
+    print(f"profile case {op} x{reps} done")
+
+
+def run_rollout(device) -> dict:
+    """30-layer streaming rollout, 1.3B shapes: 4 warm-up chunks with every
+    layer dual-stream (the even layers accumulating statistics), absorb +
+    eviction of the 15 even layers, then 20 chunks with L-/F-layers."""
+    from ar_video_diffusion_b200.rollout import Rollout
+    w = synth.WORKLOADS["rollout"]
+    ro = Rollout(w, device=device)
+    reps = ro.run()
+    post = [r for r in reps if r.phase == "post"]
+    warm = [r for r in reps if r.phase == "warmup"]
+    last = reps[-1]
+    flops_last = 0.0
+    F_tok = w.frame_tokens
+    n_k_f = (last.chunk + 1) * w.n_q
+    for l in range(w.n_layers):
+        n_k = (w.sink_frames * F_tok + w.n_q) if l in ro.absorbed else n_k_f
+        flops_last += 4.0 * w.n_q * n_k * w.head_dim * w.n_heads + 2.0 * w.n_q * w.d_model ** 2
+    res = {
+        "workload": "rollout: 30 layers, 1.3B shapes, 4 warm-up + 20 post-transition chunks, even layers absorbed",
+        "chunk_ms": [round(r.gpu_ms, 3) for r in reps],
+        "warmup_chunk_ms_mean": round(sum(r.gpu_ms for r in warm) / len(warm), 3),
+        "post_chunk_ms_first": round(post[0].gpu_ms, 3),
+        "post_chunk_ms_last": round(post[-1].gpu_ms, 3),
+        "last_chunk_tflops": round(flops_last / (last.gpu_ms * 1e-3) / 1e12, 1),
+        "absorb_ms_per_layer": round(sum(ro.absorb_ms) / len(ro.absorb_ms), 4),
+        "kv_bytes_last": last.kv_bytes,
+        "kv_bytes_all_f_last": last.kv_bytes_all_f,
+        "kv_removed_frac": round(1 - last.kv_bytes / last.kv_bytes_all_f, 4),
+    }
+    del ro
+    torch.cuda.empty_cache()
     return res
 
 
@@ -385,6 +499,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer streaming rollout")
+    ap.add_argument("--profile", choices=["dual", "full", "local", "gram", "project", "merge", "absorb"],
+                    help="run only this op --steps times on the wan1.3b shapes (for ncu captures), no timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -408,6 +525,9 @@ def main():
         raise SystemExit("bench.py needs a CUDA device for the GPU arm")
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
+    if args.profile:
+        run_profile_case(args.profile, args.steps, device)
+        return
     res = run_ours(args, rank, world, device)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:

@@ -279,3 +279,88 @@ def test_local_attention_project_matches_oracle():
     a_ref, _ = orc.attention(case["q"], np.concatenate([ks, kc]), np.concatenate([vs, vc]), 2)
     assert max_rel(host(a_loc), a_ref) <= ATTN_MAX_REL
     assert max_rel(host(y), orc.project(a_ref, Wn)) <= ATTN_MAX_REL
+
+
+def _layer_outputs(w, chunk=1):
+    x = synth.single_layer_inputs(w, chunk)
+    status = ispa.new_status()
+    out = ispa.dual_attention(dev(x["q"], "bf16"), [(dev(x["k_sink"], "bf16"), dev(x["v_sink"], "bf16")),
+                                                   (dev(x["k_cur"], "bf16"), dev(x["v_cur"], "bf16"))],
+                              [(dev(x["k_hist"], "bf16"), dev(x["v_hist"], "bf16"))], w.n_heads, status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "dual_attention")
+    return x, out
+
+
+def _check_sampled_rows(w, x, out, n_rows, seed):
+    rows = np.sort(np.random.default_rng(seed).choice(w.n_q, n_rows, replace=False))
+    rows[-1] = w.n_q - 1
+    got = {k: host(v) for k, v in out.items()}
+    ref = orc.dual_stream(x["q"][rows], [(x["k_sink"], x["v_sink"]), (x["k_cur"], x["v_cur"])],
+                          [(x["k_hist"], x["v_hist"])], w.n_heads)
+    _check_dual(got, ref, rows=rows)
+
+
+def _check_gram_entries(A, Dl, G, R, n_pairs, seed):
+    """G[i, j] and R[i, j] at seeded (i, j), each an fp64 dot product over all
+    rows.  The products of bf16 values are exact in fp32, so the only error is
+    the fp32 summation: bounded here by GRAM_REL times the sum of |products|."""
+    g = np.random.default_rng(seed)
+    D = A.shape[1]
+    ii, jj = g.integers(0, D, n_pairs), g.integers(0, D, n_pairs)
+    Ah = A.float().cpu().numpy().astype(np.float64)
+    Dh = Dl.float().cpu().numpy().astype(np.float64)
+    Gh, Rh = G.cpu().numpy(), R.cpu().numpy()
+    for i, j in zip(ii, jj):
+        pg, pr = Ah[:, i] * Ah[:, j], Ah[:, i] * Dh[:, j]
+        assert abs(Gh[i, j] - pg.sum()) <= GRAM_REL * np.abs(pg).sum() + 1e-30
+        assert abs(Rh[i, j] - pr.sum()) <= GRAM_REL * np.abs(pr).sum() + 1e-30
+
+
+def test_long_history_layer_sampled_rows_and_gram():
+    """Long-history stress: 93600 history tokens (60 latent frames); 128 query
+    rows against the oracle, and the statistics accumulated over 93600 rows
+    checked entry by entry."""
+    w = synth.WORKLOADS["long_hist"]
+    x, out = _layer_outputs(w)
+    _check_sampled_rows(w, x, out, 128, 21)
+    # statistics over 93600 rows: 20 chunks' worth of (A_loc, delta) rows
+    g = np.random.default_rng(22)
+    n = 93600
+    A = dev(synth.round_bf16((g.standard_normal((n, w.d_model)) * 0.2).astype(np.float32)), "bf16")
+    Dl = dev(synth.round_bf16((g.standard_normal((n, w.d_model)) * 0.05).astype(np.float32)), "bf16")
+    G = torch.empty(w.d_model, w.d_model, device="cuda")
+    R = torch.empty(w.d_model, w.d_model, device="cuda")
+    ispa.gram_accumulate(A, Dl, G, R, zero_first=True)
+    torch.cuda.synchronize()
+    _check_gram_entries(A, Dl, G, R, 64, 23)
+
+
+def test_wan14b_layer_sampled_rows_statistics_and_absorb():
+    """Wan-14B-shaped layer (40 heads, D = 5120): sampled attention rows, the
+    statistics of 4 warm-up chunks (18720 rows) entry by entry, and the
+    5120 x 5120 absorb solve against an fp64 solve of the same G, R."""
+    w = synth.WORKLOADS["wan14b"]
+    x, out = _layer_outputs(w)
+    _check_sampled_rows(w, x, out, 48, 31)
+    D = w.d_model
+    G = torch.empty(D, D, device="cuda")
+    R = torch.empty(D, D, device="cuda")
+    As, Ds = [], []
+    for c in range(w.warm_chunks):
+        if c != 1:
+            _, out = _layer_outputs(w, c)
+        ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=(c == 0))
+        As.append(out["a_loc"])
+        Ds.append(out["a_delta"])
+    torch.cuda.synchronize()
+    _check_gram_entries(torch.cat(As), torch.cat(Ds), G, R, 32, 32)
+    W = synth.weight(w, 0)
+    status = ispa.new_status()
+    dW, Wn = ispa.absorb_solve(G, R, dev(W, "bf16"), lambda_rel=orc.LAMBDA_REL, status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "absorb_solve")
+    Gh, Rh = host(G), host(R)
+    Gh = 0.5 * (Gh + Gh.T)  # the solve reads the lower triangle only
+    dW_ref = orc.absorb(Gh, Rh, W, orc.ridge_lambda(Gh))
+    assert fro_rel(host(dW), dW_ref) <= DW_REL_BF16
