@@ -278,7 +278,7 @@ def run_ours(args, rank, world, device):
     pk, src = peaks()
     tc_peak = pk["bf16_tflops"]
     achieved = F / (t_dual / args.steps * 1e-3) / 1e12
-    traffic = load_traffic("dual_attention_kernel")
+    traffic = load_traffic("dual_attention_kernel<128,3>")
     res = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -438,12 +438,22 @@ def merge_bench(ispa, w, device, sets=4, iters=20) -> float:
 
 
 def load_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of `kernel` from profiles/traffic.md, or None when
+    the kernel's source has changed since that capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
-    with open(p) as f:
-        return json.load(f).get(kernel)
+    for line in open(p):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) != 4 or cells[0] != kernel:
+            continue
+        src = os.path.join(ROOT, cells[1])
+        if not os.path.exists(src):
+            return None
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return int(cells[3]) if digest == cells[2] else None
+    return None
 
 
 # --------------------------------------------------------- CPU baseline
