@@ -40,6 +40,8 @@ constexpr int kThreads = 384;  // 12 warps
 constexpr int kMaxSeg = ISPA_MAX_SEGMENTS;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
+// bit j set: column pair j (mod 8) of a score row takes 2^x from exp2_fma2
+constexpr uint32_t kEmuPairs = 0x00u;
 
 struct Params {
   CUtensorMap q_map;
@@ -311,12 +313,15 @@ __device__ void softmax_slot(const Params& p, uint8_t* smem, int s, uint32_t tme
         for (int j = 0; j < 32; ++j)
           if (c * 32 + j >= valid) r[c][j] = __float_as_uint(-INFINITY);
     }
-    float mx = -INFINITY;
+    // row maximum: four independent three-input chains, then combined
+    float mc[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < 4; ++c) {
+      mc[c] = fmaxf(__uint_as_float(r[c][0]), __uint_as_float(r[c][1]));
 #pragma unroll
-      for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(r[c][j]));
-    const float m_tile = mx * sl2;
+      for (int j = 1; j < 16; ++j) mc[c] = fmax3(mc[c], __uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1]));
+    }
+    const float m_tile = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * sl2;
     if (fresh) {
       m_used = m_tile;
     } else if (__any_sync(0xffffffffu, m_tile > m_used + kRescaleLog2)) {
@@ -335,19 +340,32 @@ __device__ void softmax_slot(const Params& p, uint8_t* smem, int s, uint32_t tme
       tmem_wait_st();
       m_used = m_new;
     }
-    float sum = 0.f;
+    // P = 2^(s * scale_log2 - m): pairs of columns with packed fp32 math; a
+    // fixed quarter of the pairs evaluate 2^x on the FMA pipe (kEmuPairs) to
+    // relieve the MUFU pipe, the rest use ex2.approx.
+    const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_used, -m_used);
+    float2 sum2[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
+      sum2[c] = make_float2(0.f, 0.f);
       uint32_t pk[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(r[c][2 * j]), sl2, -m_used));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(r[c][2 * j + 1]), sl2, -m_used));
-        sum += p0 + p1;
-        pk[j] = pack_bf16x2(p0, p1);
+        const float2 x = ffma2(make_float2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1])), sc2, nm2);
+        float2 pv;
+        if (kEmuPairs & (1u << (j & 7))) {
+          pv = exp2_fma2(x);
+        } else {
+          pv.x = fast_exp2(x.x);
+          pv.y = fast_exp2(x.y);
+        }
+        sum2[c] = fadd2(sum2[c], pv);
+        pk[j] = pack_bf16x2(pv.x, pv.y);
       }
       tmem_st16(p_addr + 16 * c, pk);
     }
+    const float2 s01 = fadd2(sum2[0], sum2[1]), s23 = fadd2(sum2[2], sum2[3]);
+    const float sum = (s01.x + s01.y) + (s23.x + s23.y);
     tmem_wait_st();
     l += sum;
     tc_fence_before();

@@ -227,6 +227,56 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ----------------------------------------------------- packed fp32 math
+// sm_100 executes two fp32 lanes per instruction with the .f32x2 forms.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe, for two values at once.  Additive range reduction
+// x = n + f with n = rint(x), f in [-1/2, 1/2] (the integer is read off the
+// mantissa after adding 1.5 * 2^23), 2^f by a degree-4 polynomial whose
+// coefficients were fitted for this library by iteratively reweighted least
+// squares on Chebyshev nodes to minimise the relative error over [-1/2, 1/2]
+// (max 2.7e-6 evaluated in fp32), and 2^n added into the exponent field.
+// Inputs below -125 are clamped there (result ~2^-125, i.e. 0 for bf16 P).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
+  float2 p = ffma2(f, make_float2(0.0095701f, 0.0095701f), make_float2(0.05591786f, 0.05591786f));
+  p = ffma2(p, f, make_float2(0.24024744f, 0.24024744f));
+  p = ffma2(p, f, make_float2(0.6931218f, 0.6931218f));
+  p = ffma2(p, f, make_float2(0.9999993f, 0.9999993f));
+  const int nx = __float_as_int(t.x) - 0x4B400000;
+  const int ny = __float_as_int(t.y) - 0x4B400000;
+  return make_float2(__int_as_float(__float_as_int(p.x) + (nx << 23)),
+                     __int_as_float(__float_as_int(p.y) + (ny << 23)));
+}
+
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace ispa
