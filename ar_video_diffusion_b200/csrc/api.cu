@@ -8,10 +8,10 @@
 #include "sm100.cuh"
 
 namespace ispa {
-ispa_status_t dual_attention_bf16(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
-                                  float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
-                                  void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
-                                  int32_t* status, cudaStream_t stream);
+ispa_status_t dual_attention_bf16_db(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
+                                     float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
+                                     void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
+                                     int32_t* status, cudaStream_t stream);
 ispa_status_t dual_attention_f32(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
                                  float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
                                  void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
@@ -110,7 +110,7 @@ extern "C" ispa_status_t ispa_dual_attention(const void* q, int64_t n_q, int64_t
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)head_dim);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dt == ISPA_DT_BF16)
-    return dual_attention_bf16(q, n_q, q_stride, n_heads, head_dim, scale, segs, nl, nh, a_loc, a_full, a_delta,
+    return dual_attention_bf16_db(q, n_q, q_stride, n_heads, head_dim, scale, segs, nl, nh, a_loc, a_full, a_delta,
                                lse_loc, lse_full, dev_status, s);
   return dual_attention_f32(q, n_q, q_stride, n_heads, head_dim, scale, segs, nl, nh, a_loc, a_full, a_delta,
                             lse_loc, lse_full, s);
