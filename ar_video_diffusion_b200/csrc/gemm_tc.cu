@@ -5,13 +5,18 @@
 //  * the Layer-Absorb statistics [G | R] += A_loc^T [A_loc | A_full - A_loc]
 //    ("Instance-Specific Parametric Absorption", gist.science technical
 //    summary, section 2 stage 2): both operands are the token-major activation
-//    matrices read "MN-major" (the contraction runs over tokens, which is the
-//    row index of A_loc), so no transpose is ever materialised;
-//  * the output projection y = A W (stage 1 and stage 3 of the same section):
-//    A is K-major (token rows), W [D_in, D_out] is MN-major.
-// One CTA computes one 128 x BN tile: warp 0 issues TMA loads into an
-// NST-deep ring, warp 1 issues tcgen05.mma (M=128, N=BN, K=16), warp 2 owns
-// the tensor memory, warps 4-7 drain the accumulator (one row per thread).
+//    matrices read "MN-major" (the contraction runs over tokens, the row index
+//    of A_loc), so no transpose is ever materialised; only the tiles of G that
+//    touch its lower triangle are computed (G is symmetric and the solve reads
+//    its lower triangle), and the token range is split across CTAs whose
+//    partial sums are added into G, R with vector reductions in L2;
+//  * the output projection y = A W (stages 1 and 3 of the same section): A is
+//    K-major (token rows), W [D_in, D_out] is MN-major.
+// One CTA computes a 256 x BN tile as two 128-row halves that share every B
+// tile (two M=128 MMAs per K step), which halves the operand traffic per FLOP
+// against a 128-row tile: warp 0 issues TMA loads into an NST-deep ring,
+// warp 1 issues tcgen05.mma, warp 2 owns the 2*BN tensor-memory columns and
+// warps 4-11 drain the two accumulators (one row per thread).
 #include <cstring>
 
 #include "internal.h"
@@ -20,17 +25,19 @@
 namespace ispa {
 namespace gemm {
 
-constexpr int kBM = 128;
+constexpr int kBM = 256;  // two tensor-core M=128 halves
 constexpr int kBK = 64;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 
-enum Mode : int { kStoreBf16 = 0, kStoreF32 = 1, kAccumF32 = 2 };
+enum Mode : int { kStoreBf16 = 0, kStoreF32 = 1, kReduceF32 = 2 };
 
 struct Params {
   CUtensorMap a_map;
   CUtensorMap b_map[2];
   int32_t M, N, K;
-  int32_t n_split;  // columns [0, n_split) come from b_map[0] / c[0], the rest from b_map[1] / c[1]
+  int32_t n_split;      // columns [0, n_split) come from b_map[0] / c[0], the rest from b_map[1] / c[1]
+  int32_t lower_only0;  // skip tiles of the first column range that lie strictly above the diagonal
+  int32_t k_per_split;  // K rows per blockIdx.z, a multiple of kBK
   void* c[2];
   int64_t ldc;
   int32_t mode;
@@ -39,7 +46,7 @@ struct Params {
 
 template <int BN, int NST>
 struct Layout {
-  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kABytes = kBM * kBK * 2;  // 32 KB
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBars = NST * kStage;
@@ -49,9 +56,25 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 template <bool A_MN, bool B_MN, int BN, int NST>
 __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_constant__ Params p) {
   using L = Layout<BN, NST>;
+  const int n0g = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int half_n = n0g >= p.n_split ? 1 : 0;
+  const int n0 = n0g - half_n * p.n_split;
+  // whole-CTA early exit (before any barrier or tensor-memory use): a tile of
+  // a lower-triangular output that lies strictly above the diagonal
+  if (half_n == 0 && p.lower_only0 && n0 > m0 + kBM - 1) return;
+  const int k_begin = blockIdx.z * p.k_per_split;
+  const int k_end = min(p.K, k_begin + p.k_per_split);
+  if (k_begin >= k_end) return;
+  const int nk = (k_end - k_begin + kBK - 1) / kBK;
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);
@@ -60,12 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   uint64_t* teardown = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0g = blockIdx.x * BN, m0 = blockIdx.y * kBM;
-  const int half = n0g >= p.n_split ? 1 : 0;
-  const int n0 = n0g - half * p.n_split;
-  const int nk = (p.K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
@@ -78,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
     fence_barrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -88,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA
-    const CUtensorMap* bm = &p.b_map[half];
+    const CUtensorMap* bm = &p.b_map[half_n];
     tma_prefetch_desc(&p.a_map);
     tma_prefetch_desc(bm);
     int kb = 0;
@@ -97,11 +115,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
       if (kb >= NST && !mbar_wait(&empty[stage], ((kb / NST) - 1) & 1, abort_flag)) break;
       uint8_t* sa = smem + stage * L::kStage;
       uint8_t* sb = sa + L::kABytes;
-      const int k0 = kb * kBK;
+      const int k0 = k_begin + kb * kBK;
       mbar_arrive_expect_tx(&full[stage], L::kStage);
       if (A_MN) {
-        tma_load_2d(sa, &p.a_map, &full[stage], m0, k0);
-        tma_load_2d(sa + 8192, &p.a_map, &full[stage], m0 + 64, k0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_load_2d(sa + c * 8192, &p.a_map, &full[stage], m0 + 64 * c, k0);
       } else {
         tma_load_2d(sa, &p.a_map, &full[stage], k0, m0);
       }
@@ -118,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
-    constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN, A_MN, B_MN);
     const uint32_t base = smem_u32(smem);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -132,9 +150,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
       const uint32_t sb = sa + L::kABytes;
 #pragma unroll
       for (int kk = 0; kk < kBK / 16; ++kk) {
-        const uint64_t da = A_MN ? sdesc_sw128(sa + kk * 2048, 8192, 1024) : sdesc_sw128(sa + kk * 32, 16, 1024);
         const uint64_t db = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
-        umma_ss(tmem, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // rows 128h..128h+127 of the A tile: MN-major blocks 2h, 2h+1 / K-major rows
+          const uint64_t da = A_MN ? sdesc_sw128(sa + h * 16384 + kk * 2048, 8192, 1024)
+                                   : sdesc_sw128(sa + h * 16384 + kk * 32, 16, 1024);
+          umma_ss(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
       }
       umma_commit(&empty[stage]);
     }
@@ -143,14 +166,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
     mbar_wait_drain(teardown, 0, 100000000ull);
   } else if (warp >= 4) {
     // ----------------------------------------------------------- epilogue
+    const int h = (warp - 4) >> 2;
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const int gm = m0 + row;
-    bool ok = __all_sync(0xffffffffu, nk == 0 ? true : mbar_wait(acc_full, 0, abort_flag));
+    const int gm = m0 + h * 128 + wq * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag));
     if (ok) {
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16);
-      const int n_cols = p.n_split < p.N ? (half ? p.N - p.n_split : p.n_split) : p.N;
+      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
+      const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -159,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
         const int gn = n0 + 32 * c;
         if (gm >= p.M || gn >= n_cols) continue;
         if (p.mode == kStoreBf16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c[half]) + (int64_t)gm * p.ldc + gn);
+          uint4* dst =
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c[half_n]) + (int64_t)gm * p.ldc + gn);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 u;
@@ -170,19 +194,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
             dst[v] = u;
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c[half]) + (int64_t)gm * p.ldc + gn);
+          float* dst = static_cast<float*>(p.c[half_n]) + (int64_t)gm * p.ldc + gn;
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            float4 x = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-            if (p.mode == kAccumF32) {
-              const float4 o = dst[v];
-              x.x += o.x;
-              x.y += o.y;
-              x.z += o.z;
-              x.w += o.w;
-            }
-            dst[v] = x;
+            const float a = __uint_as_float(r[4 * v]), b = __uint_as_float(r[4 * v + 1]);
+            const float c2 = __uint_as_float(r[4 * v + 2]), d = __uint_as_float(r[4 * v + 3]);
+            if (p.mode == kReduceF32)
+              red_add_v4(dst + 4 * v, a, b, c2, d);
+            else
+              reinterpret_cast<float4*>(dst)[v] = make_float4(a, b, c2, d);
           }
         }
       }
@@ -192,24 +212,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, BN);
+  if (warp == 2) tmem_dealloc(tmem, 2 * BN);
   if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
 }
 
 template <bool A_MN, bool B_MN, int BN, int NST>
-static ispa_status_t launch(const Params& p, cudaStream_t stream) {
+static ispa_status_t launch(const Params& p, int k_splits, cudaStream_t stream) {
   using L = Layout<BN, NST>;
   auto kern = gemm_bf16_kernel<A_MN, B_MN, BN, NST>;
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
-  dim3 grid(p.N / BN, (p.M + kBM - 1) / kBM);
+  dim3 grid(p.N / BN, (p.M + kBM - 1) / kBM, k_splits);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
   return check_launch("gemm_bf16_kernel");
 }
 
 }  // namespace gemm
 
-// [G | R] (+)= A_loc^T [A_loc | delta]  (bf16 inputs, fp32 outputs).
+// [G | R] (+)= A_loc^T [A_loc | delta]  (bf16 inputs, fp32 outputs).  Only the
+// lower triangle of G (and all of R) is produced; the K range (rows) is split
+// across CTAs so that the launch fills the GPU, and the partial products are
+// added into G, R in L2 (they are zeroed first when `overwrite`).
 ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, int64_t D, int64_t row_stride,
                         float* G, float* R, bool overwrite, cudaStream_t stream) {
   using namespace gemm;
@@ -219,16 +242,35 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   if (!encode_map_bf16_2d(&p.a_map, a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&p.b_map[0], a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&p.b_map[1], a_delta, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  if (overwrite) {
+    cudaMemsetAsync(G, 0, (size_t)D * D * 4, stream);
+    cudaMemsetAsync(R, 0, (size_t)D * D * 4, stream);
+  }
   p.M = (int32_t)D;
   p.N = (int32_t)(2 * D);
   p.K = (int32_t)n_rows;
   p.n_split = (int32_t)D;
+  p.lower_only0 = 1;
   p.c[0] = G;
   p.c[1] = R;
   p.ldc = D;
-  p.mode = overwrite ? kStoreF32 : kAccumF32;
-  if (D % 256 == 0) return launch<true, true, 256, 4>(p, stream);
-  return launch<true, true, 128, 6>(p, stream);
+  p.mode = kReduceF32;
+  const int BN = D % 256 == 0 ? 256 : 128;
+  const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
+  int64_t tiles = m_tiles * n_tiles;  // R
+  for (int64_t i = 0; i < m_tiles; ++i)
+    for (int64_t j = 0; j < n_tiles; ++j) tiles += (j * BN <= i * kBM + kBM - 1) ? 1 : 0;  // lower part of G
+  const int64_t k_blocks = (n_rows + kBK - 1) / kBK;
+  const int sms = num_sms();
+  // one CTA per SM: the largest split count that still fits in one wave
+  int64_t splits = sms / tiles;
+  if (splits > k_blocks / 8) splits = k_blocks / 8;  // keep at least 8 K steps per CTA
+  if (splits < 1) splits = 1;
+  const int64_t blocks_per_split = (k_blocks + splits - 1) / splits;
+  p.k_per_split = (int32_t)(blocks_per_split * kBK);
+  splits = (k_blocks + blocks_per_split - 1) / blocks_per_split;
+  if (BN == 256) return launch<true, true, 256, 3>(p, (int)splits, stream);
+  return launch<true, true, 128, 4>(p, (int)splits, stream);
 }
 
 // y[n_rows, d_out] = a[n_rows, d_in] * w[d_in, d_out]  (bf16 in/out).
@@ -244,11 +286,13 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   p.N = (int32_t)d_out;
   p.K = (int32_t)d_in;
   p.n_split = (int32_t)d_out;
+  p.k_per_split = (int32_t)(((d_in + kBK - 1) / kBK) * kBK);
   p.c[0] = y;
   p.c[1] = y;
   p.ldc = d_out;
   p.mode = kStoreBf16;
-  if (d_out % 128 == 0) return launch<false, true, 128, 6>(p, stream);
+  if (d_out % 256 == 0) return launch<false, true, 256, 3>(p, 1, stream);
+  if (d_out % 128 == 0) return launch<false, true, 128, 4>(p, 1, stream);
   return unsupported("bf16 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);
 }
 

@@ -128,7 +128,9 @@ ISPA_API ispa_status_t ispa_lse_merge(const void* o_loc, const float* lse_loc, c
  * summed over the n_rows rows of one call (the warm-up rows, [gist §2.1]).
  * a_loc, a_delta [n_rows, d_model], dtype dt, row stride row_stride elements.
  * G, R [d_model, d_model] fp32 row-major, accumulated in place; zero_first != 0
- * overwrites them instead.  d_model must be a multiple of 128 (bf16) or 4
+ * overwrites them instead.  G is symmetric: only its lower triangle (row >= col)
+ * is guaranteed; entries above the diagonal are unspecified (ispa_absorb_solve
+ * reads the lower triangle only).  d_model must be a multiple of 128 (bf16) or 4
  * (fp32).  n_rows == 0 is a no-op (or a zero fill when zero_first != 0).
  */
 ISPA_API ispa_status_t ispa_gram_accumulate(const void* a_loc, const void* a_delta, int64_t n_rows, int64_t d_model,
