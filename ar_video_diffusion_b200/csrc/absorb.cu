@@ -5,8 +5,9 @@
 // section 2 stage 2 "Layer Absorb"), then W_new = W + dW (stage 3).
 //
 // fp32 throughout, all on the device, stream ordered:
-//   1. trace(G) -> lambda (one block, fp64 sum);  M = G + lambda I;
-//   2. S = R W  (written straight into dW, which the solves then update in place);
+//   1. S = R W, written straight into dW (which the solves then update in
+//      place): on the tensor cores as hi(R) W + lo(R) W when W is bf16;
+//   2. trace(G) -> lambda (one block, fp64 sum);  M = G + lambda I;
 //   3. right-looking blocked Cholesky M = L L^T with 64 x 64 panels: the
 //      diagonal block is factored in shared memory by one CTA (which also
 //      forms its inverse), the panel below is multiplied by that inverse, and
@@ -145,66 +146,76 @@ __global__ void shift_kernel(const float* __restrict__ G, float* __restrict__ M,
 
 // Factor the 64 x 64 diagonal block k of M in place (lower triangle) and
 // write the inverse of its Cholesky factor to Linv (64 x 64, row-major).
-// Column-by-column: at step j the pivot is square-rooted, column j of L is
+// Column by column: at step j the pivot is square-rooted, column j of L is
 // scaled, the trailing lower triangle gets the rank-1 update, and the same
-// elimination is applied to X (initially I), which ends as L^-1.  Thread t owns
-// column t % 64 of rows t / 64 + 4 a, a = 0..15.
+// elimination is applied to X (initially I), which ends as L^-1.  Thread t
+// keeps column t % 64 of rows t / 64 + 4 a (a = 0..15) of A and of X in
+// registers; only column j of A and row j of X go through shared memory.  The
+// column loop is unrolled so that the register holding row j is static.
 __global__ void __launch_bounds__(256) potrf_diag_kernel(float* M, int D, int k, float* Linv, int32_t* status) {
-  __shared__ float A[kT][kT + 1];
-  __shared__ float X[kT][kT + 1];
-  __shared__ float s_inv;
+  __shared__ float colbuf[2][kT];  // column j of the current A, double-buffered by the parity of j
+  __shared__ float rowx[kT];  // row j of the current X (already scaled)
   __shared__ int bad;
   const int tid = threadIdx.x;
   const int c = tid & 63, r0 = tid >> 6;
   float* blk = M + (int64_t)k * kT * D + (int64_t)k * kT;
+  float a[16], x[16];
 #pragma unroll
-  for (int a = 0; a < 16; ++a) {
-    const int i = r0 + 4 * a;
-    A[i][c] = blk[(int64_t)i * D + c];
-    X[i][c] = (i == c) ? 1.f : 0.f;
+  for (int t = 0; t < 16; ++t) {
+    const int i = r0 + 4 * t;
+    a[t] = blk[(int64_t)i * D + c];
+    x[t] = (i == c) ? 1.f : 0.f;
   }
   if (tid == 0) bad = -1;
-  __syncthreads();
-#pragma unroll 1
-  for (int j = 0; j < kT; ++j) {
-    if (tid == 0) {
-      float d = A[j][j];
-      if (!(d > 0.f) || !isfinite(d)) {
-        if (bad < 0) bad = j;
-        d = 1.f;
-      }
-      const float sq = sqrtf(d);
-      A[j][j] = sq;
-      s_inv = 1.0f / sq;
-    }
-    __syncthreads();
-    const float inv = s_inv;
-    if (tid < kT) {
-      if (tid > j) A[tid][j] *= inv;
-      X[j][tid] *= inv;
-    }
-    __syncthreads();
-    const float acj = A[c][j];
-    const float xjc = X[j][c];
 #pragma unroll
-    for (int a = 0; a < 16; ++a) {
-      const int i = r0 + 4 * a;
-      if (i > j) {
-        const float aij = A[i][j];
-        if (c > j && c <= i) A[i][c] -= aij * acj;
-        X[i][c] -= aij * xjc;
+  for (int j = 0; j < kT; ++j) {
+    // step j writes column j while slower threads may still read column j-1
+    float* colj = colbuf[j & 1];
+    if (c == j) {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) colj[r0 + 4 * t] = a[t];
+    }
+    __syncthreads();
+    float d = colj[j];
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (tid == 0 && bad < 0) bad = j;
+      d = 1.f;
+    }
+    const float ljj = sqrtf(d);
+    const float inv = 1.0f / ljj;
+    if (r0 == (j & 3)) {  // owner of row j of X
+      x[j >> 2] *= inv;
+      rowx[c] = x[j >> 2];
+    }
+    if (c == j) {  // this column becomes column j of L
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const int i = r0 + 4 * t;
+        a[t] = (i == j) ? ljj : (i > j ? a[t] * inv : a[t]);
       }
     }
     __syncthreads();
+    const float lcj = colj[c] * inv;  // L[c][j] for c > j
+    const float xjc = rowx[c];        // X[j][c]
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const int i = r0 + 4 * t;
+      if (i > j) {
+        const float lij = colj[i] * inv;
+        if (c > j && c <= i) a[t] -= lij * lcj;
+        x[t] -= lij * xjc;
+      }
+    }
   }
+  __syncthreads();
   if (tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = k * kT + bad;
   }
 #pragma unroll
-  for (int a = 0; a < 16; ++a) {
-    const int i = r0 + 4 * a;
-    if (c <= i) blk[(int64_t)i * D + c] = A[i][c];
-    Linv[i * kT + c] = X[i][c];
+  for (int t = 0; t < 16; ++t) {
+    const int i = r0 + 4 * t;
+    if (c <= i) blk[(int64_t)i * D + c] = a[t];
+    Linv[i * kT + c] = x[t];
   }
 }
 
@@ -274,6 +285,17 @@ __global__ void __launch_bounds__(256) diag_apply_kernel(float* X, int D, int k,
     for (int b = 0; b < 4; ++b) blk[(int64_t)(ty + 16 * a) * D + tx + 16 * b] = acc[a][b];
 }
 
+// R (fp32) -> hi = bf16(R), lo = bf16(R - hi): R = hi + lo to about 2^-16 relative.
+__global__ void split_bf16_kernel(const float* __restrict__ R, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float v = R[e];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[e] = h;
+    lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
 template <typename TW>
 __global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ dW, TW* __restrict__ Wn, int64_t n) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
@@ -289,6 +311,10 @@ __global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ 
 
 size_t absorb_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
 
+// C[M, N] (= | +=) A[M, K] W[K, N] on the tensor cores (bf16 operands, fp32 C).
+ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_stride, const void* w, int64_t N,
+                               float* c, int64_t ldc, bool accumulate, cudaStream_t stream);
+
 ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D64,
                                   double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
                                   int32_t* status, cudaStream_t st) {
@@ -299,14 +325,25 @@ ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W,
   float* Linv = M + (int64_t)D * D;
   double* lam = reinterpret_cast<double*>(Linv + (int64_t)D * kT);
 
-  trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
   const int sms = num_sms();
-  shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
-  // S = R W, written into dW
-  if (w_dt == ISPA_DT_BF16)
+  // S = R W, written into dW.  With bf16 W the product runs on the tensor
+  // cores as hi(R) W + lo(R) W, the two bf16 halves of R staged in M's storage
+  // before M is formed.
+  if (w_dt == ISPA_DT_BF16 && D % 128 == 0) {
+    __nv_bfloat16* Rh = reinterpret_cast<__nv_bfloat16*>(M);
+    __nv_bfloat16* Rl = Rh + (int64_t)D * D;
+    split_bf16_kernel<<<sms * 4, 256, 0, st>>>(R, Rh, Rl, (int64_t)D * D);
+    ispa_status_t s1 = gemm_rm_bf16_f32(Rh, D, D, D, W, D, dW, D, false, st);
+    if (s1 != ISPA_OK) return s1;
+    s1 = gemm_rm_bf16_f32(Rl, D, D, D, W, D, dW, D, true, st);
+    if (s1 != ISPA_OK) return s1;
+  } else if (w_dt == ISPA_DT_BF16) {
     gemm_f32(st, D, D, D, 1.f, R, D, 1, static_cast<const __nv_bfloat16*>(W), D, 1, 0.f, dW, D);
-  else
+  } else {
     gemm_f32(st, D, D, D, 1.f, R, D, 1, static_cast<const float*>(W), D, 1, 0.f, dW, D);
+  }
+  trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
+  shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
   // Cholesky
   for (int k = 0; k < nb; ++k) {
     float* Lk = Linv + (int64_t)k * kT * kT;

@@ -273,6 +273,28 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   return launch<true, true, 128, 4>(p, (int)splits, stream);
 }
 
+// C[M, N] (= | +=) A[M, K] W[K, N]: bf16 row-major A and W, fp32 C (ldc).
+ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_stride, const void* w, int64_t N,
+                               float* c, int64_t ldc, bool accumulate, cudaStream_t stream) {
+  using namespace gemm;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  if (!encode_map_bf16_2d(&p.a_map, a, K, M, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.b_map[0], w, N, K, N * 2, 64, 64)) return ISPA_ERR_CUDA;
+  p.b_map[1] = p.b_map[0];
+  p.M = (int32_t)M;
+  p.N = (int32_t)N;
+  p.K = (int32_t)K;
+  p.n_split = (int32_t)N;
+  p.k_per_split = (int32_t)(((K + kBK - 1) / kBK) * kBK);
+  p.c[0] = c;
+  p.c[1] = c;
+  p.ldc = ldc;
+  p.mode = accumulate ? kReduceF32 : kStoreF32;
+  if (N % 128) return unsupported("tensor-core GEMM needs N %% 128 == 0");
+  return launch<false, true, 128, 4>(p, 1, stream);
+}
+
 // y[n_rows, d_out] = a[n_rows, d_in] * w[d_in, d_out]  (bf16 in/out).
 ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t d_out, int64_t a_stride,
                            const void* w, void* y, cudaStream_t stream) {
