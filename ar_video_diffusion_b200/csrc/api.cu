@@ -124,6 +124,7 @@ extern "C" ispa_status_t ispa_lse_merge(const void* o_loc, const float* lse_loc,
   if (!o_loc || !lse_loc || !o_hist || !lse_hist || !a_full) return invalid("required pointer is NULL");
   if (n_q <= 0 || n_heads <= 0) return invalid("n_q and n_heads must be positive");
   if (head_dim <= 0 || head_dim % 8) return unsupported("head_dim must be a positive multiple of 8");
+  if (n_heads > 64) return unsupported("at most 64 heads");
   for (const void* p : {o_loc, o_hist, (const void*)a_full, (const void*)a_delta})
     if (p && !aligned16(p)) return invalid("matrices must be 16-byte aligned");
   return lse_merge_launch(o_loc, lse_loc, o_hist, lse_hist, n_q, n_heads, head_dim, dt, a_full, a_delta, lse_full,

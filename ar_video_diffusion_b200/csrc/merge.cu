@@ -5,9 +5,8 @@
 //   L = logaddexp(L_loc, L_hist),  A_full = e^(L_loc-L) O_loc + e^(L_hist-L) O_hist,
 //   delta = A_full - O_loc.
 //
-// Pure streaming work (HBM-bound): every thread moves 16-byte vectors of both
-// branch outputs, grid-stride over the [n_q, D] matrices; the per-(head,row)
-// weights come from the two LSE arrays, which stay in L1/L2.
+// Pure streaming work (HBM-bound): blocks of whole rows, 16-byte vectors of
+// both branch outputs, the per-(row, head) weights computed once per block.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -64,63 +63,61 @@ __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) {
                : "memory");
 }
 
-// Each thread handles kUnroll independent 16-byte vectors per pass so that
-// enough loads are in flight to cover HBM latency.
+constexpr int kRowsPerBlock = 4;
+constexpr int kMaxHeads = 64;
+
+// One block fuses kRowsPerBlock whole rows.  The per-(row, head) weights
+// e^(L_loc - L), e^(L_hist - L) and L are computed once into shared memory
+// (and L written out); the block then streams the rows' 16-byte vectors with
+// packed fp32 math, so the per-vector work stays within the instruction
+// budget of an HBM-bound stream.
 template <typename T>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const uint4* __restrict__ o_loc,
                                                         const float* __restrict__ lse_loc,
                                                         const uint4* __restrict__ o_hist,
                                                         const float* __restrict__ lse_hist, int64_t n_q, int D,
-                                                        int head_dim, uint4* __restrict__ a_full,
+                                                        int head_dim, int n_heads, uint4* __restrict__ a_full,
                                                         uint4* __restrict__ a_delta, float* __restrict__ lse_full) {
   constexpr int N = Vec<T>::kN;
-  constexpr int kUnroll = 2;
+  __shared__ float2 wts[kRowsPerBlock][kMaxHeads];
   const int vec_per_row = D / N;
-  const int64_t total = n_q * vec_per_row;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e0 < total; e0 += stride * kUnroll) {
-    uint4 ua[kUnroll], ub[kUnroll];
-    float wl[kUnroll], wh[kUnroll], Ls[kUnroll];
-    bool act[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t e = e0 + u * stride;
-      act[u] = e < total;
-      if (!act[u]) continue;
-      ua[u] = ld_stream(o_loc + e);
-      ub[u] = ld_stream(o_hist + e);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (!act[u]) continue;
-      const int64_t e = e0 + u * stride;
-      const int64_t row = e / vec_per_row;
-      const int head = (int)(e - row * vec_per_row) * N / head_dim;
-      const float ll = __ldg(lse_loc + (int64_t)head * n_q + row);
-      const float lh = __ldg(lse_hist + (int64_t)head * n_q + row);
+  const int vec_per_head = head_dim / N;
+  for (int64_t r0 = (int64_t)blockIdx.x * kRowsPerBlock; r0 < n_q; r0 += (int64_t)gridDim.x * kRowsPerBlock) {
+    const int rows = n_q - r0 < kRowsPerBlock ? (int)(n_q - r0) : kRowsPerBlock;
+    for (int t = threadIdx.x; t < rows * n_heads; t += blockDim.x) {
+      const int rr = t / n_heads, h = t - rr * n_heads;
+      const int64_t li = (int64_t)h * n_q + r0 + rr;
+      const float ll = __ldg(lse_loc + li), lh = __ldg(lse_hist + li);
       const float mx = fmaxf(ll, lh);
-      Ls[u] = mx + logf(expf(ll - mx) + expf(lh - mx));
-      wl[u] = expf(ll - Ls[u]);
-      wh[u] = expf(lh - Ls[u]);
+      const float L = mx + logf(expf(ll - mx) + expf(lh - mx));
+      wts[rr][h] = make_float2(expf(ll - L), expf(lh - L));
+      if (lse_full) lse_full[li] = L;
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (!act[u]) continue;
-      const int64_t e = e0 + u * stride;
+    __syncthreads();
+    const int nvec = rows * vec_per_row;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      const int rr = v / vec_per_row;
+      const int h = (v - rr * vec_per_row) / vec_per_head;
+      const int64_t e = (r0 + rr) * vec_per_row + (v - rr * vec_per_row);
+      const uint4 ua = ld_stream(o_loc + e), ub = ld_stream(o_hist + e);
+      const float2 w = wts[rr][h];
       float a[N], b[N], f[N], d[N];
-      unpack(ua[u], a, (T*)nullptr);
-      unpack(ub[u], b, (T*)nullptr);
+      unpack(ua, a, (T*)nullptr);
+      unpack(ub, b, (T*)nullptr);
 #pragma unroll
-      for (int j = 0; j < N; ++j) {
-        f[j] = wl[u] * a[j] + wh[u] * b[j];
-        d[j] = f[j] - a[j];
+      for (int j = 0; j < N; j += 2) {
+        const float2 fa = ffma2(make_float2(a[j], a[j + 1]), make_float2(w.x, w.x),
+                                make_float2(b[j] * w.y, b[j + 1] * w.y));
+        const float2 da = fadd2(fa, make_float2(-a[j], -a[j + 1]));
+        f[j] = fa.x;
+        f[j + 1] = fa.y;
+        d[j] = da.x;
+        d[j + 1] = da.y;
       }
       st_stream(a_full + e, pack(f, (T*)nullptr));
       if (a_delta) st_stream(a_delta + e, pack(d, (T*)nullptr));
-      const int64_t row = e / vec_per_row;
-      const int col = (int)(e - row * vec_per_row) * N;
-      if (lse_full && col % head_dim == 0) lse_full[(int64_t)(col / head_dim) * n_q + row] = Ls[u];
     }
+    __syncthreads();
   }
 }
 
@@ -130,18 +127,16 @@ ispa_status_t lse_merge_launch(const void* o_loc, const float* lse_loc, const vo
                                int64_t n_q, int32_t n_heads, int32_t head_dim, ispa_dtype_t dt, void* a_full,
                                void* a_delta, float* lse_full, cudaStream_t stream) {
   const int D = n_heads * head_dim;
-  const int N = dt == ISPA_DT_BF16 ? 8 : 4;
-  const int64_t total = n_q * (D / N);
-  const int64_t want = (total + 511) / 512;  // two vectors per thread
-  const int cap = num_sms() * 8;
-  const int blocks = (int)(want < cap ? want : cap);
+  const int64_t row_blocks = (n_q + merge::kRowsPerBlock - 1) / merge::kRowsPerBlock;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  const int blocks = (int)(row_blocks < cap ? row_blocks : cap);
   if (dt == ISPA_DT_BF16)
     merge::lse_merge_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
-        (const uint4*)o_loc, lse_loc, (const uint4*)o_hist, lse_hist, n_q, D, head_dim, (uint4*)a_full,
+        (const uint4*)o_loc, lse_loc, (const uint4*)o_hist, lse_hist, n_q, D, head_dim, n_heads, (uint4*)a_full,
         (uint4*)a_delta, lse_full);
   else
     merge::lse_merge_kernel<float><<<blocks, 256, 0, stream>>>((const uint4*)o_loc, lse_loc, (const uint4*)o_hist,
-                                                               lse_hist, n_q, D, head_dim, (uint4*)a_full,
+                                                               lse_hist, n_q, D, head_dim, n_heads, (uint4*)a_full,
                                                                (uint4*)a_delta, lse_full);
   return check_launch("lse_merge_kernel");
 }

@@ -278,7 +278,7 @@ def run_ours(args, rank, world, device):
     pk, src = peaks()
     tc_peak = pk["bf16_tflops"]
     achieved = F / (t_dual / args.steps * 1e-3) / 1e12
-    traffic = load_traffic("dual_attention_kernel<128,3>")
+    traffic = load_traffic("attention_kernel<128,3>")
     res = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -315,7 +315,7 @@ def run_ours(args, rank, world, device):
             "lse_merge_gbs": round(merge_gbs, 1)},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_peak, 4), "traffic": traffic,
-                     "kernel": "dual_attention_kernel<128,3>", "peak_source": f"{src} bf16 burst",
+                     "kernel": "attn2::attention_kernel<128,3>", "peak_source": f"{src} bf16 burst",
                      "frac_of_spec_2250": round(achieved / 2250.0, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
