@@ -65,7 +65,9 @@ def gram_flops(w, rows) -> float:
 
 def absorb_launches(D: int) -> int:
     nb = D // 64
-    return 7 * nb  # trace, shift, R W, W_new + 3nb-2 Cholesky + 2(2nb-1) solves
+    # split of R, two tensor-core products for R W, trace, shift, W_new,
+    # 3nb-2 Cholesky launches and 2(2nb-1) triangular-solve launches
+    return 7 * nb + 2
 
 
 def cores() -> int:
