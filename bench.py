@@ -63,6 +63,21 @@ def gram_flops(w, rows) -> float:
     return rows * D * (D + 1) + 2.0 * rows * D * D
 
 
+def max_over_ranks(times_ms, world: int, device) -> list:
+    """Elementwise max over the ranks of per-rank device times (ms); every rank
+    takes the same collective step, and gets the same list back."""
+    t = torch.tensor([float(v) for v in times_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def replica_tflops(flop_per_step: float, steps: int, world: int, t_max_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps of
+    `flop_per_step` FLOPs, over the slowest rank's time."""
+    return world * flop_per_step * steps / (t_max_ms * 1e-3) / 1e12
+
+
 def absorb_launches(D: int) -> int:
     nb = D // 64
     # split of R, two tensor-core products for R W, trace, shift, W_new,
@@ -231,12 +246,9 @@ def run_ours(args, rank, world, device):
     mean = [comp_ms[n] for n, _ in comps]  # ms per component
     t_dual = comp_ms["dual_attention"] * args.steps
     # max over ranks of the time that defines `value`, and of the step time
-    vals = torch.tensor([t_dual, total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    t_dual_max, total_max = (float(v) for v in vals.tolist())
+    t_dual_max, total_max = max_over_ranks([t_dual, total_ms], world, device)
     F = attn_flops(w)
-    value = world * F * args.steps / (t_dual_max * 1e-3) / 1e12
+    value = replica_tflops(F, args.steps, world, t_dual_max)
 
     # e2e through the public API with host buffers: pinned H2D of the chunk's
     # new inputs (queries and the current chunk's K, V; the sink/history cache
@@ -265,10 +277,8 @@ def run_ours(args, rank, world, device):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * F * args.steps / (float(e2e_ms.item()) * 1e-3) / 1e12
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, device)
+    e2e_value = replica_tflops(F, args.steps, world, e2e_ms)
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = out_a.numel() * 2 + out_l.numel() * 4
 

@@ -1,0 +1,112 @@
+"""Host side of the N > 1 benchmark path, on CPU with two gloo ranks.
+
+The hot path is replicated, not sharded: with N processes every rank runs the
+same layer, and the only collectives are the barriers and the max over ranks
+of the device times that define the throughput.  These tests run that
+reduction and the reference arm's rank handling as real separate processes.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+RANK_CODE = r"""
+import datetime, json, os, sys
+sys.path.insert(0, os.environ["ISPA_ROOT"])
+import torch
+import torch.distributed as dist
+import bench
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+rank, world = dist.get_rank(), dist.get_world_size()
+times = json.loads(os.environ["RANK_TIMES"])[rank]
+got = bench.max_over_ranks(times, world, torch.device("cpu"))
+value = bench.replica_tflops(2.0e12, 4, world, got[0])
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "world": world, "max": got, "value": value}))
+"""
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _run_ranks(code, world, extra_env, args=(), timeout=120):
+    port = _free_port()
+    procs = []
+    for r in range(world):
+        env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(r),
+                   LOCAL_RANK=str(r), WORLD_SIZE=str(world), ISPA_ROOT=ROOT, **extra_env)
+        cmd = [sys.executable, "-c", code] if code else [sys.executable, os.path.join(ROOT, "bench.py"), *args]
+        procs.append(subprocess.Popen(cmd, env=env, cwd=ROOT, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                      text=True))
+    outs = []
+    try:
+        for p in procs:
+            out, err = p.communicate(timeout=timeout)
+            outs.append((p.returncode, out, err))
+    finally:
+        for p in procs:
+            if p.poll() is None:
+                p.kill()
+    return outs
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    # rank 0 is slower on the first timing, rank 1 on the second
+    times = [[30.0, 7.5, 1.0], [20.0, 9.25, 1.0]]
+    outs = _run_ranks(RANK_CODE, 2, {"RANK_TIMES": json.dumps(times)})
+    results = []
+    for rc, out, err in outs:
+        assert rc == 0, err[-2000:]
+        results.append(json.loads(out.strip().splitlines()[-1]))
+    assert sorted(r["rank"] for r in results) == [0, 1]
+    for r in results:
+        assert r["world"] == 2
+        assert r["max"] == [30.0, 9.25, 1.0]
+        # 2 replicas x 4 steps x 2 TFLOP over the slowest rank's 30 ms
+        assert r["value"] == pytest.approx(2 * 4 * 2.0 / 30e-3)
+
+
+def test_replica_tflops_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch
+    assert bench.max_over_ranks([1.5, 2.5], 1, torch.device("cpu")) == [1.5, 2.5]
+    assert bench.replica_tflops(1.0e12, 10, 1, 1000.0) == pytest.approx(10.0)
+    # weak scaling: N replicas over the same slowest time give N times the value
+    assert bench.replica_tflops(1.0e12, 10, 8, 1000.0) == pytest.approx(80.0)
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    # under torchrun only rank 0 runs the oracle arm; rank 1 exits at once
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+               MASTER_PORT=str(_free_port()))
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, cwd=ROOT, capture_output=True, text=True,
+                       timeout=120)
+    assert p.returncode == 0, p.stderr[-2000:]
+    assert p.stdout.strip() == ""
+
+
+def test_reference_arm_rank0_line():
+    env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["value"] > 0
