@@ -79,10 +79,10 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + NST * kTileBytes;
-  static constexpr int kXs = kV + NST * kTileBytes;  // half 1's (m, l) per row at the local checkpoint
+  static constexpr int kXs = kV + NST * kTileBytes;  // warpgroup 1's (m, l) per row at the local checkpoint
   static constexpr int kBars = kXs + 2 * kBM * 4;
-  // kv_full[NST], kv_empty[NST], q_full, s_full[2], p_full[2 halves][2 tile parities], pv_done, xsum[2], teardown
-  static constexpr int kNumBars = 2 * NST + 1 + 2 + 4 + 1 + 2 + 1;
+  // kv_full[NST], kv_empty[NST], q_full, s_full[2], p_full[2], pv_done[2], ck_done, xsum[2], teardown
+  static constexpr int kNumBars = 2 * NST + 1 + 2 + 2 + 2 + 1 + 2 + 1;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -169,65 +169,74 @@ __device__ void producer(const Params& p, uint8_t* smem, uint64_t* q_full, uint6
 }
 
 // ------------------------------------------------------------- MMA issuer
+// The whole warp runs the loop; one elected lane issues.  Key tile i belongs to softmax
+// warpgroup i & 1, whose S buffer and O accumulator it uses.
 template <int HD, int NST>
 __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uint64_t* kv_full, uint64_t* kv_empty,
-                           uint64_t* s_full, uint64_t* p_full, uint64_t* pv_done, uint64_t* teardown,
-                           volatile int* abort_flag, uint32_t tmem) {
+                           uint64_t* s_full, uint64_t* p_full, uint64_t* pv_done, uint64_t* ck_done,
+                           uint64_t* teardown, volatile int* abort_flag, uint32_t tmem) {
   using L = Layout<HD, NST>;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
   const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
   const int T = p.n_tiles, n_loc = p.n_local_tiles;
+  const bool ck = p.dual && n_loc > 0 && n_loc < T;  // a local result is taken between the tiles
 
+  // the whole warp runs the loop and every wait; the elected lane issues
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+  };
   auto issue_s = [&](int j) -> bool {
     const int stage = j % NST;
-    if (!mbar_wait(&kv_full[stage], (j / NST) & 1, abort_flag)) return false;
+    if (!wait(&kv_full[stage], (j / NST) & 1)) return false;
     tc_fence_after();
     const uint32_t kb = sK + stage * L::kTileBytes;
     const uint32_t d = tmem + kTmS + (j & 1) * 128;
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-      umma_ss(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+      umma_ss_warp(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
+                   kk > 0 ? 1u : 0u);
     }
-    umma_commit(&s_full[j & 1]);
+    umma_commit_warp(&s_full[j & 1]);
     return true;
   };
 
-  bool ok = mbar_wait(q_full, 0, abort_flag);
+  bool ok = wait(q_full, 0);
   tc_fence_after();
   if (ok && T > 0) ok = issue_s(0);
   if (ok && T > 1) ok = issue_s(1);
+  bool ck_seen = false;
   for (int i = 0; ok && i < T; ++i) {
-    const bool fresh = (i == 0) || (p.dual && i == n_loc);
+    const int w = i & 1;
+    const bool first_hist = ck && i >= n_loc && i - 2 < n_loc;
+    const bool fresh = i < 2 || first_hist;
+    if (first_hist && !ck_seen) {
+      // the first history products overwrite the accumulators; the local
+      // result must have been read out of them first
+      if (!wait(ck_done, 0)) break;
+      ck_seen = true;
+    }
     const int stage = i % NST;
     const uint32_t vb = sV + stage * L::kTileBytes;
-    const uint32_t pb = tmem + kTmS + (i & 1) * 128;
-    // O_h += P_h V_h: keys 64h..64h+63, P_h in columns [64h, 64h + 32) of the S buffer
-    for (int h = 0; h < 2; ++h) {
-      // p_full[2 h + (i & 1)]: a half can run at most one tile ahead of this
-      // wait (the tile after next needs S(i + 2), issued below), so one barrier
-      // per tile parity keeps every parity wait unambiguous
-      if (!mbar_wait(&p_full[2 * h + (i & 1)], (i >> 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    const uint32_t pb = tmem + kTmS + w * 128;
+    // p_full[w] completes once per tile of warpgroup w; its next phase needs
+    // S(i + 2), issued below, so the parity is unambiguous
+    if (!wait(&p_full[w], (i >> 1) & 1)) break;
+    tc_fence_after();
+    // O_w += P V: P (bf16, 128 keys) in the first 64 columns of the S buffer
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = 4 * h + k4;
-        umma_ts(tmem + kTmO + h * HD, pb + h * 64 + k4 * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024),
-                kIdescPV, (k4 > 0 || !fresh) ? 1u : 0u);
-      }
-    }
-    if (!ok) break;
-    umma_commit(&kv_empty[stage]);
-    umma_commit(pv_done);
+    for (int kk = 0; kk < 8; ++kk)
+      umma_ts_warp(tmem + kTmO + w * HD, pb + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024), kIdescPV,
+                   (kk > 0 || !fresh) ? 1u : 0u);
+    umma_commit_warp(&kv_empty[stage]);
+    umma_commit_warp(&pv_done[w]);
     if (i + 2 < T) ok = issue_s(i + 2);
   }
   // every MMA must have completed before tensor memory is released
-  umma_commit(teardown);
+  umma_commit_warp(teardown);
   mbar_wait_drain(teardown, 0, 100000000ull);
+  __syncwarp();
 }
 
 // ------------------------------------------------------------------ softmax
@@ -239,13 +248,14 @@ __device__ __forceinline__ uint32_t pack_p_bf16x2(float lo, float hi) {
 }
 
 struct Row {
-  int half, lane, row, grow;
+  int wg, lane, row, grow;
   bool row_ok;
   uint32_t lane_base;
 };
 
-// Merged, normalised accumulator for channels [c0, c0 + 32 * n32) of this row:
-// (O_0 w0 + O_1 w1) / lt, with O_h the two halves' accumulators.
+// Merged, normalised accumulator for channels [32 cc, 32 cc + 32) of this
+// row: (O_0 w0 + O_1 w1) / lt.  A weight of 0 means that accumulator holds
+// nothing of this result (it may hold stale data) and is not read.
 template <int HD>
 __device__ __forceinline__ void load_merged(const Row& r, int cc, float w0, float w1, float inv, float (&x)[32]) {
   uint32_t a[32], b[32];
@@ -253,139 +263,157 @@ __device__ __forceinline__ void load_merged(const Row& r, int cc, float w0, floa
   tmem_ld32(r.lane_base + kTmO + HD + 32 * cc, b);
   tmem_wait_ld();
 #pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = (__uint_as_float(a[j]) * w0 + __uint_as_float(b[j]) * w1) * inv;
+  for (int j = 0; j < 32; ++j) {
+    const float u = w0 != 0.f ? __uint_as_float(a[j]) * w0 : 0.f;
+    const float v = w1 != 0.f ? __uint_as_float(b[j]) * w1 : 0.f;
+    x[j] = (u + v) * inv;
+  }
+}
+
+// Waits (all lanes) for the product of warpgroup w's tile number k (counted
+// per warpgroup) to have completed.
+__device__ __forceinline__ bool wait_pv(uint64_t* pv_done, int w, int k, volatile int* abort_flag) {
+  if (k < 0) return true;
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[w], k & 1, abort_flag));
+  tc_fence_after();
+  return ok;
 }
 
 template <int HD, int NST>
 __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t* s_full, uint64_t* p_full,
-                        uint64_t* pv_done, uint64_t* xsum, volatile int* abort_flag, int q0, int head) {
+                        uint64_t* pv_done, uint64_t* ck_done, uint64_t* xsum, volatile int* abort_flag, int q0,
+                        int head) {
   using L = Layout<HD, NST>;
-  float* xck = reinterpret_cast<float*>(smem + L::kXs);  // checkpoint: half 1's (m, l) per row
-  float* xfin = reinterpret_cast<float*>(smem + L::kQ);  // final: [half][m, l, lse_loc][row]; Q is dead by then
+  float* xck = reinterpret_cast<float*>(smem + L::kXs);  // checkpoint: warpgroup 1's (m, l) per row
+  float* xfin = reinterpret_cast<float*>(smem + L::kQ);  // final: [wg][m, l, lse_loc][row]; Q is dead by then
   Row r;
-  const int w = threadIdx.x >> 5;
-  r.half = (w - 4) >> 2;
+  const int warp = threadIdx.x >> 5;
+  r.wg = (warp - 4) >> 2;
   r.lane = threadIdx.x & 31;
-  r.row = (w & 3) * 32 + r.lane;
+  r.row = (warp & 3) * 32 + r.lane;
   r.grow = q0 + r.row;
   r.row_ok = r.grow < p.n_q;
-  r.lane_base = tmem + ((uint32_t)((w & 3) * 32) << 16);
-  const uint32_t o_own = r.lane_base + kTmO + r.half * HD;
+  r.lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const int w = r.wg;
+  const uint32_t o_own = r.lane_base + kTmO + w * HD;
+  const uint32_t sbuf = r.lane_base + kTmS + w * 128;
   const float sl2 = p.scale_log2;
   const int T = p.n_tiles, n_loc = p.n_local_tiles;
   const bool dual = p.dual != 0;
+  const bool ck = dual && n_loc > 0 && n_loc < T;
+  bool ck_pending = ck;
   bool ok = true;
 
   float m_used = -INFINITY, l = 0.f, lse_loc2 = 0.f;
+  bool o_live = false;  // O_w holds products of the current accumulation
+
+  // local result: the two warpgroups' accumulators are merged, normalised and
+  // written (A_loc, LSE_loc) by warpgroup 0; then both restart
+  auto checkpoint = [&](int k_next) -> bool {
+    if (!wait_pv(pv_done, w, k_next - 1, abort_flag)) return false;  // own last local product
+    if (w == 1) {
+      xck[r.row] = m_used;
+      xck[kBM + r.row] = l;
+      mbar_arrive(&xsum[0]);
+    } else {
+      if (!wait_pv(pv_done, 1, (n_loc >> 1) - 1, abort_flag)) return false;  // warpgroup 1's last local product
+      if (!__all_sync(0xffffffffu, mbar_wait(&xsum[0], 0, abort_flag))) return false;
+      const float m1 = xck[r.row], l1 = xck[kBM + r.row];
+      const float mm = fmaxf(m_used, m1);
+      const float w0 = l > 0.f ? ex2(m_used - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
+      const float lt = l * w0 + l1 * w1;
+      const float inv = 1.0f / lt;
+      __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD;
 #pragma unroll 1
-  for (int i = 0; i < T; ++i) {
-    const int b = i & 1;
-    ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (i >> 1) & 1, abort_flag));
+      for (int cc = 0; cc < HD / 32; ++cc) {
+        float x[32];
+        load_merged<HD>(r, cc, w0, w1, inv, x);
+        if (r.row_ok) store_bf16x32(dst + 32 * cc, x);
+      }
+      lse_loc2 = mm + log2f(lt);
+      if (r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
+      tc_fence_before();
+      __syncwarp();
+      if (r.lane == 0) mbar_arrive(ck_done);
+    }
+    m_used = -INFINITY;
+    l = 0.f;
+    o_live = false;
+    return true;
+  };
+
+#pragma unroll 1
+  for (int i = w; i < T; i += 2) {
+    const int k = i >> 1;  // this warpgroup's tile count
+    if (ck_pending && i >= n_loc) {
+      ck_pending = false;
+      if (!(ok = checkpoint(k))) break;
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait(&s_full[w], k & 1, abort_flag));
     if (!ok) break;
     tc_fence_after();
-    const bool boundary = dual && i == n_loc && i > 0;
-    if (boundary) {
-      // local branch complete: half 0 merges both halves and writes A_loc, LSE_loc
-      ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      if (r.half == 1) {
-        xck[r.row] = m_used;
-        xck[kBM + r.row] = l;
-        mbar_arrive(&xsum[0]);
-      } else {
-        ok = __all_sync(0xffffffffu, mbar_wait(&xsum[0], 0, abort_flag));
-        if (!ok) break;
-        const float m1 = xck[r.row], l1 = xck[kBM + r.row];
-        const float mm = fmaxf(m_used, m1);
-        const float w0 = ex2(m_used - mm), w1 = ex2(m1 - mm);
-        const float lt = l * w0 + l1 * w1;
-        const float inv = 1.0f / lt;
-        __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD;
-#pragma unroll 1
-        for (int cc = 0; cc < HD / 32; ++cc) {
-          float x[32];
-          load_merged<HD>(r, cc, w0, w1, inv, x);
-          if (r.row_ok) store_bf16x32(dst + 32 * cc, x);
-        }
-        lse_loc2 = mm + log2f(lt);
-        if (r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
-      }
-      m_used = -INFINITY;
-      l = 0.f;
-    }
-    const bool fresh = (i == 0) || boundary;
     int seg, tok0, valid;
     tile_info(p, i, seg, tok0, valid);
 
-    const uint32_t s_cols = r.lane_base + kTmS + b * 128 + r.half * 64;
-    uint32_t s[2][32];
-    tmem_ld32(s_cols, s[0]);
-    tmem_ld32(s_cols + 32, s[1]);
-    tmem_wait_ld();
-    const int vloc = valid - r.half * 64;  // valid keys within this half
-    if (vloc < 64) {
+    // the whole 128-key row of S in registers
+    uint32_t s[4][32];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc)
+    for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, s[c]);
+    tmem_wait_ld();
+    if (valid < kBN) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (cc * 32 + j >= vloc) s[cc][j] = __float_as_uint(-INFINITY);
+          if (c * 32 + j >= valid) s[c][j] = __float_as_uint(-INFINITY);
     }
-    // P = 2^(s * scale_log2 - m) for this half's 64 keys into the first 32
-    // columns of its half of the S buffer; returns the sum of P
-    const uint32_t p_cols = r.lane_base + kTmS + b * 128 + r.half * 64;
+    // P = 2^(s * scale_log2 - m) as bf16 into the first 64 columns of the S
+    // buffer (whose values are all in registers by now); returns the sum of P
     auto exponentiate = [&](float m) -> float {
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
-      float2 sum2[2];
+      float2 sum2[4];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        sum2[cc] = make_float2(0.f, 0.f);
+      for (int c = 0; c < 4; ++c) {
+        sum2[c] = make_float2(0.f, 0.f);
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float2 x =
-              ffma2(make_float2(__uint_as_float(s[cc][2 * j]), __uint_as_float(s[cc][2 * j + 1])), sc2, nm2);
+              ffma2(make_float2(__uint_as_float(s[c][2 * j]), __uint_as_float(s[c][2 * j + 1])), sc2, nm2);
           const float2 pv = (kEmuPairs & (1u << (j & 7))) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
-          sum2[cc] = fadd2(sum2[cc], pv);
+          sum2[c] = fadd2(sum2[c], pv);
           pk[j] = pack_p_bf16x2(pv.x, pv.y);
         }
-        tmem_st16(p_cols + 16 * cc, pk);
+        tmem_st16(sbuf + 16 * c, pk);
       }
-      const float2 st2 = fadd2(sum2[0], sum2[1]);
+      const float2 st2 = fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3]));
       return st2.x + st2.y;
     };
     auto tile_max = [&]() -> float {
-      float mc[4];
+      float mc[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         const uint32_t* v = &s[q >> 1][(q & 1) * 16];
         mc[q] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
         for (int j = 1; j < 8; ++j) mc[q] = fmax3(mc[q], __uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
       }
-      // an all-masked half gives -inf
-      return fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
+      const float a = fmax3(mc[0], mc[1], mc[2]), b = fmax3(mc[3], mc[4], mc[5]), c = fmaxf(mc[6], mc[7]);
+      return fmax3(a, b, c) * sl2;  // -inf if all masked
     };
-    float psum;
-    if (fresh || m_used == -INFINITY) {
-      // (after all-masked tiles O_h and l are exactly 0, so no rescale is due)
-      m_used = tile_max();
-      // a half whose keys are all masked so far shifts by 0: its P is exactly 0
-      psum = exponentiate(m_used == -INFINITY ? 0.f : m_used);
-    } else {
-      // exponentials with the running maximum straight away; the tile maximum
-      // is computed alongside and only a growth beyond 2^8 (rare) forces a
-      // rescale of O_h and a second pass over this tile
-      psum = exponentiate(m_used);
-      const float m_tile = tile_max();
-      if (__any_sync(0xffffffffu, m_tile > m_used + kRescaleLog2)) {
-        tmem_wait_st();  // the first pass's P stores complete before they are overwritten
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (i - 1) & 1, abort_flag));  // O_h quiescent
-        if (!ok) break;
-        tc_fence_after();
-        const float m_new = fmaxf(m_used, m_tile);
-        const float f = ex2(m_used - m_new);
-        l *= f;
+    // exponentials with the running maximum straight away, the tile maximum
+    // alongside; a growth beyond 2^8 (rare, and always at the start of an
+    // accumulation) rescales what was accumulated and redoes the tile.  O_w
+    // is quiescent here: S(i) was issued after this warpgroup's previous
+    // product, and its completion implies that product's.
+    const bool first = __any_sync(0xffffffffu, m_used == -INFINITY);
+    float psum = first ? 0.f : exponentiate(m_used);
+    const float m_tile = tile_max();
+    if (first || __any_sync(0xffffffffu, m_tile > m_used + kRescaleLog2)) {
+      const float m_new = fmaxf(m_used, m_tile);
+      // rows whose keys are all masked so far keep m = -inf: their P is exactly 0
+      const float f = (m_used == -INFINITY || m_new == -INFINITY) ? 0.f : ex2(m_used - m_new);
+      if (o_live) {
 #pragma unroll 1
         for (int cc = 0; cc < HD / 32; ++cc) {
           uint32_t o[32];
@@ -395,57 +423,64 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
           tmem_st32(o_own + 32 * cc, o);
         }
-        m_used = m_new;
-        psum = exponentiate(m_used);
       }
+      tmem_wait_st();  // the first pass's P stores complete before they are overwritten
+      l *= f;
+      m_used = m_new;
+      psum = exponentiate(m_used == -INFINITY ? 0.f : m_used);
     }
     l += psum;
+    if (!ok) break;
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (r.lane == 0) mbar_arrive(&p_full[2 * r.half + b]);
+    if (r.lane == 0) mbar_arrive(&p_full[w]);
+    o_live = true;
   }
   if (!ok || *abort_flag) return;
-  ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (T - 1) & 1, abort_flag));
-  if (!ok) return;
-  tc_fence_after();
-  // final merge of the two halves' statistics (the Q tile is no longer read)
-  xfin[(r.half * 3 + 0) * kBM + r.row] = m_used;
-  xfin[(r.half * 3 + 1) * kBM + r.row] = l;
-  xfin[(r.half * 3 + 2) * kBM + r.row] = lse_loc2;
+  if (ck_pending) {  // no history tile fell to this warpgroup
+    if (!checkpoint((T - w + 1) >> 1)) return;
+  }
+  // both accumulators final (own first, so the other is at most one phase behind)
+  const int n_own = (T - w + 1) >> 1, n_other = (T - (1 - w) + 1) >> 1;
+  if (!wait_pv(pv_done, w, n_own - 1, abort_flag)) return;
+  if (!wait_pv(pv_done, 1 - w, n_other - 1, abort_flag)) return;
+  // final merge of the two warpgroups' statistics (the Q tile is no longer read)
+  xfin[(w * 3 + 0) * kBM + r.row] = m_used;
+  xfin[(w * 3 + 1) * kBM + r.row] = l;
+  xfin[(w * 3 + 2) * kBM + r.row] = lse_loc2;
   mbar_arrive(&xsum[1]);
-  ok = __all_sync(0xffffffffu, mbar_wait(&xsum[1], 0, abort_flag));
-  if (!ok) return;
+  if (!__all_sync(0xffffffffu, mbar_wait(&xsum[1], 0, abort_flag))) return;
   const float m0 = xfin[r.row], l0 = xfin[kBM + r.row];
   const float m1 = xfin[3 * kBM + r.row], l1 = xfin[4 * kBM + r.row];
-  lse_loc2 = xfin[2 * kBM + r.row];  // computed by half 0 at the checkpoint
+  lse_loc2 = xfin[2 * kBM + r.row];  // computed by warpgroup 0 at the checkpoint
   const float mm = fmaxf(m0, m1);
   const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
   const float lt = l0 * w0 + l1 * w1;
   const float inv = 1.0f / lt;
   const float lse2 = mm + log2f(lt);
   const int64_t li = (int64_t)head * p.n_q + r.grow;
-  const int64_t base = (int64_t)r.grow * p.out_stride + head * HD + r.half * (HD / 2);
-  const int c_first = r.half * (HD / 64);  // this half's 32-channel blocks
+  const int64_t base = (int64_t)r.grow * p.out_stride + head * HD + w * (HD / 2);
+  const int c_first = w * (HD / 64);  // this warpgroup's 32-channel blocks
 
   if (!dual || T == n_loc) {  // single pass, or dual with no history (A_full = A_loc, delta = 0)
 #pragma unroll 1
-    for (int k = 0; k < HD / 64; ++k) {
+    for (int kc = 0; kc < HD / 64; ++kc) {
       float x[32];
-      load_merged<HD>(r, c_first + k, w0, w1, inv, x);
+      load_merged<HD>(r, c_first + kc, w0, w1, inv, x);
       if (!r.row_ok) continue;
-      store_bf16x32(p.a_full + base + 32 * k, x);
+      store_bf16x32(p.a_full + base + 32 * kc, x);
       if (dual) {
-        store_bf16x32(p.a_loc + base + 32 * k, x);
+        store_bf16x32(p.a_loc + base + 32 * kc, x);
         if (p.a_delta) {
           float z[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) z[j] = 0.f;
-          store_bf16x32(p.a_delta + base + 32 * k, z);
+          store_bf16x32(p.a_delta + base + 32 * kc, z);
         }
       }
     }
-    if (r.half == 0 && r.row_ok) {
+    if (w == 0 && r.row_ok) {
       if (p.lse_full) p.lse_full[li] = lse2 * kLn2;
       if (dual && p.lse_loc) p.lse_loc[li] = lse2 * kLn2;
     }
@@ -456,21 +491,21 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
   const float lse_full2 = mx + log2f(exp2f(lse_loc2 - mx) + exp2f(lse2 - mx));
   const float wgt = exp2f(lse2 - lse_full2);
 #pragma unroll 1
-  for (int k = 0; k < HD / 64; ++k) {
+  for (int kc = 0; kc < HD / 64; ++kc) {
     float oh[32];
-    load_merged<HD>(r, c_first + k, w0, w1, inv, oh);
+    load_merged<HD>(r, c_first + kc, w0, w1, inv, oh);
     if (!r.row_ok) continue;
     float a[32], full[32], dl[32];
-    unpack_bf16x32(reinterpret_cast<const uint4*>(p.a_loc + base + 32 * k), a);
+    unpack_bf16x32(reinterpret_cast<const uint4*>(p.a_loc + base + 32 * kc), a);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       dl[j] = wgt * (oh[j] - a[j]);
       full[j] = a[j] + dl[j];
     }
-    store_bf16x32(p.a_full + base + 32 * k, full);
-    if (p.a_delta) store_bf16x32(p.a_delta + base + 32 * k, dl);
+    store_bf16x32(p.a_full + base + 32 * kc, full);
+    if (p.a_delta) store_bf16x32(p.a_delta + base + 32 * kc, dl);
   }
-  if (r.half == 0 && r.row_ok && p.lse_full) p.lse_full[li] = lse_full2 * kLn2;
+  if (w == 0 && r.row_ok && p.lse_full) p.lse_full[li] = lse_full2 * kLn2;
 }
 
 // ------------------------------------------------------------------- kernel
@@ -485,8 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   uint64_t* q_full = kv_empty + NST;
   uint64_t* s_full = q_full + 1;
   uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 4;
-  uint64_t* xsum = pv_done + 1;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* ck_done = pv_done + 2;
+  uint64_t* xsum = ck_done + 1;
   uint64_t* teardown = xsum + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -500,10 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], 4);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(ck_done, 4);
     mbar_init(&xsum[0], 128);
     mbar_init(&xsum[1], 256);
     mbar_init(teardown, 1);
@@ -519,13 +557,20 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) producer<HD, NST>(p, smem, q_full, kv_full, kv_empty, abort_flag, q0, head);
-  } else if (warp == 1) {
-    if (lane == 0)
-      mma_issuer<HD, NST>(p, smem, q_full, kv_full, kv_empty, s_full, p_full, pv_done, teardown, abort_flag, tmem);
-  } else if (warp >= 4) {
-    softmax<HD, NST>(p, smem, tmem, s_full, p_full, pv_done, xsum, abort_flag, q0, head);
+  // registers: the control warpgroup (producer, MMA issuer, tensor-memory
+  // owner) needs few, the softmax warpgroups hold a whole row of S:
+  // 128 x 88 + 256 x 208 = 384 x 168, the launch budget
+  if (warp >= 4) {
+    regs_inc<208>();
+    softmax<HD, NST>(p, smem, tmem, s_full, p_full, pv_done, ck_done, xsum, abort_flag, q0, head);
+  } else {
+    regs_dec<88>();
+    if (warp == 0) {
+      if (lane == 0) producer<HD, NST>(p, smem, q_full, kv_full, kv_empty, abort_flag, q0, head);
+    } else if (warp == 1) {
+      mma_issuer<HD, NST>(p, smem, q_full, kv_full, kv_empty, s_full, p_full, pv_done, ck_done, teardown, abort_flag,
+                          tmem);
+    }
   }
 
   tc_fence_before();
