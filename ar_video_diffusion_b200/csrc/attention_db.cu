@@ -9,27 +9,31 @@
 //
 // One CTA owns 128 query rows of one head and walks the key tiles (128 keys)
 // of the local segments first, then of the history segments.
-//   warp 0      TMA producer: K and V tiles into an NST-stage ring;
-//   warp 1      tcgen05 issuer: S(j) = Q K(j)^T (both operands K-major in
-//               shared memory) and O_h += P_h(j) V_h(j) for the two key halves
-//               h (P from tensor memory, V MN-major in shared memory);
+//   warps 0, 3  TMA producers: Q and the K tiles (warp 0), the V tiles
+//               (warp 3), each into its own NST-stage ring (a K tile is
+//               released once S(j) is done, a V tile after PV(j));
+//   warp 1      tcgen05 issuer, the whole warp converged, one elected lane
+//               issuing: S(j) = Q K(j)^T (both operands K-major in shared
+//               memory) and O_w += P(j) V(j) (P from tensor memory, V
+//               MN-major in shared memory);
 //   warp 2      allocates / frees the 512 tensor-memory columns;
-//   warps 4-11  softmax: two warpgroups split every 128-key S tile into two
-//               64-key halves; thread = (half, query row = TMEM lane).
-// Tensor memory: S double buffer (2 x 128 columns) and one O accumulator per
-// key half (2 x head_dim columns).  Each half runs its own online softmax
-// (its own running maximum and sum) over its 64 keys of every tile, so the
-// halves never exchange anything per tile; their partial results are merged
-// once, when a result is normalised.  The issue order S(0), S(1), PV(0),
-// S(2), PV(1), ... lets the softmax of tile j+1 run while PV(j) and S(j+2)
-// execute.  Each half writes its bf16 P into the first 32 columns of its own
-// half of the S buffer it just read.  Online softmax in the log2 domain with a
-// lazily updated maximum: O_h is rescaled only when the running maximum grows
-// by more than 2^8.
-// Dual mode: at the first history tile the local result is normalised,
-// written (A_loc, LSE_loc) and the accumulator restarts; the epilogue fuses
-// the history result with A_loc (logaddexp of the two LSEs).  Single-pass
-// mode runs one softmax over every tile.
+//   warps 4-11  softmax: two warpgroups; warpgroup w owns the key tiles
+//               j = w mod 2; thread = query row = TMEM lane.
+// Tensor memory: one S buffer and one O accumulator per warpgroup
+// (2 x 128 + 2 x head_dim columns).  Each warpgroup runs its own online
+// softmax (running maximum and sum) over its tiles; the two are merged once,
+// when a result is normalised.  The issue order S(0), S(1), PV(0), S(2),
+// PV(1), ... lets one warpgroup exponentiate while the other's products run.
+// A softmax thread holds the whole 128-key row of S in registers (the
+// warpgroups' register budget is raised with setmaxnreg) and writes the bf16
+// P into the first 64 columns of its S buffer.  Online softmax in the log2
+// domain with a lazily updated maximum: O_w is rescaled only when the
+// running maximum grows by more than 2^8.
+// Dual mode: before its first history tile each warpgroup takes a local
+// checkpoint; warpgroup 0 merges both accumulators and writes A_loc, LSE_loc,
+// and both restart; the epilogue fuses the history result with A_loc
+// (logaddexp of the two LSEs).  Single-pass mode runs one softmax over every
+// tile.
 #include <cstring>
 
 #include "internal.h"
@@ -57,6 +61,8 @@ struct Params {
   CUtensorMap v_map[kMaxSeg];
   int32_t seg_tokens[kMaxSeg];
   int32_t seg_first_tile[kMaxSeg + 1];
+  int32_t seg_last_tile[kMaxSeg];   // last (possibly partial) tile of each segment, -1 if unused
+  int32_t seg_last_valid[kMaxSeg];  // valid keys in that tile
   int32_t n_seg;
   int32_t n_local_tiles;
   int32_t n_tiles;
@@ -82,7 +88,7 @@ struct Layout {
   static constexpr int kXs = kV + NST * kTileBytes;  // warpgroup 1's (m, l) per row at the local checkpoint
   static constexpr int kBars = kXs + 2 * kBM * 4;
   // kv_full[NST], kv_empty[NST], q_full, s_full[2], p_full[2], pv_done[2], ck_done, xsum[2], teardown
-  static constexpr int kNumBars = 2 * NST + 1 + 2 + 2 + 2 + 1 + 2 + 1;
+  static constexpr int kNumBars = 4 * NST + 1 + 2 + 2 + 2 + 1 + 2 + 1;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -130,41 +136,40 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
 }
 
 // ------------------------------------------------------------------ producer
+// One producer thread per operand: a K tile is released once S(j) is done,
+// a V tile only after PV(j).
 template <int HD, int NST>
-__device__ void producer(const Params& p, uint8_t* smem, uint64_t* q_full, uint64_t* kv_full, uint64_t* kv_empty,
-                         volatile int* abort_flag, int q0, int head) {
+__device__ void producer(const Params& p, uint8_t* smem, bool v_side, uint64_t* q_full, uint64_t* full,
+                         uint64_t* empty, volatile int* abort_flag, int q0, int head) {
   using L = Layout<HD, NST>;
-  tma_prefetch_desc(&p.q_map);
-  mbar_arrive_expect_tx(q_full, L::kTileBytes);
+  if (!v_side) {
+    tma_prefetch_desc(&p.q_map);
+    mbar_arrive_expect_tx(q_full, L::kTileBytes);
 #pragma unroll
-  for (int c = 0; c < HD / 64; ++c)
-    tma_load_2d(smem + L::kQ + c * L::kBoxBytes, &p.q_map, q_full, head * HD + 64 * c, q0);
+    for (int c = 0; c < HD / 64; ++c)
+      tma_load_2d(smem + L::kQ + c * L::kBoxBytes, &p.q_map, q_full, head * HD + 64 * c, q0);
+  }
+  uint8_t* ring = smem + (v_side ? L::kV : L::kK);
+  const CUtensorMap* maps = v_side ? p.v_map : p.k_map;
   int n = 0;
   bool ok = true;
   for (; n < p.n_tiles; ++n) {
     const int stage = n % NST;
-    if (n >= NST && !mbar_wait(&kv_empty[stage], ((n / NST) - 1) & 1, abort_flag)) {
+    if (n >= NST && !mbar_wait(&empty[stage], ((n / NST) - 1) & 1, abort_flag)) {
       ok = false;
       break;
     }
     int seg, tok0, valid;
     tile_info(p, n, seg, tok0, valid);
-    if (n < p.n_seg) {
-      tma_prefetch_desc(&p.k_map[n]);
-      tma_prefetch_desc(&p.v_map[n]);
-    }
-    mbar_arrive_expect_tx(&kv_full[stage], 2 * L::kTileBytes);
+    if (n < p.n_seg) tma_prefetch_desc(&maps[n]);
+    mbar_arrive_expect_tx(&full[stage], L::kTileBytes);
 #pragma unroll
-    for (int c = 0; c < HD / 64; ++c) {
-      tma_load_2d(smem + L::kK + stage * L::kTileBytes + c * L::kBoxBytes, &p.k_map[seg], &kv_full[stage],
-                  head * HD + 64 * c, tok0);
-      tma_load_2d(smem + L::kV + stage * L::kTileBytes + c * L::kBoxBytes, &p.v_map[seg], &kv_full[stage],
-                  head * HD + 64 * c, tok0);
-    }
+    for (int c = 0; c < HD / 64; ++c)
+      tma_load_2d(ring + stage * L::kTileBytes + c * L::kBoxBytes, &maps[seg], &full[stage], head * HD + 64 * c, tok0);
   }
-  if (!ok) {  // unwinding after a timeout: wait (bounded) for copies in flight
-    mbar_wait_drain(q_full, 0, 100000000ull);
-    for (int j = n > NST ? n - NST : 0; j < n; ++j) mbar_wait_drain(&kv_full[j % NST], (j / NST) & 1, 100000000ull);
+  if (!ok) {
+    if (!v_side) mbar_wait_drain(q_full, 0, 100000000ull);
+    for (int j = n > NST ? n - NST : 0; j < n; ++j) mbar_wait_drain(&full[j % NST], (j / NST) & 1, 100000000ull);
   }
 }
 
@@ -173,7 +178,7 @@ __device__ void producer(const Params& p, uint8_t* smem, uint64_t* q_full, uint6
 // warpgroup i & 1, whose S buffer and O accumulator it uses.
 template <int HD, int NST>
 __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uint64_t* kv_full, uint64_t* kv_empty,
-                           uint64_t* s_full, uint64_t* p_full, uint64_t* pv_done, uint64_t* ck_done,
+                           uint64_t* v_full, uint64_t* v_empty, uint64_t* s_full, uint64_t* p_full, uint64_t* pv_done, uint64_t* ck_done,
                            uint64_t* teardown, volatile int* abort_flag, uint32_t tmem) {
   using L = Layout<HD, NST>;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
@@ -199,6 +204,7 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uin
                    kk > 0 ? 1u : 0u);
     }
     umma_commit_warp(&s_full[j & 1]);
+    umma_commit_warp(&kv_empty[stage]);
     return true;
   };
 
@@ -222,6 +228,7 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uin
     const uint32_t pb = tmem + kTmS + w * 128;
     // p_full[w] completes once per tile of warpgroup w; its next phase needs
     // S(i + 2), issued below, so the parity is unambiguous
+    if (!wait(&v_full[stage], (i / NST) & 1)) break;
     if (!wait(&p_full[w], (i >> 1) & 1)) break;
     tc_fence_after();
     // O_w += P V: P (bf16, 128 keys) in the first 64 columns of the S buffer
@@ -229,7 +236,7 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uin
     for (int kk = 0; kk < 8; ++kk)
       umma_ts_warp(tmem + kTmO + w * HD, pb + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024), kIdescPV,
                    (kk > 0 || !fresh) ? 1u : 0u);
-    umma_commit_warp(&kv_empty[stage]);
+    umma_commit_warp(&v_empty[stage]);
     umma_commit_warp(&pv_done[w]);
     if (i + 2 < T) ok = issue_s(i + 2);
   }
@@ -352,8 +359,10 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
     ok = __all_sync(0xffffffffu, mbar_wait(&s_full[w], k & 1, abort_flag));
     if (!ok) break;
     tc_fence_after();
-    int seg, tok0, valid;
-    tile_info(p, i, seg, tok0, valid);
+    int valid = kBN;
+#pragma unroll
+    for (int q = 0; q < kMaxSeg; ++q)
+      if (i == p.seg_last_tile[q]) valid = p.seg_last_valid[q];
 
     // the whole 128-key row of S in registers
     uint32_t s[4][32];
@@ -517,7 +526,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + NST;
-  uint64_t* q_full = kv_empty + NST;
+  uint64_t* v_full = kv_empty + NST;
+  uint64_t* v_empty = v_full + NST;
+  uint64_t* q_full = v_empty + NST;
   uint64_t* s_full = q_full + 1;
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
@@ -534,6 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
     for (int i = 0; i < NST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
@@ -566,10 +579,12 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   } else {
     regs_dec<88>();
     if (warp == 0) {
-      if (lane == 0) producer<HD, NST>(p, smem, q_full, kv_full, kv_empty, abort_flag, q0, head);
+      if (lane == 0) producer<HD, NST>(p, smem, false, q_full, kv_full, kv_empty, abort_flag, q0, head);
     } else if (warp == 1) {
-      mma_issuer<HD, NST>(p, smem, q_full, kv_full, kv_empty, s_full, p_full, pv_done, ck_done, teardown, abort_flag,
+      mma_issuer<HD, NST>(p, smem, q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, pv_done, ck_done, teardown, abort_flag,
                           tmem);
+    } else if (warp == 3) {
+      if (lane == 0) producer<HD, NST>(p, smem, true, nullptr, v_full, v_empty, abort_flag, q0, head);
     }
   }
 
@@ -618,6 +633,10 @@ ispa_status_t dual_attention_bf16_db(const void* q, int64_t n_q, int64_t q_strid
     if (i + 1 == n_local_seg) local_tiles = tiles;
   }
   p.seg_first_tile[n_seg] = tiles;
+  for (int i = 0; i < kMaxSeg; ++i) {
+    p.seg_last_tile[i] = i < n_seg ? p.seg_first_tile[i + 1] - 1 : -1;
+    p.seg_last_valid[i] = i < n_seg ? (int32_t)(segs[i].n_tokens - (int64_t)(p.seg_first_tile[i + 1] - 1 - p.seg_first_tile[i]) * kBN) : kBN;
+  }
   p.n_seg = n_seg;
   p.n_tiles = tiles;
   p.n_local_tiles = local_tiles;
