@@ -63,6 +63,24 @@ def gram_flops(w, rows) -> float:
     return rows * D * (D + 1) + 2.0 * rows * D * D
 
 
+def solve_flops(D: int) -> float:
+    """Algorithmic FLOPs of one absorb solve: Cholesky D^3/3, S = R W 2 D^3 and
+    the two triangular solves with D right-hand sides 2 D^3."""
+    return (1.0 / 3.0 + 4.0) * float(D) ** 3
+
+
+def chunk_roofline_ms(w, peak_tflops: float) -> dict:
+    """Lower bound of each chunk's latency: the tensor-core time of its dense
+    contractions at the peak (every step of a chunk is tensor-bound)."""
+    D = w.d_model
+    proj = 2.0 * w.n_q * D * D
+    local = 4.0 * w.n_q * (w.n_sink + w.n_q) * w.head_dim * w.n_heads
+    full = attn_flops(w)
+    to_ms = lambda f: f / (peak_tflops * 1e12) * 1e3
+    return {"l_layer": to_ms(local + proj), "f_layer": to_ms(full + proj),
+            "warmup_f_layer": to_ms(full + proj + gram_flops(w, w.n_q))}
+
+
 def max_over_ranks(times_ms, world: int, device) -> list:
     """Elementwise max over the ranks of per-rank device times (ms); every rank
     takes the same collective step, and gets the same list back."""
@@ -312,6 +330,9 @@ def run_ours(args, rank, world, device):
                              "breakdown and the value",
                    "parallelism": f"replicas x{world}"},
         "absorb_ms_per_layer": round(float(mean[3]), 4),
+        "absorb_tflops": round(solve_flops(D) / (mean[3] * 1e-3) / 1e12, 3),
+        "chunk_latency_roofline_frac": {k: round(v / lat, 4) for (k, v), lat in zip(
+            chunk_roofline_ms(w, tc_peak).items(), (mean[4], mean[5] + mean[6], mean[0] + mean[1] + mean[2]))},
         "chunk_latency_ms": {"l_layer": round(float(mean[4]), 4),
                              "f_layer": round(float(mean[5] + mean[6]), 4),
                              "warmup_f_layer": round(float(mean[0] + mean[1] + mean[2]), 4)},
