@@ -15,6 +15,9 @@ its section:
   [gist §2.3]  same page, stage 3 "Memory-Efficient Inference" (W_new = W + dW,
                eviction of K_hist, V_hist for the K selected layers)
   [gist §3]    same page, "Key Contributions" item 2 (online-softmax grounding)
+  [gist sel]   same page, "Dynamic Layer Selection" (all layers ranked by
+               their reconstruction error after the warm-up; the lowest are
+               converted to L-layers)
   [abstract]   mlsanity.com arXiv abstract (up to 50% of the KV cache removed)
 
 Everything is plain numpy in float64: attention materialises the score matrix
@@ -31,7 +34,11 @@ argument below):
   * "A" is the concatenated multi-head attention output [n, D], the input of
     the output projection W [D_in, D_out] with y = A @ W;
   * the matrix norm of the objective is Frobenius;
-  * lambda = lambda_abs + lambda_rel * trace(G) / D, G the un-normalised sum.
+  * lambda = lambda_abs + lambda_rel * trace(G) / D, G the un-normalised sum;
+  * a layer's reconstruction error is the relative squared Frobenius error of
+    the absorbed local stream over the warm-up rows,
+    ||A_loc (W + dW) - A_full W||^2 / ||A_full W||^2, and selection takes the
+    K smallest with ties to the lower layer index.
 Pinned by tests/test_oracle.py (closed forms, special cases, a library
 attention routine, brute-force minimisation of the objective, invariants).
 """
@@ -166,6 +173,30 @@ def objective(a_loc, a_full, W, dW, lam: float) -> float:
     a_loc, a_full, W, dW = _f64(a_loc), _f64(a_full), _f64(W), _f64(dW)
     r = a_loc @ (W + dW) - a_full @ W
     return float(np.sum(r * r) + lam * np.sum(dW * dW))
+
+
+def reconstruction_error(a_loc, a_full, W, dW) -> float:
+    """Reconstruction error of one layer after the warm-up [gist sel]: the
+    relative squared Frobenius error of the absorbed local stream,
+    ||A_loc (W + dW) - A_full W||^2 / ||A_full W||^2 (0 when both vanish,
+    +inf when only the denominator does)."""
+    a_loc, a_full, W, dW = _f64(a_loc), _f64(a_full), _f64(W), _f64(dW)
+    target = a_full @ W
+    r = a_loc @ (W + dW) - target
+    num, den = float(np.sum(r * r)), float(np.sum(target * target))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else math.inf
+    return num / den
+
+
+def select_layers(eps: Sequence[float], k: int) -> List[int]:
+    """The k layers converted to L-layers [gist sel]: the k smallest
+    reconstruction errors, ties to the lower layer index, NaN ranked after
+    every number; returned in increasing layer order."""
+    if not 0 <= k <= len(eps):
+        raise ValueError("k must lie in [0, number of layers]")
+    order = sorted(range(len(eps)), key=lambda l: (math.isnan(eps[l]), 0.0 if math.isnan(eps[l]) else eps[l], l))
+    return sorted(order[:k])
 
 
 def modulated_weight(W, dW) -> np.ndarray:

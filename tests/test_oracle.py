@@ -248,6 +248,84 @@ def test_modulated_weight_reconstructs_full_stream_exactly_when_possible():
     assert np.max(np.abs(orc.project(a_loc, W_new) - orc.project(a_full, W))) < 1e-10
 
 
+# ------------------------------------------------------- layer selection
+def test_reconstruction_error_zero_when_streams_agree():
+    a_loc, _, W = _ridge_case(80, 30, 5)
+    G, R = orc.gram(a_loc, a_loc - a_loc)
+    dW = orc.absorb(G, R, W, orc.ridge_lambda(G))
+    assert orc.reconstruction_error(a_loc, a_loc, W, dW) == 0.0
+
+
+def test_reconstruction_error_vanishes_for_exact_linear_history():
+    # A_full = A_loc M: lam -> 0 absorbs the history exactly
+    a_loc = _rand(81, 80, 6)
+    a_full = a_loc @ (np.eye(6) + 0.3 * _rand(82, 6, 6))
+    W = _rand(83, 6, 6)
+    G, R = orc.gram(a_loc, a_full - a_loc)
+    assert orc.reconstruction_error(a_loc, a_full, W, orc.absorb(G, R, W, 0.0)) < 1e-20
+
+
+def test_reconstruction_error_scalar_closed_form():
+    # D = 1, hand-evaluated: dW from the scalar ridge formula, then the ratio
+    a_l = np.array([[1.0], [2.0], [-1.0]])
+    a_f = np.array([[1.5], [1.0], [0.0]])
+    w, lam = 0.7, 0.25
+    dw = w * (1 * 0.5 + 2 * (-1.0) + (-1) * 1.0) / (1 + 4 + 1 + lam)
+    num = sum((al * (w + dw) - af * w) ** 2 for al, af in [(1.0, 1.5), (2.0, 1.0), (-1.0, 0.0)])
+    den = sum((af * w) ** 2 for af in (1.5, 1.0, 0.0))
+    got = orc.reconstruction_error(a_l, a_f, np.array([[w]]), np.array([[dw]]))
+    assert abs(got - num / den) < 1e-14
+
+
+def test_reconstruction_error_limits_and_invariance():
+    a_loc, a_full, W = _ridge_case(84, 50, 6)
+    G, R = orc.gram(a_loc, a_full - a_loc)
+    # lam -> inf: dW -> 0, the error tends to ||dA W||^2 / ||A_full W||^2
+    e_inf = orc.reconstruction_error(a_loc, a_full, W, orc.absorb(G, R, W, 1e12 * np.trace(G)))
+    d = (a_full - a_loc) @ W
+    t = a_full @ W
+    assert abs(e_inf - np.sum(d * d) / np.sum(t * t)) < 1e-9
+    # the ridge minimiser can only lower the error term against dW = 0 as lam -> 0
+    e0 = orc.reconstruction_error(a_loc, a_full, W, orc.absorb(G, R, W, 0.0))
+    assert e0 <= e_inf
+    # scaling W scales dW and both norms alike
+    lam = orc.ridge_lambda(G)
+    e1 = orc.reconstruction_error(a_loc, a_full, W, orc.absorb(G, R, W, lam))
+    e3 = orc.reconstruction_error(a_loc, a_full, 3.0 * W, orc.absorb(G, R, 3.0 * W, lam))
+    assert abs(e1 - e3) < 1e-12 * max(1.0, e1)
+
+
+def test_reconstruction_error_from_statistics():
+    # the closed form the GPU evaluates: with E = dA^T dA,
+    # num = <dW, G dW> - 2 <dW, R W> + <W, E W>, den = <W, (G + R + R^T + E) W>
+    a_loc, a_full, W = _ridge_case(85, 64, 7, 5)
+    dA = a_full - a_loc
+    G, R = orc.gram(a_loc, dA)
+    E = dA.T @ dA
+    dW = orc.absorb(G, R, W, orc.ridge_lambda(G))
+    num = np.sum(dW * (G @ dW)) - 2 * np.sum(dW * (R @ W)) + np.sum(W * (E @ W))
+    den = np.sum(W * ((G + R + R.T + E) @ W))
+    assert abs(orc.reconstruction_error(a_loc, a_full, W, dW) - num / den) < 1e-12
+
+
+def test_select_layers_bruteforce_with_ties():
+    import itertools
+    rng = np.random.default_rng(86)
+    for trial in range(40):
+        n = int(rng.integers(1, 8))
+        eps = list(rng.choice([0.1, 0.2, 0.3, 0.5], size=n))  # many ties
+        if trial % 5 == 0 and n > 1:
+            eps[int(rng.integers(n))] = float("nan")
+        for k in range(n + 1):
+            def key(sub):
+                vals = [math.inf if math.isnan(eps[l]) else eps[l] for l in sub]
+                return (sum(math.isnan(eps[l]) for l in sub), sorted(vals), list(sub))
+            best = min(itertools.combinations(range(n), k), key=key)
+            assert orc.select_layers(eps, k) == list(best), (eps, k)
+    with pytest.raises(ValueError):
+        orc.select_layers([0.1, 0.2], 3)
+
+
 # ---------------------------------------------------------------- bookkeeping
 def test_chunk_token_ranges_closed_form():
     F, cf = 1560, 3
