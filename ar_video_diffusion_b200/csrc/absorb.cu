@@ -382,6 +382,92 @@ ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W,
   return check_launch("absorb_solve");
 }
 
+// ------------------------------------------------------- layer selection
+// Reconstruction error of one layer after the warm-up ("Instance-Specific
+// Parametric Absorption", gist.science technical summary, "Dynamic Layer
+// Selection"), ||A_loc (W + dW) - A_full W||^2 / ||A_full W||^2, from the
+// warm-up statistics alone: with dA = A_full - A_loc, G = A_loc^T A_loc,
+// R = A_loc^T dA, E = dA^T dA,
+//   num = <dW, G dW> - 2 <dW, R W> + <W, E W>,
+//   den = <W, G W> + 2 <W, R W> + <W, E W>,
+// <X, Y> the Frobenius inner product.  Products in fp32, sums in fp64.
+namespace simt {
+
+// out = the symmetric matrix whose lower triangle (row >= col) is that of in
+__global__ void symmetrize_kernel(const float* __restrict__ in, float* __restrict__ out, int D) {
+  const int64_t n = (int64_t)D * D;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e / D), j = (int)(e - (int64_t)i * D);
+    out[e] = i >= j ? in[e] : in[(int64_t)j * D + i];
+  }
+}
+
+// *out += coef * <x, y> (fp64 accumulation)
+template <typename TX>
+__global__ void frob_dot_kernel(const TX* __restrict__ x, const float* __restrict__ y, int64_t n, double coef,
+                                double* __restrict__ out) {
+  __shared__ double part[8];
+  double acc = 0.0;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+    acc += (double)to_f32(x[e]) * (double)y[e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];
+    atomicAdd(out, coef * t);
+  }
+}
+
+}  // namespace simt
+
+size_t layer_error_workspace_bytes(int64_t D) { return (size_t)3 * D * D * sizeof(float); }
+
+template <typename TW>
+static void layer_error_impl(const float* G, const float* R, const float* E, const TW* W, const float* dW, int D,
+                             float* ws, double* num_den, cudaStream_t st) {
+  using namespace simt;
+  const int64_t n = (int64_t)D * D;
+  float* Gs = ws;
+  float* Es = ws + n;
+  float* P = ws + 2 * n;
+  const int sms = num_sms();
+  symmetrize_kernel<<<sms * 4, 256, 0, st>>>(G, Gs, D);
+  symmetrize_kernel<<<sms * 4, 256, 0, st>>>(E, Es, D);
+  cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st);
+  double* num = num_den;
+  double* den = num_den + 1;
+  gemm_f32(st, D, D, D, 1.f, Gs, D, 1, dW, D, 1, 0.f, P, D);  // G dW
+  frob_dot_kernel<float><<<sms * 2, 256, 0, st>>>(dW, P, n, 1.0, num);
+  gemm_f32(st, D, D, D, 1.f, R, D, 1, W, D, 1, 0.f, P, D);  // R W
+  frob_dot_kernel<float><<<sms * 2, 256, 0, st>>>(dW, P, n, -2.0, num);
+  frob_dot_kernel<TW><<<sms * 2, 256, 0, st>>>(W, P, n, 2.0, den);
+  gemm_f32(st, D, D, D, 1.f, Es, D, 1, W, D, 1, 0.f, P, D);  // E W
+  frob_dot_kernel<TW><<<sms * 2, 256, 0, st>>>(W, P, n, 1.0, num);
+  frob_dot_kernel<TW><<<sms * 2, 256, 0, st>>>(W, P, n, 1.0, den);
+  gemm_f32(st, D, D, D, 1.f, Gs, D, 1, W, D, 1, 0.f, P, D);  // G W
+  frob_dot_kernel<TW><<<sms * 2, 256, 0, st>>>(W, P, n, 1.0, den);
+}
+
+ispa_status_t layer_error_launch(const float* G, const float* R, const float* E, const void* W, ispa_dtype_t w_dt,
+                                 const float* dW, int64_t D, void* workspace, double* num_den, cudaStream_t st) {
+  float* ws = static_cast<float*>(workspace);
+  if (w_dt == ISPA_DT_BF16)
+    layer_error_impl(G, R, E, static_cast<const __nv_bfloat16*>(W), dW, (int)D, ws, num_den, st);
+  else
+    layer_error_impl(G, R, E, static_cast<const float*>(W), dW, (int)D, ws, num_den, st);
+  return check_launch("layer_error");
+}
+
+// fp32 path of the symmetric statistics: E (+)= X^T X (every entry written).
+ispa_status_t sym_gram_f32(const float* x, int64_t n_rows, int64_t D, int64_t row_stride, float* E, bool overwrite,
+                           cudaStream_t st) {
+  simt::gemm_f32(st, (int)D, (int)D, (int)n_rows, 1.f, x, 1, row_stride, x, row_stride, 1, overwrite ? 0.f : 1.f, E, D);
+  return check_launch("sym_gram_f32");
+}
+
 // fp32 activation path of the statistics: [G | R] (+)= A_loc^T [A_loc | delta].
 ispa_status_t gram_f32(const float* a_loc, const float* a_delta, int64_t n_rows, int64_t D, int64_t row_stride,
                        float* G, float* R, bool overwrite, cudaStream_t st) {

@@ -1,6 +1,7 @@
 // C ABI of libispa: argument validation and dispatch to the kernels.  Nothing
 // here allocates, frees or synchronises; every launch goes to the caller's
 // stream.  Host bookkeeping of the streaming KV cache lives here too.
+#include <climits>
 #include <cmath>
 #include <cstring>
 
@@ -27,6 +28,13 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
                            const void* w, void* y, cudaStream_t stream);
 ispa_status_t project_f32(const float* a, int64_t n_rows, int64_t d_in, int64_t d_out, int64_t a_stride,
                           const float* w, float* y, cudaStream_t st);
+ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t row_stride, float* E, bool overwrite,
+                            cudaStream_t stream);
+ispa_status_t sym_gram_f32(const float* x, int64_t n_rows, int64_t D, int64_t row_stride, float* E, bool overwrite,
+                           cudaStream_t st);
+size_t layer_error_workspace_bytes(int64_t D);
+ispa_status_t layer_error_launch(const float* G, const float* R, const float* E, const void* W, ispa_dtype_t w_dt,
+                                 const float* dW, int64_t D, void* workspace, double* num_den, cudaStream_t st);
 size_t absorb_workspace_bytes(int64_t D);
 ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D,
                                   double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
@@ -155,6 +163,73 @@ extern "C" ispa_status_t ispa_gram_accumulate(const void* a_loc, const void* a_d
   if (dt == ISPA_DT_BF16) return gram_bf16(a_loc, a_delta, n_rows, d_model, row_stride, G, R, zero_first != 0, s);
   return gram_f32(static_cast<const float*>(a_loc), static_cast<const float*>(a_delta), n_rows, d_model, row_stride,
                   G, R, zero_first != 0, s);
+}
+
+extern "C" ispa_status_t ispa_sym_gram_accumulate(const void* x, int64_t n_rows, int64_t d_model, int64_t row_stride,
+                                                  ispa_dtype_t dt, float* E, int32_t zero_first, void* stream) {
+  if (!valid_dtype(dt)) return unsupported("unknown dtype %d", (int)dt);
+  if (!E) return invalid("E is required");
+  if (n_rows < 0 || d_model <= 0) return invalid("n_rows must be >= 0 and d_model > 0");
+  if (row_stride < d_model) return invalid("row_stride < d_model");
+  if (dt == ISPA_DT_BF16 && d_model % 128) return unsupported("bf16 statistics need d_model % 128 == 0");
+  if (dt == ISPA_DT_F32 && d_model % 4) return unsupported("fp32 statistics need d_model % 4 == 0");
+  if (d_model > 16384 || n_rows > INT32_MAX / 2) return unsupported("problem too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n_rows == 0) {
+    if (!zero_first) return ISPA_OK;
+    cudaMemsetAsync(E, 0, (size_t)d_model * d_model * 4, s);
+    return check_launch("memset");
+  }
+  if (!x) return invalid("x is required");
+  if (!aligned16(x) || !aligned16(E) || (row_stride * elem_bytes(dt)) % 16)
+    return invalid("pointers must be 16-byte aligned");
+  if (dt == ISPA_DT_BF16) return sym_gram_bf16(x, n_rows, d_model, row_stride, E, zero_first != 0, s);
+  return sym_gram_f32(static_cast<const float*>(x), n_rows, d_model, row_stride, E, zero_first != 0, s);
+}
+
+extern "C" size_t ispa_layer_error_workspace_bytes(int64_t d_model) {
+  return d_model > 0 ? layer_error_workspace_bytes(d_model) : 0;
+}
+
+extern "C" ispa_status_t ispa_layer_error(const float* G, const float* R, const float* E, const void* W,
+                                          ispa_dtype_t w_dt, const float* delta_w, int64_t d_model, void* workspace,
+                                          size_t workspace_bytes, double* num_den, void* stream) {
+  if (!valid_dtype(w_dt)) return unsupported("unknown dtype %d", (int)w_dt);
+  if (!G || !R || !E || !W || !delta_w || !workspace || !num_den) return invalid("required pointer is NULL");
+  if (d_model <= 0 || d_model > 16384) return unsupported("d_model must lie in [1, 16384]");
+  if (workspace_bytes < layer_error_workspace_bytes(d_model)) {
+    set_last_error("workspace holds %zu bytes, %zu needed", workspace_bytes, layer_error_workspace_bytes(d_model));
+    return ISPA_ERR_WORKSPACE;
+  }
+  if ((reinterpret_cast<uintptr_t>(num_den) & 7u) != 0) return invalid("num_den must be 8-byte aligned");
+  for (const void* p : {(const void*)G, (const void*)R, (const void*)E, W, (const void*)delta_w,
+                        (const void*)workspace})
+    if (!aligned16(p)) return invalid("matrices must be 16-byte aligned");
+  return layer_error_launch(G, R, E, W, w_dt, delta_w, d_model, workspace, num_den, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, uint8_t* selected) {
+  if (n_layers < 0 || n_layers > 4096) return invalid("n_layers must lie in [0, 4096]");
+  if (k < 0 || k > n_layers) return invalid("k must lie in [0, n_layers]");
+  if (n_layers > 0 && (!eps || !selected)) return invalid("eps and selected are required");
+  // rank: numbers before NaN, increasing value, then increasing layer index
+  int32_t order[4096];
+  for (int32_t l = 0; l < n_layers; ++l) order[l] = l;
+  auto before = [&](int32_t a, int32_t b) {
+    const bool na = std::isnan(eps[a]), nb = std::isnan(eps[b]);
+    if (na != nb) return nb;
+    if (!na && eps[a] != eps[b]) return eps[a] < eps[b];
+    return a < b;
+  };
+  for (int32_t i = 1; i < n_layers; ++i) {  // insertion sort: stable, n_layers is small
+    const int32_t v = order[i];
+    int32_t j = i;
+    for (; j > 0 && before(v, order[j - 1]); --j) order[j] = order[j - 1];
+    order[j] = v;
+  }
+  for (int32_t l = 0; l < n_layers; ++l) selected[l] = 0;
+  for (int32_t i = 0; i < k; ++i) selected[order[i]] = 1;
+  return ISPA_OK;
 }
 
 extern "C" size_t ispa_absorb_workspace_bytes(int64_t d_model) {

@@ -273,6 +273,43 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   return launch<true, true, 128, 4>(p, (int)splits, stream);
 }
 
+// E (+)= X^T X (bf16 input, fp32 output): the lower triangle of a symmetric
+// Gram matrix, with the same kernel, tiling and one-wave K split as gram_bf16
+// but a single column range.
+ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t row_stride, float* E, bool overwrite,
+                            cudaStream_t stream) {
+  using namespace gemm;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  if (!encode_map_bf16_2d(&p.a_map, x, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  p.b_map[0] = p.a_map;
+  p.b_map[1] = p.a_map;
+  if (overwrite) cudaMemsetAsync(E, 0, (size_t)D * D * 4, stream);
+  p.M = (int32_t)D;
+  p.N = (int32_t)D;
+  p.K = (int32_t)n_rows;
+  p.n_split = (int32_t)D;
+  p.lower_only0 = 1;
+  p.c[0] = E;
+  p.c[1] = E;
+  p.ldc = D;
+  p.mode = kReduceF32;
+  const int BN = D % 256 == 0 ? 256 : 128;
+  const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
+  int64_t tiles = 0;
+  for (int64_t i = 0; i < m_tiles; ++i)
+    for (int64_t j = 0; j < n_tiles; ++j) tiles += (j * BN <= i * kBM + kBM - 1) ? 1 : 0;
+  const int64_t k_blocks = (n_rows + kBK - 1) / kBK;
+  int64_t splits = num_sms() / tiles;
+  if (splits > k_blocks / 8) splits = k_blocks / 8;
+  if (splits < 1) splits = 1;
+  const int64_t blocks_per_split = (k_blocks + splits - 1) / splits;
+  p.k_per_split = (int32_t)(blocks_per_split * kBK);
+  splits = (k_blocks + blocks_per_split - 1) / blocks_per_split;
+  if (BN == 256) return launch<true, true, 256, 3>(p, (int)splits, stream);
+  return launch<true, true, 128, 4>(p, (int)splits, stream);
+}
+
 // C[M, N] (= | +=) A[M, K] W[K, N]: bf16 row-major A and W, fp32 C (ldc).
 ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_stride, const void* w, int64_t N,
                                float* c, int64_t ldc, bool accumulate, cudaStream_t stream) {

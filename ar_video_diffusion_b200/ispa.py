@@ -29,7 +29,8 @@ DT_BF16, DT_F32 = 0, 1
 MAX_SEGMENTS = 8
 
 # every symbol declared in include/ispa.h
-EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "ispa_absorb_workspace_bytes",
+EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "ispa_sym_gram_accumulate",
+            "ispa_layer_error_workspace_bytes", "ispa_layer_error", "ispa_select_layers", "ispa_absorb_workspace_bytes",
             "ispa_absorb_solve", "ispa_absorb_solve_noalloc", "ispa_project", "ispa_local_attention_project",
             "ispa_chunk_token_ranges", "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
             "ispa_version")
@@ -64,6 +65,10 @@ def lib() -> ctypes.CDLL:
                                           vp, vp, vp]),
             "ispa_lse_merge": (i32, [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]),
             "ispa_gram_accumulate": (i32, [vp, vp, i64, i64, i64, i32, vp, vp, i32, vp]),
+            "ispa_sym_gram_accumulate": (i32, [vp, i64, i64, i64, i32, vp, i32, vp]),
+            "ispa_layer_error_workspace_bytes": (sz, [i64]),
+            "ispa_layer_error": (i32, [vp, vp, vp, vp, i32, vp, i64, vp, sz, vp, vp]),
+            "ispa_select_layers": (i32, [c.POINTER(f64), i32, i32, c.POINTER(c.c_uint8)]),
             "ispa_absorb_workspace_bytes": (sz, [i64]),
             "ispa_absorb_solve": (i32, [vp, vp, vp, i32, i64, f64, f64, vp, vp, vp, sz, vp, vp]),
             "ispa_absorb_solve_noalloc": (i32, [vp, vp, vp, i32, i64, f64, f64, vp, vp, vp, vp]),
@@ -143,6 +148,24 @@ def ispa_lse_merge(o_loc, lse_loc, o_hist, lse_hist, n_q, n_heads, head_dim, dt,
 def ispa_gram_accumulate(a_loc, a_delta, n_rows, d_model, row_stride, dt, G, R, zero_first, stream):
     _check(lib().ispa_gram_accumulate(a_loc, a_delta, n_rows, d_model, row_stride, dt, G, R, zero_first, stream),
            "ispa_gram_accumulate")
+
+
+def ispa_sym_gram_accumulate(x, n_rows, d_model, row_stride, dt, E, zero_first, stream):
+    _check(lib().ispa_sym_gram_accumulate(x, n_rows, d_model, row_stride, dt, E, zero_first, stream),
+           "ispa_sym_gram_accumulate")
+
+
+def ispa_layer_error_workspace_bytes(d_model: int) -> int:
+    return lib().ispa_layer_error_workspace_bytes(d_model)
+
+
+def ispa_layer_error(G, R, E, W, w_dt, delta_w, d_model, workspace, workspace_bytes, num_den, stream):
+    _check(lib().ispa_layer_error(G, R, E, W, w_dt, delta_w, d_model, workspace, workspace_bytes, num_den, stream),
+           "ispa_layer_error")
+
+
+def ispa_select_layers(eps, n_layers, k, selected):
+    _check(lib().ispa_select_layers(eps, n_layers, k, selected), "ispa_select_layers")
 
 
 def ispa_absorb_workspace_bytes(d_model: int) -> int:
@@ -255,6 +278,36 @@ def gram_accumulate(a_loc: torch.Tensor, a_delta: torch.Tensor, G: torch.Tensor,
     n, D = a_loc.shape
     ispa_gram_accumulate(_dev(a_loc, "a_loc"), _dev(a_delta, "a_delta"), n, D, _row_stride(a_loc, "a_loc"),
                          _dtype_code(a_loc), _dev(G, "G"), _dev(R, "R"), int(zero_first), _stream(stream))
+
+
+def sym_gram_accumulate(x: torch.Tensor, E: torch.Tensor, zero_first: bool = False, stream=None):
+    """E (+)= x^T x, lower triangle (x = A_full - A_loc for the layer selection)."""
+    n, D = x.shape
+    ispa_sym_gram_accumulate(_dev(x, "x"), n, D, _row_stride(x, "x"), _dtype_code(x), _dev(E, "E"), int(zero_first),
+                             _stream(stream))
+
+
+def layer_error(G: torch.Tensor, R: torch.Tensor, E: torch.Tensor, W: torch.Tensor, delta_w: torch.Tensor,
+                workspace: Optional[torch.Tensor] = None, num_den: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Device float64 tensor [num, den]: the layer's reconstruction error is num / den."""
+    D = G.shape[0]
+    if workspace is None:
+        workspace = torch.empty(ispa_layer_error_workspace_bytes(D), dtype=torch.uint8, device=G.device)
+    if num_den is None:
+        num_den = torch.empty(2, dtype=torch.float64, device=G.device)
+    ispa_layer_error(_dev(G, "G"), _dev(R, "R"), _dev(E, "E"), _dev(W, "W"), _dtype_code(W), _dev(delta_w, "delta_w"),
+                     D, _dev(workspace, "workspace"), workspace.numel(), _dev(num_den, "num_den"), _stream(stream))
+    return num_den
+
+
+def select_layers(eps: Sequence[float], k: int) -> List[int]:
+    """Indices (increasing) of the k layers with the smallest error, ties to the lower index."""
+    n = len(eps)
+    arr = (ctypes.c_double * max(n, 1))(*[float(e) for e in eps])
+    sel = (ctypes.c_uint8 * max(n, 1))()
+    ispa_select_layers(arr, n, k, sel)
+    return [l for l in range(n) if sel[l]]
 
 
 def absorb_workspace(d_model: int, device="cuda") -> torch.Tensor:

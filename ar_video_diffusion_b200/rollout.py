@@ -9,7 +9,12 @@ section 2):
     layers selected for absorption accumulate G and R from their rows;
   * transition (stage 2, "Layer Absorb"): each selected layer solves
     dW = (G + lambda I)^-1 R W, forms W_new = W + dW and evicts its history
-    K/V, keeping only the sink frame;
+    K/V, keeping only the sink frame.  The selected layers are either a fixed
+    set (the even layers by default) or, with ``selection="instance"``, the K
+    layers of lowest reconstruction error ("Dynamic Layer Selection" of the
+    same page): every layer then also accumulates E = dA^T dA, is absorbed at
+    the transition and ranked by eps = ||A_loc W_new - A_full W||^2 /
+    ||A_full W||^2, evaluated from G, R, E without its activations;
   * later chunks (stage 3): selected layers (L-layers) attend to sink +
     current only and project with W_new; the others (F-layers) attend to the
     whole growing cache and project with W.
@@ -41,11 +46,23 @@ class ChunkReport:
 class Rollout:
     def __init__(self, w: synth.Workload, absorbed: Optional[Sequence[int]] = None, device="cuda",
                  lambda_rel: float = 1e-2,
-                 on_layer: Optional[Callable[[int, int, dict], None]] = None):
+                 on_layer: Optional[Callable[[int, int, dict], None]] = None,
+                 selection: str = "fixed", rank_all: bool = False):
+        """``absorbed``: the fixed L-layer set (default: even layers); with
+        ``selection="instance"`` only its size K is used and the K layers of
+        lowest reconstruction error are chosen at the transition.
+        ``rank_all``: rank every layer (eps of each) even for a fixed set."""
+        if selection not in ("fixed", "instance"):
+            raise ValueError("selection must be 'fixed' or 'instance'")
         self.w = w
         self.device = torch.device(device)
         self.L = w.n_layers
         self.absorbed = sorted(set(range(0, self.L, 2) if absorbed is None else absorbed))
+        self.selection = selection
+        self.k_select = len(self.absorbed)
+        self.rank = rank_all or selection == "instance"
+        if selection == "instance":
+            self.absorbed = []  # chosen at the transition
         self.mask = 0
         for l in self.absorbed:
             self.mask |= 1 << l
@@ -70,8 +87,12 @@ class Rollout:
             n = warm if l in self.absorbed else full
             self.k.append(torch.empty(n, D, **bf))
             self.v.append(torch.empty(n, D, **bf))
-        self.G = {l: torch.zeros(D, D, **f32) for l in self.absorbed}
-        self.R = {l: torch.zeros(D, D, **f32) for l in self.absorbed}
+        self.stats_layers = list(range(self.L)) if self.rank else list(self.absorbed)
+        self.G = {l: torch.zeros(D, D, **f32) for l in self.stats_layers}
+        self.R = {l: torch.zeros(D, D, **f32) for l in self.stats_layers}
+        self.E = {l: torch.zeros(D, D, **f32) for l in self.stats_layers} if self.rank else {}
+        self.eps: List[float] = []      # reconstruction error of every layer (when ranked)
+        self.select_ms = 0.0
         self.transitioned = False
         n_q = self.chunk_tokens
         self.q = [torch.empty(n_q, D, **bf) for _ in range(self.L)]
@@ -114,19 +135,53 @@ class Rollout:
                 self.v[l][pos:pos + self.F].copy_(v)
 
     # ------------------------------------------------------------ transition
+    def rank_layers(self):
+        """Absorb every layer and evaluate its reconstruction error; with
+        instance selection, choose the K layers of lowest error."""
+        stream = torch.cuda.current_stream(self.device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ws = torch.empty(ispa.ispa_layer_error_workspace_bytes(self.D), dtype=torch.uint8, device=self.device)
+        num_den = torch.empty(self.L, 2, dtype=torch.float64, device=self.device)
+        cand, ev = {}, {}
+        e0.record(stream)
+        for l in range(self.L):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            dW, Wn = ispa.absorb_solve(self.G[l], self.R[l], self.W[l], lambda_rel=self.lambda_rel,
+                                       workspace=self.workspace, status=self.status)
+            a1.record(stream)
+            ispa.layer_error(self.G[l], self.R[l], self.E[l], self.W[l], dW, workspace=ws, num_den=num_den[l])
+            cand[l], ev[l] = (dW, Wn), (a0, a1)
+        e1.record(stream)
+        torch.cuda.synchronize(self.device)
+        self.select_ms = e0.elapsed_time(e1)  # every layer's absorb and error
+        nd = num_den.cpu().tolist()
+        self.eps = [n / d if d > 0 else float("nan") for n, d in nd]
+        if self.selection == "instance":
+            self.absorbed = ispa.select_layers(self.eps, self.k_select)
+            self.mask = 0
+            for l in self.absorbed:
+                self.mask |= 1 << l
+        for l in self.absorbed:
+            self.dW[l], self.W_new[l] = cand[l]
+        self.absorb_ms = [ev[l][0].elapsed_time(ev[l][1]) for l in self.absorbed]
+
     def transition(self):
         """Absorb the history of every selected layer and evict its K/V."""
         stream = torch.cuda.current_stream(self.device)
         sink = self.w.sink_frames * self.F
         events = []
+        if self.rank:
+            self.rank_layers()
         for l in self.absorbed:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            dW, Wn = ispa.absorb_solve(self.G[l], self.R[l], self.W[l], lambda_rel=self.lambda_rel,
-                                       workspace=self.workspace, status=self.status)
+            if not self.rank:
+                dW, Wn = ispa.absorb_solve(self.G[l], self.R[l], self.W[l], lambda_rel=self.lambda_rel,
+                                           workspace=self.workspace, status=self.status)
+                self.dW[l], self.W_new[l] = dW, Wn
             e1.record(stream)
             events.append((e0, e1))
-            self.dW[l], self.W_new[l] = dW, Wn
             # keep the sink frame, drop the history: a buffer for sink + one chunk
             k_small = torch.empty(sink + self.chunk_tokens, self.D, dtype=torch.bfloat16, device=self.device)
             v_small = torch.empty_like(k_small)
@@ -134,10 +189,12 @@ class Rollout:
             v_small[:sink].copy_(self.v[l][:sink])
             self.k[l], self.v[l] = k_small, v_small
         torch.cuda.synchronize(self.device)
-        self.absorb_ms = [a.elapsed_time(b) for a, b in events]
+        if not self.rank:
+            self.absorb_ms = [a.elapsed_time(b) for a, b in events]
         self.transitioned = True
         self.G.clear()
         self.R.clear()
+        self.E.clear()
 
     # ----------------------------------------------------------------- chunk
     def run_chunk(self, c: int):
@@ -163,9 +220,11 @@ class Rollout:
                     if r["hist"][1] > r["hist"][0] else []
                 if warm:
                     ispa.dual_attention(self.q[l], local, hist, H, out=self.out, status=self.status)
-                    if l in self.absorbed:
+                    if l in self.G:
                         ispa.gram_accumulate(self.out["a_loc"], self.out["a_delta"], self.G[l], self.R[l],
                                              zero_first=(c == 0))
+                        if self.rank:
+                            ispa.sym_gram_accumulate(self.out["a_delta"], self.E[l], zero_first=(c == 0))
                 else:
                     ispa.dual_attention(self.q[l], local, hist, H, dual=False, out=self.out, status=self.status)
                 ispa.project(self.out["a_full"], self.W[l], self.y)

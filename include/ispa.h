@@ -137,6 +137,51 @@ ISPA_API ispa_status_t ispa_gram_accumulate(const void* a_loc, const void* a_del
                                    int64_t row_stride, ispa_dtype_t dt, float* G, float* R, int32_t zero_first,
                                    void* stream);
 
+/*
+ * ispa_sym_gram_accumulate -- E += x^T x for the instance-specific layer
+ * selection ("Dynamic Layer Selection" of the gist.science technical summary):
+ * with x = A_full - A_loc over the warm-up rows, E completes, together with
+ * G and R of ispa_gram_accumulate, the statistics from which a layer's
+ * reconstruction error follows without storing its activations.
+ * x [n_rows, d_model], dtype dt, row stride row_stride elements; E
+ * [d_model, d_model] fp32 row-major, accumulated in place (zero_first != 0
+ * overwrites).  Only the lower triangle of E (row >= col) is guaranteed.
+ * d_model must be a multiple of 128 (bf16) or 4 (fp32).  n_rows == 0 is a
+ * no-op (or a zero fill when zero_first != 0).
+ */
+ISPA_API ispa_status_t ispa_sym_gram_accumulate(const void* x, int64_t n_rows, int64_t d_model, int64_t row_stride,
+                                                ispa_dtype_t dt, float* E, int32_t zero_first, void* stream);
+
+/* Bytes of device workspace ispa_layer_error needs for d_model (3 d^2 floats). */
+ISPA_API size_t ispa_layer_error_workspace_bytes(int64_t d_model);
+
+/*
+ * ispa_layer_error -- reconstruction error of one layer after the warm-up
+ * ("Dynamic Layer Selection": all layers are ranked by it and the lowest are
+ * converted to L-layers).  The error is read as the relative squared
+ * Frobenius error of the absorbed local stream over the warm-up rows,
+ *   eps = ||A_loc (W + dW) - A_full W||^2 / ||A_full W||^2,
+ * evaluated from the statistics: with dA = A_full - A_loc, G = A_loc^T A_loc,
+ * R = A_loc^T dA, E = dA^T dA (lower triangles of G and E are read),
+ *   num_den[0] = <dW, G dW> - 2 <dW, R W> + <W, E W>,
+ *   num_den[1] = <W, G W> + 2 <W, R W> + <W, E W>,
+ * and eps = num_den[0] / num_den[1].  G, R, E, delta_w fp32 [D, D]; W [D, D]
+ * in w_dt; num_den: two device doubles (8-byte aligned), overwritten.  fp32
+ * products, fp64 sums.  workspace: at least ispa_layer_error_workspace_bytes
+ * bytes, 16-byte aligned.  Asynchronous on `stream`.
+ */
+ISPA_API ispa_status_t ispa_layer_error(const float* G, const float* R, const float* E, const void* W,
+                                        ispa_dtype_t w_dt, const float* delta_w, int64_t d_model, void* workspace,
+                                        size_t workspace_bytes, double* num_den, void* stream);
+
+/*
+ * ispa_select_layers -- host bookkeeping of the layer selection: selected[l]
+ * = 1 for the k layers with the smallest eps[l] (host array of n_layers
+ * doubles), ties to the lower layer index, NaN ranked after every number;
+ * 0 elsewhere.  0 <= k <= n_layers <= 4096.
+ */
+ISPA_API ispa_status_t ispa_select_layers(const double* eps, int32_t n_layers, int32_t k, uint8_t* selected);
+
 /* Bytes of device workspace ispa_absorb_solve needs for d_model. */
 ISPA_API size_t ispa_absorb_workspace_bytes(int64_t d_model);
 

@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from ar_video_diffusion_b200 import build as ispa_build
@@ -90,3 +92,33 @@ def test_kv_bytes_bit_exact(L):
                 assert ispa.ispa_kv_bytes(chunk, 30, m, trans, 1560, 3, 1536, 2) == \
                     orc.kv_bytes(chunk, 30, m, trans, 1560, 3, 1536, 2)
     assert ispa.ispa_kv_bytes(23, 30, mask, True, 1560, 3, 1536, 2) == 15 * 112320 * 6144 + 15 * 6240 * 6144
+
+
+def test_layer_selection_host_logic_bit_exact(L):
+    # the library's selection against the oracle's on random errors with ties and NaN
+    rng = np.random.default_rng(91)
+    for trial in range(200):
+        n = int(rng.integers(0, 40))
+        eps = [float(x) for x in rng.choice([0.01, 0.02, 0.05, 0.3, 1.0, 2.5], size=n)]
+        for j in range(n):
+            if rng.random() < 0.1:
+                eps[j] = float("nan")
+        k = int(rng.integers(0, n + 1))
+        assert ispa.select_layers(eps, k) == orc.select_layers(eps, k), (eps, k)
+
+
+def test_layer_selection_entry_points_reject_before_launch(L):
+    arr = (ctypes.c_double * 4)(0.1, 0.2, 0.3, 0.4)
+    sel = (ctypes.c_uint8 * 4)()
+    assert L.ispa_select_layers(arr, 4, 5, sel) == 1     # k > n_layers
+    assert L.ispa_select_layers(arr, -1, 0, sel) == 1
+    assert L.ispa_select_layers(None, 4, 2, sel) == 1
+    # layer error: NULL matrix, short workspace, unsupported dtype
+    p = ctypes.c_void_p(256)
+    assert L.ispa_layer_error(None, p, p, p, 0, p, 128, p, 1 << 20, p, None) == 1
+    assert L.ispa_layer_error(p, p, p, p, 0, p, 128, p, 16, p, None) == 6
+    assert L.ispa_layer_error(p, p, p, p, 9, p, 128, p, 1 << 20, p, None) == 2
+    assert ispa.ispa_layer_error_workspace_bytes(1536) == 3 * 1536 * 1536 * 4
+    # symmetric statistics: bf16 needs d_model % 128 == 0; NULL E
+    assert L.ispa_sym_gram_accumulate(p, 10, 96, 96, 0, p, 0, None) == 2
+    assert L.ispa_sym_gram_accumulate(p, 10, 128, 128, 0, None, 0, None) == 1
