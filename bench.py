@@ -441,6 +441,36 @@ def run_rollout(device) -> dict:
     }
     del ro
     torch.cuda.empty_cache()
+    res["layer_selection"] = run_layer_selection(device)
+    return res
+
+
+def run_layer_selection(device) -> dict:
+    """The same 30 layers through the warm-up with every layer accumulating
+    G, R and E, then the instance-specific choice of K = 15 layers by
+    reconstruction error (all 30 absorbed and ranked), against the fixed
+    even-layer set on the same errors."""
+    import dataclasses
+    from ar_video_diffusion_b200 import ispa
+    from ar_video_diffusion_b200.rollout import Rollout
+    w = dataclasses.replace(synth.WORKLOADS["rollout"], post_chunks=0)
+    ro = Rollout(w, device=device, selection="instance")
+    ro.run()
+    ro.transition()
+    even = list(range(0, w.n_layers, 2))
+    eps = ro.eps
+    res = {
+        "workload": "30 layers, 1.3B shapes, 4 warm-up chunks; K = 15 of 30 chosen by reconstruction error",
+        "selected": ro.absorbed,
+        "eps": [round(e, 6) for e in eps],
+        "eps_sum_selected": round(sum(eps[l] for l in ro.absorbed), 6),
+        "eps_sum_even_layers": round(sum(eps[l] for l in even), 6),
+        "rank_ms_all_layers": round(ro.select_ms, 3),
+        "rank_ms_per_layer": round(ro.select_ms / w.n_layers, 4),
+    }
+    assert ro.absorbed == ispa.select_layers(eps, len(even))
+    del ro
+    torch.cuda.empty_cache()
     return res
 
 
