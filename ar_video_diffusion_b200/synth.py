@@ -83,6 +83,10 @@ WORKLOADS: Dict[str, Workload] = {
     "long_hist": Workload("long_hist", seed=2, n_heads=12, head_dim=128, frame_tokens=1560,
                           sink_frames=1, chunk_frames=3, hist_frames=60, dtype="bf16",
                           warm_chunks=20),
+    # a long-lived F-layer: 129 latent frames (201240 tokens) of history
+    "hist_200k": Workload("hist_200k", seed=5, n_heads=12, head_dim=128, frame_tokens=1560,
+                          sink_frames=1, chunk_frames=3, hist_frames=129, dtype="bf16",
+                          warm_chunks=1),
     "wan14b": Workload("wan14b", seed=3, n_heads=40, head_dim=128, frame_tokens=1560,
                        sink_frames=1, chunk_frames=3, hist_frames=12, dtype="bf16",
                        warm_chunks=4),

@@ -302,6 +302,7 @@ def run_ours(args, rank, world, device):
 
     # standalone LSE merge over rotating buffer sets larger than L2
     merge_gbs = merge_bench(ispa, w, device)
+    long_hist = long_history_bench(ispa, device)
 
     rollout = None if args.no_rollout else run_rollout(device)
 
@@ -354,6 +355,7 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": d2h},
         "clocks": clk,
         "gpu_launches": args.steps * (7 + absorb_launches(D)),
+        "long_history": long_hist,
         "rollout": rollout,
     }
     return res
@@ -470,6 +472,52 @@ def run_layer_selection(device) -> dict:
     }
     assert ro.absorbed == ispa.select_layers(eps, len(even))
     del ro
+    torch.cuda.empty_cache()
+    return res
+
+
+def long_history_bench(ispa, device, iters=5) -> dict:
+    """A long-lived F-layer: the dual-stream and the single-pass attention of
+    one 4680-query chunk over 129 latent frames (201240 tokens) of history,
+    K/V drawn by the device generator, timed as CUDA-graph replays."""
+    w = synth.WORKLOADS["hist_200k"]
+    F, D, H = w.frame_tokens, w.d_model, w.n_heads
+    n_frames = w.sink_frames + w.hist_frames + w.chunk_frames
+    k = torch.empty(n_frames * F, D, dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    for f in range(n_frames):
+        kf, vf = synth.frame_kv_device(w, 0, f, device)
+        k[f * F:(f + 1) * F].copy_(kf)
+        v[f * F:(f + 1) * F].copy_(vf)
+    q = synth.chunk_q_device(w, 0, 1, device)
+    s, h = w.n_sink, w.n_sink + w.n_hist
+    local = [(k[:s], v[:s]), (k[h:], v[h:])]
+    hist = [(k[s:h], v[s:h])]
+    status = ispa.new_status(device)
+    out = ispa.dual_attention(q, local, hist, H, status=status)
+    fout = ispa.dual_attention(q, local, hist, H, dual=False, status=status)
+    res = {"n_hist": w.n_hist, "n_keys": w.n_sink + w.n_hist + w.n_q}
+    side = torch.cuda.Stream(device)
+    stream = torch.cuda.current_stream(device)
+    for name, fn in (("dual", lambda: ispa.dual_attention(q, local, hist, H, out=out, status=status)),
+                     ("full", lambda: ispa.dual_attention(q, local, hist, H, dual=False, out=fout, status=status))):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+            fn()
+        g.replay()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / iters
+        res[name + "_ms"] = round(ms, 4)
+        res[name + "_tflops"] = round(attn_flops(w) / (ms * 1e-3) / 1e12, 1)
+    if int(status[0].item()) != 0:
+        raise RuntimeError("device status during the long-history benchmark")
+    del k, v
     torch.cuda.empty_cache()
     return res
 

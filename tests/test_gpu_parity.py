@@ -338,6 +338,28 @@ def test_long_history_layer_sampled_rows_and_gram():
     _check_gram_entries(A, Dl, G, R, 64, 23)
 
 
+def test_history_200k_dual_and_single_pass_sampled_rows():
+    """A long-lived F-layer: 201240 history tokens (129 latent frames), 1572
+    key tiles per query tile.  64 query rows of the dual-stream outputs and of
+    the single-pass (F-layer) outputs against the oracle."""
+    w = synth.WORKLOADS["hist_200k"]
+    x, out = _layer_outputs(w)
+    _check_sampled_rows(w, x, out, 64, 41)
+    status = ispa.new_status()
+    full = ispa.dual_attention(dev(x["q"], "bf16"), [(dev(x["k_sink"], "bf16"), dev(x["v_sink"], "bf16")),
+                                                    (dev(x["k_cur"], "bf16"), dev(x["v_cur"], "bf16"))],
+                               [(dev(x["k_hist"], "bf16"), dev(x["v_hist"], "bf16"))], w.n_heads, dual=False,
+                               status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "dual_attention")
+    # the single pass computes exactly the dual stream's fused A_full
+    rows = np.sort(np.random.default_rng(42).choice(w.n_q, 64, replace=False))
+    ref = orc.dual_stream(x["q"][rows], [(x["k_sink"], x["v_sink"]), (x["k_cur"], x["v_cur"])],
+                          [(x["k_hist"], x["v_hist"])], w.n_heads)
+    assert max_rel(host(full["a_full"])[rows], ref["a_full"]) <= ATTN_MAX_REL
+    assert max_abs(host(full["lse_full"])[:, rows], ref["lse_full"]) <= LSE_ABS
+
+
 def test_wan14b_layer_sampled_rows_statistics_and_absorb():
     """Wan-14B-shaped layer (40 heads, D = 5120): sampled attention rows, the
     statistics of 4 warm-up chunks (18720 rows) entry by entry, and the
