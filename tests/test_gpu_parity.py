@@ -55,14 +55,16 @@ def _check_dual(got, ref, rows=None, dual=True):
 
 # (seed, n_q, H, d, local segment lengths, history segment lengths)
 DUAL_CASES = [
-    (1, 300, 2, 128, [100, 300], [700]),        # ragged everywhere, slot A continues into history
+    (1, 300, 2, 128, [100, 300], [700]),        # ragged everywhere; even number of local tiles
     (2, 130, 3, 64, [16, 64], [256]),           # head_dim 64
-    (3, 257, 2, 128, [128, 256], [128]),        # history shorter than local (slot B only)
+    (3, 257, 2, 128, [128, 256], [128]),        # odd local tiles, one history tile: warpgroup 0 has no
+                                                # history tile and takes its checkpoint after its loop
     (4, 200, 1, 128, [1560 // 8, 4680 // 8], []),  # no history at all
     (5, 1, 2, 128, [1], [5]),                  # one query row, one local key
     (6, 129, 2, 128, [3, 200, 17], [64, 1, 300, 129]),  # many segments, tiny ones
     (7, 64, 2, 64, [16, 64], [0, 256]),         # an empty history segment is ignored
     (8, 390, 4, 128, [200, 390], [2500]),       # long history
+    (9, 77, 2, 128, [50], []),                  # a single key tile: warpgroup 1 owns no tile
 ]
 
 
@@ -74,7 +76,7 @@ def test_dual_attention_bf16_matches_oracle(seed, n_q, H, d, loc, his):
     _check_dual(got, ref)
 
 
-@pytest.mark.parametrize("seed,n_q,H,d,loc,his", DUAL_CASES[:3] + DUAL_CASES[5:6])
+@pytest.mark.parametrize("seed,n_q,H,d,loc,his", DUAL_CASES[:3] + DUAL_CASES[5:6] + DUAL_CASES[8:9])
 def test_single_pass_attention_bf16_matches_oracle(seed, n_q, H, d, loc, his):
     case = synth.random_case(seed, n_q, H, d, loc + his, dtype="bf16")
     got = _run_dual(case, len(loc), H, "bf16", dual=False)
