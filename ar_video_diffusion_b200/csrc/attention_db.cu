@@ -28,7 +28,9 @@
 // warpgroups' register budget is raised with setmaxnreg) and writes the bf16
 // P into the first 64 columns of its S buffer.  Online softmax in the log2
 // domain with a lazily updated maximum: O_w is rescaled only when the
-// running maximum grows by more than 2^8.
+// running maximum grows by more than 2^16 (P <= 2^16 is exact-range in bf16
+// and keeps the fp32 sums far from overflow; relative precision does not
+// depend on the scale).
 // Dual mode: before its first history tile each warpgroup takes a local
 // checkpoint; warpgroup 0 merges both accumulators and writes A_loc, LSE_loc,
 // and both restart; the epilogue fuses the history result with A_loc
@@ -46,7 +48,7 @@ constexpr int kBM = 128;       // query rows per CTA (= tensor-memory lanes)
 constexpr int kBN = 128;       // keys per tile
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kMaxSeg = ISPA_MAX_SEGMENTS;
-constexpr float kRescaleLog2 = 8.0f;
+constexpr float kRescaleLog2 = 16.0f;  // lazy rescale threshold (log2)
 constexpr float kLn2 = 0.69314718055994530942f;
 // tensor-memory column map
 constexpr uint32_t kTmS = 0;    // S buffers at 0 and 128
@@ -411,7 +413,7 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
       return fmax3(a, b, c) * sl2;  // -inf if all masked
     };
     // exponentials with the running maximum straight away, the tile maximum
-    // alongside; a growth beyond 2^8 (rare, and always at the start of an
+    // alongside; a growth beyond 2^16 (rare, and always at the start of an
     // accumulation) rescales what was accumulated and redoes the tile.  O_w
     // is quiescent here: S(i) was issued after this warpgroup's previous
     // product, and its completion implies that product's.
