@@ -51,8 +51,8 @@ constexpr int kMaxSeg = ISPA_MAX_SEGMENTS;
 constexpr float kRescaleLog2 = 16.0f;  // lazy rescale threshold (log2)
 constexpr float kLn2 = 0.69314718055994530942f;
 // tensor-memory column map
-constexpr uint32_t kTmS = 0;    // S buffers at 0 and 128
-constexpr uint32_t kTmO = 256;  // O accumulators: half h at kTmO + h * head_dim
+constexpr uint32_t kTmS = 0;    // S buffers: warpgroup w at kTmS + 128 w
+constexpr uint32_t kTmO = 256;  // O accumulators: warpgroup w at kTmO + w * head_dim
 // bit j set: column pair j (mod 8) of a score row takes 2^x from the FMA-pipe
 // polynomial (exp2_fma2) instead of the special-function unit
 constexpr uint32_t kEmuPairs = 0x00u;
