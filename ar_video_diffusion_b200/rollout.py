@@ -233,6 +233,33 @@ class Rollout:
                 info.update(q=self.q[l], y=self.y, out=self.out)
                 self.on_layer(l, c, info)
 
+    def chunk_graph_ms(self, c: int, iters: int = 5) -> float:
+        """Device time of chunk c's launches (every layer's attention and
+        projection) captured into one CUDA graph and replayed: the chunk
+        latency without host launch gaps.  Chunk c's key ranges are used with
+        whatever the caches hold, which does not change the work."""
+        if self.on_layer is not None:
+            raise RuntimeError("chunk graphs need on_layer=None")
+        if c < self.w.warm_chunks or not self.transitioned:
+            raise ValueError("only post-transition chunks are captured")
+        stream = torch.cuda.current_stream(self.device)
+        self.run_chunk(c)  # every first-call set-up happens outside the capture
+        torch.cuda.synchronize(self.device)
+        side = torch.cuda.Stream(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+            self.run_chunk(c)
+        g.replay()
+        torch.cuda.synchronize(self.device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(self.device)
+        del g
+        return e0.elapsed_time(e1) / iters
+
     def run(self, on_chunk_start: Optional[Callable[[int], None]] = None) -> List[ChunkReport]:
         stream = torch.cuda.current_stream(self.device)
         for c in range(self.n_chunks):

@@ -429,12 +429,21 @@ def run_rollout(device) -> dict:
     for l in range(w.n_layers):
         n_k = (w.sink_frames * F_tok + w.n_q) if l in ro.absorbed else n_k_f
         flops_last += 4.0 * w.n_q * n_k * w.head_dim * w.n_heads + 2.0 * w.n_q * w.d_model ** 2
+    # the first and the last post-transition chunk again, each as one CUDA graph
+    g_first = ro.chunk_graph_ms(w.warm_chunks)
+    g_last = ro.chunk_graph_ms(last.chunk)
+    if int(ro.status[0].item()) != 0:
+        raise RuntimeError("device status during the chunk graphs")
     res = {
         "workload": "rollout: 30 layers, 1.3B shapes, 4 warm-up + 20 post-transition chunks, even layers absorbed",
         "chunk_ms": [round(r.gpu_ms, 3) for r in reps],
         "warmup_chunk_ms_mean": round(sum(r.gpu_ms for r in warm) / len(warm), 3),
         "post_chunk_ms_first": round(post[0].gpu_ms, 3),
         "post_chunk_ms_last": round(post[-1].gpu_ms, 3),
+        "post_chunk_graph_ms_first": round(g_first, 3),
+        "post_chunk_graph_ms_last": round(g_last, 3),
+        "post_chunk_graph_tflops_last": round(flops_last / (g_last * 1e-3) / 1e12, 1),
+        "post_chunk_graph_roofline_frac_last": round(flops_last / (peaks()[0]["bf16_tflops"] * 1e12) * 1e3 / g_last, 4),
         "last_chunk_tflops": round(flops_last / (last.gpu_ms * 1e-3) / 1e12, 1),
         "absorb_ms_per_layer": round(sum(ro.absorb_ms) / len(ro.absorb_ms), 4),
         "kv_bytes_last": last.kv_bytes,
