@@ -122,3 +122,27 @@ def test_layer_selection_entry_points_reject_before_launch(L):
     # symmetric statistics: bf16 needs d_model % 128 == 0; NULL E
     assert L.ispa_sym_gram_accumulate(p, 10, 96, 96, 0, p, 0, None) == 2
     assert L.ispa_sym_gram_accumulate(p, 10, 128, 128, 0, None, 0, None) == 1
+
+
+def test_segment_limit_and_empty_queries_rejected_before_launch(L):
+    seg_t = ispa.KVSegment
+    p = 256  # aligned fake device address: validation runs before any launch
+    def segs(n, tokens=16):
+        arr = (seg_t * max(n, 1))()
+        for i in range(n):
+            arr[i] = seg_t(p, p, tokens, 128)
+        return arr
+    q = ctypes.c_void_p(p)
+    out = ctypes.c_void_p(p)
+    # 4 local + 5 history non-empty segments: one more than ISPA_MAX_SEGMENTS
+    r = L.ispa_dual_attention(q, 10, 128, 1, 128, 0, 0.0, segs(4), 4, segs(5), 5, out, out, None, None, None, None,
+                              None)
+    assert r == 2 and "segments" in L.ispa_last_error().decode()
+    # no query rows
+    r = L.ispa_dual_attention(q, 0, 128, 1, 128, 0, 0.0, segs(1), 1, segs(1), 1, out, out, None, None, None, None,
+                              None)
+    assert r == 1
+    # dual mode with an empty local set
+    r = L.ispa_dual_attention(q, 10, 128, 1, 128, 0, 0.0, segs(1, 0), 1, segs(1), 1, out, out, None, None, None, None,
+                              None)
+    assert r == 1 and "local" in L.ispa_last_error().decode()

@@ -65,6 +65,7 @@ DUAL_CASES = [
     (7, 64, 2, 64, [16, 64], [0, 256]),         # an empty history segment is ignored
     (8, 390, 4, 128, [200, 390], [2500]),       # long history
     (9, 77, 2, 128, [50], []),                  # a single key tile: warpgroup 1 owns no tile
+    (10, 140, 2, 128, [10, 130, 30, 40], [50, 129, 70, 1]),  # the maximum of 8 segments
 ]
 
 
