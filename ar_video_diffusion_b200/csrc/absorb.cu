@@ -146,76 +146,146 @@ __global__ void shift_kernel(const float* __restrict__ G, float* __restrict__ M,
 
 // Factor the 64 x 64 diagonal block k of M in place (lower triangle) and
 // write the inverse of its Cholesky factor to Linv (64 x 64, row-major).
-// Column by column: at step j the pivot is square-rooted, column j of L is
-// scaled, the trailing lower triangle gets the rank-1 update, and the same
-// elimination is applied to X (initially I), which ends as L^-1.  Thread t
-// keeps column t % 64 of rows t / 64 + 4 a (a = 0..15) of A and of X in
-// registers; only column j of A and row j of X go through shared memory.  The
-// column loop is unrolled so that the register holding row j is static.
+// Blocked by 16: each 16 x 16 diagonal block is factored by one warp in
+// registers (a row per lane, pivots and columns exchanged with shuffles) and
+// inverted column by column by the same warp; the CTA then forms the 16-column
+// panel below, L_ik = A_ik L_kk^-T, and the rank-16 update of the trailing
+// lower triangle from shared memory.  The off-diagonal blocks of L^-1 follow
+// from X_ik = -X_ii sum_{j=k}^{i-1} L_ij X_jk, one block diagonal at a time.
+// A pivot <= 0 or non-finite records ISPA_ERR_NOT_SPD and its row; the
+// factorisation then continues with the pivot replaced by 1.
+constexpr int kSub = 16;
+
 __global__ void __launch_bounds__(256) potrf_diag_kernel(float* M, int D, int k, float* Linv, int32_t* status) {
-  __shared__ float colbuf[2][kT];  // column j of the current A, double-buffered by the parity of j
-  __shared__ float rowx[kT];  // row j of the current X (already scaled)
+  __shared__ float A[kT][kT + 1];  // the block, then L (lower triangle)
+  __shared__ float X[kT][kT + 1];  // L^-1 (lower triangle, zero above)
+  __shared__ float T[3][kSub][kSub + 1];
   __shared__ int bad;
-  const int tid = threadIdx.x;
-  const int c = tid & 63, r0 = tid >> 6;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float* blk = M + (int64_t)k * kT * D + (int64_t)k * kT;
-  float a[16], x[16];
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const int i = r0 + 4 * t;
-    a[t] = blk[(int64_t)i * D + c];
-    x[t] = (i == c) ? 1.f : 0.f;
+  for (int e = tid; e < kT * kT; e += 256) {
+    const int i = e >> 6, j = e & 63;
+    A[i][j] = blk[(int64_t)i * D + j];
+    X[i][j] = 0.f;
   }
   if (tid == 0) bad = -1;
-#pragma unroll
-  for (int j = 0; j < kT; ++j) {
-    // step j writes column j while slower threads may still read column j-1
-    float* colj = colbuf[j & 1];
-    if (c == j) {
-#pragma unroll
-      for (int t = 0; t < 16; ++t) colj[r0 + 4 * t] = a[t];
-    }
-    __syncthreads();
-    float d = colj[j];
-    if (!(d > 0.f) || !isfinite(d)) {
-      if (tid == 0 && bad < 0) bad = j;
-      d = 1.f;
-    }
-    const float ljj = sqrtf(d);
-    const float inv = 1.0f / ljj;
-    if (r0 == (j & 3)) {  // owner of row j of X
-      x[j >> 2] *= inv;
-      rowx[c] = x[j >> 2];
-    }
-    if (c == j) {  // this column becomes column j of L
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const int i = r0 + 4 * t;
-        a[t] = (i == j) ? ljj : (i > j ? a[t] * inv : a[t]);
-      }
-    }
-    __syncthreads();
-    const float lcj = colj[c] * inv;  // L[c][j] for c > j
-    const float xjc = rowx[c];        // X[j][c]
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int i = r0 + 4 * t;
-      if (i > j) {
-        const float lij = colj[i] * inv;
-        if (c > j && c <= i) a[t] -= lij * lcj;
-        x[t] -= lij * xjc;
-      }
-    }
-  }
   __syncthreads();
+#pragma unroll 1
+  for (int kb = 0; kb < kT / kSub; ++kb) {
+    const int o = kSub * kb;
+    if (warp == 0) {
+      // (a) factor the diagonal block: lane r (and r + 16, a duplicate) holds row r
+      const int r = lane & (kSub - 1);
+      float a[kSub];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) a[c] = (c <= r) ? A[o + r][o + c] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kSub; ++j) {
+        float d = __shfl_sync(0xffffffffu, a[j], j);
+        if (!(d > 0.f) || !isfinite(d)) {
+          if (lane == 0 && bad < 0) bad = o + j;
+          d = 1.f;
+        }
+        const float ljj = sqrtf(d);
+        const float inv = 1.0f / ljj;
+        a[j] = (r == j) ? ljj : (r > j ? a[j] * inv : 0.f);
+#pragma unroll
+        for (int c = 1; c < kSub; ++c) {  // constant trip count: every index stays static
+          if (c > j) {
+            const float lcj = __shfl_sync(0xffffffffu, a[j], c);  // L[c][j], held by lane c
+            if (r >= c) a[c] -= a[j] * lcj;
+          }
+        }
+      }
+      if (lane < kSub) {
+#pragma unroll
+        for (int c = 0; c < kSub; ++c)
+          if (c <= r) A[o + r][o + c] = a[c];
+      }
+      __syncwarp();
+      // its inverse: lane c solves L x = e_c by forward substitution
+      if (lane < kSub) {
+        const int c = lane;
+        float x[kSub];
+#pragma unroll
+        for (int rr = 0; rr < kSub; ++rr) {
+          float acc = (rr == c) ? 1.f : 0.f;
+#pragma unroll
+          for (int m = 0; m < rr; ++m) acc -= A[o + rr][o + m] * x[m];
+          x[rr] = (rr < c) ? 0.f : acc / A[o + rr][o + rr];
+        }
+#pragma unroll
+        for (int rr = 0; rr < kSub; ++rr)
+          if (rr >= c) X[o + rr][o + c] = x[rr];
+      }
+    }
+    __syncthreads();
+    // (b) panel: L[i][o + c] = sum_{m <= c} A[i][o + m] X[o + c][o + m] for rows i below the block
+    const int rows = kT - o - kSub;
+    float pv[3];  // at most 48 x 16 panel entries over 256 threads
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + 256 * q;
+      pv[q] = 0.f;
+      if (e < rows * kSub) {
+        const int i = o + kSub + e / kSub, c = e % kSub;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < kSub; ++m)
+          if (m <= c) acc += A[i][o + m] * X[o + c][o + m];
+        pv[q] = acc;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + 256 * q;
+      if (e < rows * kSub) A[o + kSub + e / kSub][o + e % kSub] = pv[q];
+    }
+    __syncthreads();
+    // (c) trailing lower triangle: A[i][j] -= sum_c L[i][o + c] L[j][o + c], o + 16 <= j <= i
+    for (int e = tid; e < rows * rows; e += 256) {
+      const int i = o + kSub + e / rows, j = o + kSub + e % rows;
+      if (j > i) continue;
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) acc += A[i][o + c] * A[j][o + c];
+      A[i][j] -= acc;
+    }
+    __syncthreads();
+  }
+  // (d) off-diagonal blocks of X = L^-1, by block distance dd = ib - jb
+#pragma unroll 1
+  for (int dd = 1; dd < kT / kSub; ++dd) {
+    const int nblk = kT / kSub - dd;
+    // T_b = sum_{jb <= m < ib} L[ib][m] X[m][jb]  (16 x 16 each, blocks b = 0..nblk-1)
+    for (int e = tid; e < nblk * kSub * kSub; e += 256) {
+      const int b = e / (kSub * kSub), rr = (e / kSub) % kSub, cc = e % kSub;
+      const int ib = b + dd, jb = b;
+      float acc = 0.f;
+      for (int m = kSub * jb; m < kSub * ib; ++m) acc += A[kSub * ib + rr][m] * X[m][kSub * jb + cc];
+      T[b][rr][cc] = acc;
+    }
+    __syncthreads();
+    // X[ib][jb] = -X[ib][ib] T_b
+    for (int e = tid; e < nblk * kSub * kSub; e += 256) {
+      const int b = e / (kSub * kSub), rr = (e / kSub) % kSub, cc = e % kSub;
+      const int ib = b + dd, jb = b;
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < kSub; ++m)
+        if (m <= rr) acc += X[kSub * ib + rr][kSub * ib + m] * T[b][m][cc];
+      X[kSub * ib + rr][kSub * jb + cc] = -acc;
+    }
+    __syncthreads();
+  }
   if (tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = k * kT + bad;
   }
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    const int i = r0 + 4 * t;
-    if (c <= i) blk[(int64_t)i * D + c] = a[t];
-    Linv[i * kT + c] = x[t];
+  for (int e = tid; e < kT * kT; e += 256) {
+    const int i = e >> 6, j = e & 63;
+    if (j <= i) blk[(int64_t)i * D + j] = A[i][j];
+    Linv[i * kT + j] = X[i][j];
   }
 }
 
