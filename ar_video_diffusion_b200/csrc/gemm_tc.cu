@@ -34,6 +34,8 @@ enum Mode : int { kStoreBf16 = 0, kStoreF32 = 1, kReduceF32 = 2 };
 struct Params {
   CUtensorMap a_map;
   CUtensorMap b_map[2];
+  CUtensorMap c_map[2];  // output maps (32 x 32 boxes) for the TMA epilogue, when c_tma
+  int32_t c_tma;
   int32_t M, N, K;
   int32_t n_split;      // columns [0, n_split) come from b_map[0] / c[0], the rest from b_map[1] / c[1]
   int32_t lower_only0;  // skip tiles of the first column range that lie strictly above the diagonal
@@ -168,9 +170,66 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
     // ----------------------------------------------------------- epilogue
     const int h = (warp - 4) >> 2;
     const int wq = warp & 3;
-    const int gm = m0 + h * 128 + wq * 32 + lane;
+    const int row0 = m0 + h * 128 + wq * 32;
+    const int gm = row0 + lane;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag));
-    if (ok) {
+    if (ok && p.c_tma) {
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
+      const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
+      // The operand ring is idle once acc_full has fired (every MMA that read
+      // it has completed).  Each warp stages its 32 rows in 32 x 32 blocks
+      // there, double-buffered (2 x 4 KB per warp), in the swizzled layout of
+      // the output map, and one lane hands each block to a TMA store or
+      // reduction: whole 128-byte lines reach L2 instead of one 16-byte
+      // piece of 32 different rows per warp instruction.
+      uint8_t* stage_base = smem + (warp - 4) * 8192;
+      const CUtensorMap* cm = &p.c_map[half_n];
+      const bool rows_in = row0 < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + 32 * c, r);
+        tmem_wait_ld();
+        uint8_t* buf = stage_base + (c & 1) * 4096;
+        if (c >= 2) {
+          if (lane == 0) bulk_wait_read<1>();  // the block staged two steps ago has been read
+          __syncwarp();
+        }
+        if (p.mode == kStoreBf16) {
+          // 64-byte rows, 64-byte swizzle: 16-byte chunk j of row `lane` sits at j ^ ((lane >> 1) & 3)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+            u.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+            u.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+            u.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = u;
+          }
+        } else {
+          // 128-byte rows, 128-byte swizzle: chunk j of row `lane` sits at j ^ (lane & 7)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int gn = n0 + 32 * c;
+          if (rows_in && gn < n_cols) {  // boxes are clipped at the matrix edge; skip wholly outside ones
+            if (p.mode == kReduceF32)
+              tma_reduce_add_2d(cm, buf, gn, row0);
+            else
+              tma_store_2d(cm, buf, gn, row0);
+          }
+          bulk_commit();
+        }
+      }
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
+    } else if (ok) {
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
       const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
@@ -216,6 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
 }
 
+// Output maps for the TMA epilogue: c[0] has inner0 columns, c[1] inner1, both
+// `rows` rows `ld` elements apart.  Outputs whose base or row pitch is not
+// 16-byte aligned keep the per-thread epilogue (c_tma = 0).
+static bool set_out_maps(Params& p, bool f32, int64_t rows, int64_t ld, int64_t inner0, int64_t inner1) {
+  const int64_t eb = f32 ? 4 : 2;
+  p.c_tma = 0;
+  if (!aligned16(p.c[0]) || !aligned16(p.c[1]) || (ld * eb) % 16 != 0) return true;
+  if (!encode_map_out_2d(&p.c_map[0], p.c[0], f32, inner0, rows, ld * eb)) return false;
+  if (!encode_map_out_2d(&p.c_map[1], p.c[1], f32, inner1, rows, ld * eb)) return false;
+  p.c_tma = 1;
+  return true;
+}
+
 template <bool A_MN, bool B_MN, int BN, int NST>
 static ispa_status_t launch(const Params& p, int k_splits, cudaStream_t stream) {
   using L = Layout<BN, NST>;
@@ -255,6 +327,7 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   p.c[1] = R;
   p.ldc = D;
   p.mode = kReduceF32;
+  if (!set_out_maps(p, true, D, D, D, D)) return ISPA_ERR_CUDA;
   const int BN = D % 256 == 0 ? 256 : 128;
   const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
   int64_t tiles = m_tiles * n_tiles;  // R
@@ -294,6 +367,7 @@ ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t ro
   p.c[1] = E;
   p.ldc = D;
   p.mode = kReduceF32;
+  if (!set_out_maps(p, true, D, D, D, D)) return ISPA_ERR_CUDA;
   const int BN = D % 256 == 0 ? 256 : 128;
   const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
   int64_t tiles = 0;
@@ -328,6 +402,7 @@ ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_st
   p.c[1] = c;
   p.ldc = ldc;
   p.mode = accumulate ? kReduceF32 : kStoreF32;
+  if (!set_out_maps(p, true, M, ldc, N, N)) return ISPA_ERR_CUDA;
   if (N % 128) return unsupported("tensor-core GEMM needs N %% 128 == 0");
   return launch<false, true, 128, 4>(p, 1, stream);
 }
@@ -350,6 +425,7 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   p.c[1] = y;
   p.ldc = d_out;
   p.mode = kStoreBf16;
+  if (!set_out_maps(p, false, n_rows, d_out, d_out, d_out)) return ISPA_ERR_CUDA;
   if (d_out % 256 == 0) return launch<false, true, 256, 3>(p, 1, stream);
   if (d_out % 128 == 0) return launch<false, true, 128, 4>(p, 1, stream);
   return unsupported("bf16 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);

@@ -82,6 +82,29 @@ bool encode_map_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint
   return true;
 }
 
+bool encode_map_out_2d(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t rows,
+                       uint64_t row_bytes) {
+  auto fn = get_encode_fn();
+  if (!fn) {
+    set_last_error("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled (output) failed (%d): inner=%llu rows=%llu row_bytes=%llu", (int)r,
+                   (unsigned long long)inner, (unsigned long long)rows, (unsigned long long)row_bytes);
+    return false;
+  }
+  return true;
+}
+
 ispa_status_t set_smem(const void* kernel, int bytes) {
   // The attribute is per device; set it once per (kernel, device) so later
   // calls (including calls made while a stream is being captured) skip it.
