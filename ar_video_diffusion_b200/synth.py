@@ -93,6 +93,12 @@ WORKLOADS: Dict[str, Workload] = {
     "rollout": Workload("rollout", seed=4, n_heads=12, head_dim=128, frame_tokens=1560,
                         sink_frames=1, chunk_frames=3, hist_frames=0, dtype="bf16",
                         warm_chunks=4, n_layers=30, post_chunks=20),
+    # the rollout schedule at a size the CPU oracle follows end to end (every
+    # row of every chunk): 2 heads, 120 tokens per frame (360 chunk queries,
+    # a ragged third query tile), 4 layers
+    "rollout_small": Workload("rollout_small", seed=6, n_heads=2, head_dim=128, frame_tokens=120,
+                              sink_frames=1, chunk_frames=3, hist_frames=0, dtype="bf16",
+                              warm_chunks=4, n_layers=4, post_chunks=2),
 }
 
 

@@ -3,6 +3,8 @@ device and the error measures the tolerances are stated in."""
 import numpy as np
 import torch
 
+from oracle import ispa_oracle as orc
+
 # Tolerances (bf16 operands, fp32 accumulation):
 ATTN_MAX_REL = 2e-2      # attention outputs: max|x - ref| / max|ref| per tensor
 LSE_ABS = 1e-3           # log-sum-exp: absolute
@@ -37,3 +39,36 @@ def max_abs(x, ref) -> float:
 def fro_rel(x, ref) -> float:
     ref = np.asarray(ref, np.float64)
     return float(np.linalg.norm(np.asarray(x, np.float64) - ref) / np.linalg.norm(ref))
+
+
+# ------------------------------------------------ streaming rollout helpers
+def cat_segments(segs, i, D):
+    return np.concatenate([host(s[i]) for s in segs]) if segs else np.zeros((0, D))
+
+
+def oracle_rollout_statistics(w, inputs, layer):
+    """The oracle's A_loc and A_full over every warm-up row of one layer, from
+    the captured seeded inputs of that layer's warm-up chunks."""
+    a_loc, a_full = [], []
+    for c in range(w.warm_chunks):
+        x = inputs[(layer, c)]
+        ref = orc.dual_stream(x["q"], [(x["k_loc"], x["v_loc"])], [(x["k_hist"], x["v_hist"])], w.n_heads)
+        a_loc.append(ref["a_loc"])
+        a_full.append(ref["a_full"])
+    return np.concatenate(a_loc), np.concatenate(a_full)
+
+
+def capture_inputs(w, store, with_y=True):
+    """on_layer hook: host copies of each layer's seeded inputs (queries and
+    the K/V segments it attends to; one local segment list concatenated) and
+    of its output."""
+    def on_layer(l, c, info):
+        torch.cuda.synchronize()
+        D = w.d_model
+        rec = {"mode": info["mode"], "q": host(info["q"]),
+               "k_loc": cat_segments(info["local"], 0, D), "v_loc": cat_segments(info["local"], 1, D),
+               "k_hist": cat_segments(info["hist"], 0, D), "v_hist": cat_segments(info["hist"], 1, D)}
+        if with_y:
+            rec["y"] = host(info["y"])
+        store[(l, c)] = rec
+    return on_layer

@@ -95,8 +95,10 @@ def test_dual_attention_f32_matches_oracle(seed, n_q, H, d, loc, his):
 
 def test_tiny_f32_workload_end_to_end():
     """Tiny fp32 layer: 4 warm-up chunks of dual attention, statistics over
-    256 rows, absorb solve; dW checked against the oracle absorb fed the exact
-    A_loc and delta the GPU statistics consumed."""
+    256 rows, absorb solve.  dW is checked against the oracle chain: the
+    oracle's own dual stream, its G, R and its solve, from the same seeded
+    inputs.  The fp32 attention path is accurate to about 1e-6 relative, so
+    the chained dW stays within the fp32 bound."""
     w = synth.WORKLOADS["tiny_f32"]
     D = w.d_model
     G = torch.zeros(D, D, device="cuda")
@@ -114,8 +116,8 @@ def test_tiny_f32_workload_end_to_end():
         ref = orc.dual_stream(x["q"], [(x["k_sink"], x["v_sink"]), (x["k_cur"], x["v_cur"])],
                               [(x["k_hist"], x["v_hist"])], w.n_heads)
         _check_dual({k: host(v) for k, v in out.items()}, ref)
-        A_rows.append(host(out["a_loc"]))
-        D_rows.append(host(out["a_delta"]))
+        A_rows.append(ref["a_loc"])
+        D_rows.append(ref["a_full"] - ref["a_loc"])
     A, Dl = np.concatenate(A_rows), np.concatenate(D_rows)
     Gr, Rr = orc.gram(A, Dl)
     assert fro_rel(host(G), Gr) <= GRAM_REL and fro_rel(host(R), Rr) <= GRAM_REL
@@ -285,6 +287,28 @@ def test_local_attention_project_matches_oracle():
     assert max_rel(host(y), orc.project(a_ref, Wn)) <= ATTN_MAX_REL
 
 
+def test_local_attention_project_wan13b_sampled_rows():
+    """Post-transition L-layer at the Wan-1.3B shapes: 4680 chunk queries
+    over sink + current keys (6240), projected with a seeded weight standing
+    in for W_new; 48 sampled rows (the last included) against the oracle."""
+    w = synth.WORKLOADS["wan1.3b"]
+    x = synth.single_layer_inputs(w, 1)
+    W = synth.weight(w, 1)
+    status = ispa.new_status()
+    y, a_loc = ispa.local_attention_project(dev(x["q"], "bf16"),
+                                            [(dev(x["k_sink"], "bf16"), dev(x["v_sink"], "bf16")),
+                                             (dev(x["k_cur"], "bf16"), dev(x["v_cur"], "bf16"))],
+                                            dev(W, "bf16"), w.n_heads, status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "local_attention_project")
+    rows = np.sort(np.random.default_rng(6).choice(w.n_q, 48, replace=False))
+    rows[-1] = w.n_q - 1
+    a_ref, _ = orc.attention(x["q"][rows], np.concatenate([x["k_sink"], x["k_cur"]]),
+                             np.concatenate([x["v_sink"], x["v_cur"]]), w.n_heads)
+    assert max_rel(host(a_loc)[rows], a_ref) <= ATTN_MAX_REL
+    assert max_rel(host(y)[rows], orc.project(a_ref, W)) <= ATTN_MAX_REL
+
+
 def _layer_outputs(w, chunk=1):
     x = synth.single_layer_inputs(w, chunk)
     status = ispa.new_status()
@@ -364,30 +388,30 @@ def test_history_200k_dual_and_single_pass_sampled_rows():
 
 
 def test_wan14b_layer_sampled_rows_statistics_and_absorb():
-    """Wan-14B-shaped layer (40 heads, D = 5120): sampled attention rows, the
-    statistics of 4 warm-up chunks (18720 rows) entry by entry, and the
-    5120 x 5120 absorb solve against an fp64 solve of the same G, R."""
+    """Wan-14B-shaped layer (40 heads, D = 5120):
+    - sampled attention rows against the oracle;
+    - the statistics of 18720 seeded bf16 rows, entry by entry;
+    - the 5120 x 5120 absorb solve against the oracle's solve of the oracle's
+      G, R of the same rows."""
     w = synth.WORKLOADS["wan14b"]
     x, out = _layer_outputs(w)
     _check_sampled_rows(w, x, out, 48, 31)
+    del out
     D = w.d_model
+    n = w.warm_chunks * w.n_q  # 18720 warm-up rows
+    A, Dl, W = _absorb_case(31, n, D, "bf16")
     G = torch.empty(D, D, device="cuda")
     R = torch.empty(D, D, device="cuda")
-    As, Ds = [], []
-    for c in range(w.warm_chunks):
-        if c != 1:
-            _, out = _layer_outputs(w, c)
-        ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=(c == 0))
-        As.append(out["a_loc"])
-        Ds.append(out["a_delta"])
+    Ad, Dd = dev(A, "bf16"), dev(Dl, "bf16")
+    for c in range(w.warm_chunks):  # accumulated chunk by chunk, as in the warm-up
+        rows = slice(c * w.n_q, (c + 1) * w.n_q)
+        ispa.gram_accumulate(Ad[rows], Dd[rows], G, R, zero_first=(c == 0))
     torch.cuda.synchronize()
-    _check_gram_entries(torch.cat(As), torch.cat(Ds), G, R, 32, 32)
-    W = synth.weight(w, 0)
+    _check_gram_entries(Ad, Dd, G, R, 32, 32)
     status = ispa.new_status()
     dW, Wn = ispa.absorb_solve(G, R, dev(W, "bf16"), lambda_rel=orc.LAMBDA_REL, status=status)
     torch.cuda.synchronize()
     ispa.raise_on_status(status, "absorb_solve")
-    Gh, Rh = host(G), host(R)
-    Gh = np.tril(Gh) + np.tril(Gh, -1).T  # only the lower triangle of G is produced
-    dW_ref = orc.absorb(Gh, Rh, W, orc.ridge_lambda(Gh))
+    Gr, Rr = orc.gram(A, Dl)
+    dW_ref = orc.absorb(Gr, Rr, W, orc.ridge_lambda(Gr))
     assert fro_rel(host(dW), dW_ref) <= DW_REL_BF16

@@ -1,8 +1,23 @@
-"""GPU parity of the streaming rollout (1.3B shapes, 4 layers, layers 0 and 2
-absorbed, 4 warm-up chunks then 2 post-transition chunks): sampled rows of
-each checked layer output against the oracle, dW of both absorbed layers
-against the oracle absorb fed the exact A_loc / delta rows the GPU statistics
-consumed, and the KV bookkeeping bit for bit."""
+"""GPU parity of the streaming rollout ("Instance-Specific Parametric
+Absorption", gist.science technical summary, section 2, stages 1-3).
+
+* The small rollout (2 heads, 360 chunk queries, 4 layers, layers 0 and 2
+  absorbed, 4 warm-up chunks then 2 post-transition chunks) is followed end to
+  end by the CPU oracle from the same seeded inputs:
+  - the oracle's own dual stream over every warm-up row gives its G, R, dW and
+    W_new;
+  - every row of every layer output is compared with the oracle's attention
+    times the oracle's weight;
+  - nothing the GPU computed enters the oracle.
+* The 1.3B-shaped rollout (4 layers) is checked where the oracle can follow
+  it: the KV bookkeeping bit for bit, the eviction, and sampled rows of
+  F-layer outputs, whose weight is the seeded W.
+
+Chained tolerance of dW: the GPU statistics consume bf16 A_loc and delta, and
+the attention outputs differ from the oracle's at the 2^-9 level.  Simulated
+in the oracle (bf16 rounding plus 2^-9 relative noise on A_loc and A_full over
+the small rollout's 1440 warm-up rows), that moves dW by 4.5e-3 relative; the
+bound is 2e-2."""
 import dataclasses
 
 import numpy as np
@@ -13,41 +28,22 @@ from ar_video_diffusion_b200 import build as ispa_build
 from ar_video_diffusion_b200 import ispa, synth
 from ar_video_diffusion_b200.rollout import Rollout
 from oracle import ispa_oracle as orc
-from helpers import ATTN_MAX_REL, DW_REL_BF16, fro_rel, host, max_rel
+from helpers import (ATTN_MAX_REL, capture_inputs, cat_segments, fro_rel, host, max_rel,
+                     oracle_rollout_statistics)
 
 pytestmark = pytest.mark.gpu
 
-CHECK = {(0, 0), (1, 2), (2, 3), (0, 4), (1, 4), (2, 5), (3, 5)}
-N_ROWS = 32
+CHAIN_DW_REL = 2e-2
 
 
-def test_rollout_layers_absorb_and_kv_bookkeeping():
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
     ispa_build.build()
-    w = dataclasses.replace(synth.WORKLOADS["rollout"], n_layers=4, post_chunks=2)
-    absorbed = [0, 2]
-    rows = np.sort(np.random.default_rng(7).choice(w.n_q, N_ROWS, replace=False))
-    rows[-1] = w.n_q - 1
-    stats = {l: ([], []) for l in absorbed}
-    checks = []
 
-    def on_layer(l, c, info):
-        if c < w.warm_chunks and l in absorbed:
-            stats[l][0].append(host(info["out"]["a_loc"]))
-            stats[l][1].append(host(info["out"]["a_delta"]))
-        if (l, c) in CHECK:
-            torch.cuda.synchronize()
-            cat = lambda segs, i: np.concatenate([host(s[i]) for s in segs]) if segs else np.zeros((0, w.d_model))
-            checks.append({"l": l, "c": c, "mode": info["mode"], "q": host(info["q"])[rows],
-                           "k_loc": cat(info["local"], 0), "v_loc": cat(info["local"], 1),
-                           "k_hist": cat(info["hist"], 0), "v_hist": cat(info["hist"], 1),
-                           "W": host(info["W"]), "y": host(info["y"])[rows]})
 
-    ro = Rollout(w, absorbed=absorbed, on_layer=on_layer)
-    reports = ro.run()
-
-    # KV bookkeeping: bit-exact against the oracle's integer arithmetic
+def _check_bookkeeping(w, ro, reports, absorbed):
     mask = orc.layer_mask(w.n_layers, absorbed)
     for rep in reports:
         trans = rep.chunk >= w.warm_chunks
@@ -59,24 +55,66 @@ def test_rollout_layers_absorb_and_kv_bookkeeping():
     for l in absorbed:
         assert ro.k[l].shape[0] == w.frame_tokens + w.n_q
 
-    # absorb: dW against the oracle solve of the rows the statistics consumed
-    for l in absorbed:
-        A, Dl = np.concatenate(stats[l][0]), np.concatenate(stats[l][1])
-        G, R = orc.gram(A, Dl)
-        W = host(ro.W[l])
-        dW_ref = orc.absorb(G, R, W, orc.ridge_lambda(G))
-        assert fro_rel(host(ro.dW[l]), dW_ref) <= DW_REL_BF16
 
-    # sampled layer outputs
-    assert len(checks) == len(CHECK)
-    for ck in checks:
-        a_loc, _ = orc.attention(ck["q"], ck["k_loc"], ck["v_loc"], w.n_heads)
-        if ck["mode"] == "L":
-            a = a_loc
+def test_small_rollout_against_the_oracle_chain():
+    w = synth.WORKLOADS["rollout_small"]
+    absorbed = [0, 2]
+    inputs = {}
+    ro = Rollout(w, absorbed=absorbed, on_layer=capture_inputs(w, inputs))
+    reports = ro.run()
+    _check_bookkeeping(w, ro, reports, absorbed)
+
+    W = {l: host(ro.W[l]) for l in range(w.n_layers)}  # the seeded weights
+    W_new_ref = {}
+    for l in absorbed:
+        a_loc, a_full = oracle_rollout_statistics(w, inputs, l)
+        G, R = orc.gram(a_loc, a_full - a_loc)
+        dW_ref = orc.absorb(G, R, W[l], orc.ridge_lambda(G))
+        assert fro_rel(host(ro.dW[l]), dW_ref) <= CHAIN_DW_REL, l
+        W_new_ref[l] = synth.round_bf16(orc.modulated_weight(W[l], dW_ref).astype(np.float32))
+
+    n_chunks = w.warm_chunks + w.post_chunks
+    assert len(inputs) == w.n_layers * n_chunks
+    for (l, c), x in sorted(inputs.items()):
+        if x["mode"] == "L":
+            assert l in absorbed and c >= w.warm_chunks and x["k_hist"].shape[0] == 0
+            a, _ = orc.attention(x["q"], x["k_loc"], x["v_loc"], w.n_heads)
+            y_ref = orc.project(a, W_new_ref[l])
         else:
-            a, _ = orc.attention(ck["q"], np.concatenate([ck["k_loc"], ck["k_hist"]]),
-                                 np.concatenate([ck["v_loc"], ck["v_hist"]]), w.n_heads)
-        y_ref = orc.project(a, ck["W"])
-        assert max_rel(ck["y"], y_ref) <= ATTN_MAX_REL, (ck["l"], ck["c"], ck["mode"])
-    modes = {(ck["l"], ck["c"]): ck["mode"] for ck in checks}
-    assert modes[(0, 4)] == "L" and modes[(1, 4)] == "F" and modes[(0, 0)] == "F"
+            assert l not in absorbed or c < w.warm_chunks
+            a, _ = orc.attention(x["q"], np.concatenate([x["k_loc"], x["k_hist"]]),
+                                 np.concatenate([x["v_loc"], x["v_hist"]]), w.n_heads)
+            y_ref = orc.project(a, W[l])
+        assert max_rel(x["y"], y_ref) <= ATTN_MAX_REL, (l, c, x["mode"])
+
+
+CHECK_F = {(0, 0), (1, 2), (2, 3), (1, 4), (3, 5)}
+N_ROWS = 32
+
+
+def test_full_size_rollout_bookkeeping_and_f_layers():
+    w = dataclasses.replace(synth.WORKLOADS["rollout"], n_layers=4, post_chunks=2)
+    absorbed = [0, 2]
+    rows = np.sort(np.random.default_rng(7).choice(w.n_q, N_ROWS, replace=False))
+    rows[-1] = w.n_q - 1
+    checks = []
+
+    def on_layer(l, c, info):
+        if (l, c) in CHECK_F:
+            torch.cuda.synchronize()
+            D = w.d_model
+            checks.append({"l": l, "c": c, "mode": info["mode"], "q": host(info["q"])[rows],
+                           "k_loc": cat_segments(info["local"], 0, D), "v_loc": cat_segments(info["local"], 1, D),
+                           "k_hist": cat_segments(info["hist"], 0, D), "v_hist": cat_segments(info["hist"], 1, D),
+                           "W": host(info["W"]), "y": host(info["y"])[rows]})
+
+    ro = Rollout(w, absorbed=absorbed, on_layer=on_layer)
+    reports = ro.run()
+    _check_bookkeeping(w, ro, reports, absorbed)
+    assert len(checks) == len(CHECK_F)
+    for ck in checks:
+        assert ck["mode"] == "F"
+        assert np.array_equal(ck["W"], host(ro.W[ck["l"]]))  # F-layers project with the seeded W
+        a, _ = orc.attention(ck["q"], np.concatenate([ck["k_loc"], ck["k_hist"]]),
+                             np.concatenate([ck["v_loc"], ck["v_hist"]]), w.n_heads)
+        assert max_rel(ck["y"], orc.project(a, ck["W"])) <= ATTN_MAX_REL, (ck["l"], ck["c"])

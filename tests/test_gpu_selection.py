@@ -13,7 +13,7 @@ from ar_video_diffusion_b200 import build as ispa_build
 from ar_video_diffusion_b200 import ispa, synth
 from ar_video_diffusion_b200.rollout import Rollout
 from oracle import ispa_oracle as orc
-from helpers import GRAM_REL, dev, fro_rel, host
+from helpers import GRAM_REL, capture_inputs, dev, fro_rel, host, oracle_rollout_statistics
 
 pytestmark = pytest.mark.gpu
 
@@ -104,39 +104,43 @@ def test_layer_error_zero_when_streams_agree():
     assert num == 0.0 and den > 0.0
 
 
+# Chained tolerance of eps in the rollout: the GPU statistics consume bf16
+# A_loc and delta from its own attention.  The same oracle simulation as the
+# rollout test (bf16 rounding plus 2^-9 relative noise on the attention
+# outputs) moves eps by about 1e-4 relative; the bound is 1e-3.
+CHAIN_EPS_REL = 1e-3
+
+
 def test_rollout_instance_selection():
-    """4 layers of the 1.3B shapes, 2 warm-up chunks, K = 2 chosen by error."""
-    w = dataclasses.replace(synth.WORKLOADS["rollout"], n_layers=4, warm_chunks=2, post_chunks=1)
-    stats = {l: ([], []) for l in range(w.n_layers)}
-
-    def on_layer(l, c, info):
-        if c < w.warm_chunks:
-            stats[l][0].append(host(info["out"]["a_loc"]))
-            stats[l][1].append(host(info["out"]["a_delta"]))
-
-    ro = Rollout(w, absorbed=[0, 2], selection="instance", on_layer=on_layer)
+    """The small rollout (4 layers, 360 chunk queries, 4 warm-up chunks), with
+    K = 2 layers chosen by reconstruction error.  Each layer's eps is checked
+    against the oracle's eps of the oracle's own dual stream over the same
+    seeded inputs."""
+    w = dataclasses.replace(synth.WORKLOADS["rollout_small"], post_chunks=1)
+    inputs = {}
+    ro = Rollout(w, absorbed=[0, 2], selection="instance", on_layer=capture_inputs(w, inputs, with_y=False))
     reports = ro.run()
     eps_o = []
     for l in range(w.n_layers):
-        a_loc = np.concatenate(stats[l][0])
-        d = np.concatenate(stats[l][1])
+        a_loc, a_full = oracle_rollout_statistics(w, inputs, l)
         W = host(ro.W[l])
-        Go, Ro = orc.gram(a_loc, d)
+        Go, Ro = orc.gram(a_loc, a_full - a_loc)
         dWo = orc.absorb(Go, Ro, W, orc.ridge_lambda(Go))
-        eps_o.append(orc.reconstruction_error(a_loc, a_loc + d, W, dWo))
+        eps_o.append(orc.reconstruction_error(a_loc, a_full, W, dWo))
     for l in range(w.n_layers):
-        assert abs(ro.eps[l] - eps_o[l]) <= EPS_REL * eps_o[l], (l, ro.eps[l], eps_o[l])
-    # the chosen layers: unique unless two errors straddle the cut within the tolerance
+        assert abs(ro.eps[l] - eps_o[l]) <= CHAIN_EPS_REL * eps_o[l], (l, ro.eps[l], eps_o[l])
+    # the rollout took the K smallest of its own eps (ties to the lower index)
+    assert ro.absorbed == sorted(sorted(range(w.n_layers), key=lambda l: (ro.eps[l], l))[:2])
+    # and the oracle's choice, unless two errors straddle the cut within the tolerance
     ref = orc.select_layers(eps_o, 2)
     srt = sorted(eps_o)
-    if srt[2] - srt[1] > 2 * EPS_REL * srt[2]:
+    if srt[2] - srt[1] > 2 * CHAIN_EPS_REL * srt[2]:
         assert ro.absorbed == ref
-    assert ro.absorbed == orc.select_layers(ro.eps, 2)
-    # the selected layers became L-layers: history evicted, bookkeeping bit-exact
-    mask = orc.layer_mask(w.n_layers, ro.absorbed)
-    for l in ro.absorbed:
-        assert ro.k[l].shape[0] == w.frame_tokens + w.n_q
-    for rep in reports:
-        trans = rep.chunk >= w.warm_chunks
-        assert rep.kv_bytes == orc.kv_bytes(rep.chunk, w.n_layers, mask, trans, w.frame_tokens, w.chunk_frames,
-                                            w.d_model, 2)
+        # the selected layers became L-layers: history evicted, bookkeeping bit-exact
+        mask = orc.layer_mask(w.n_layers, ref)
+        for l in ref:
+            assert ro.k[l].shape[0] == w.frame_tokens + w.n_q
+        for rep in reports:
+            trans = rep.chunk >= w.warm_chunks
+            assert rep.kv_bytes == orc.kv_bytes(rep.chunk, w.n_layers, mask, trans, w.frame_tokens,
+                                                w.chunk_frames, w.d_model, 2)
