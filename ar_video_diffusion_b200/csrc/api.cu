@@ -40,6 +40,13 @@ ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W,
                                   double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
                                   int32_t* status, cudaStream_t st);
 
+ispa_status_t quantize_rows_e4m3(const void* x, int64_t n_rows, int64_t K, int64_t stride, uint8_t* q, float* scale,
+                                 cudaStream_t stream);
+ispa_status_t quantize_weight_e4m3(const void* w, int64_t K, int64_t N, uint8_t* qt, float* scale,
+                                   cudaStream_t stream);
+ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_rows, int64_t d_in,
+                           const uint8_t* qw_t, const float* w_scale, int64_t d_out, void* y, cudaStream_t stream);
+
 static bool valid_dtype(ispa_dtype_t dt) { return dt == ISPA_DT_BF16 || dt == ISPA_DT_F32; }
 static int64_t elem_bytes(ispa_dtype_t dt) { return dt == ISPA_DT_BF16 ? 2 : 4; }
 
@@ -288,6 +295,67 @@ extern "C" ispa_status_t ispa_local_attention_project(const void* q, int64_t n_q
                                          stream);
   if (st != ISPA_OK) return st;
   return ispa_project(a_loc_out, n_q, D, D, D, dt, w_new, y, stream);
+}
+
+// ------------------------------------------------------------------ W8A8
+static inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+extern "C" ispa_status_t ispa_quantize_e4m3_rows(const void* x, int64_t n_rows, int64_t k, int64_t row_stride,
+                                                 ispa_dtype_t dt, uint8_t* codes, float* scales, void* stream) {
+  if (dt != ISPA_DT_BF16) return unsupported("e4m3 quantisation takes bf16 activations");
+  if (!x || !codes || !scales) return invalid("required pointer is NULL");
+  if (n_rows <= 0 || k <= 0) return invalid("sizes must be positive");
+  if (k % 16) return unsupported("e4m3 quantisation needs k %% 16 == 0 (got %lld)", (long long)k);
+  if (row_stride < k) return invalid("row_stride < k");
+  if (!aligned16(x) || !aligned16(codes) || !aligned4(scales) || (row_stride * 2) % 16)
+    return invalid("x and codes must be 16-byte aligned (rows too), scales 4-byte aligned");
+  if (n_rows > INT32_MAX / 2 || k > 65536) return unsupported("problem too large");
+  return quantize_rows_e4m3(x, n_rows, k, row_stride, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_quantize_e4m3_weight(const void* w, int64_t d_in, int64_t d_out, ispa_dtype_t dt,
+                                                   uint8_t* codes_t, float* scales, void* stream) {
+  if (dt != ISPA_DT_BF16) return unsupported("e4m3 quantisation takes a bf16 weight");
+  if (!w || !codes_t || !scales) return invalid("required pointer is NULL");
+  if (d_in <= 0 || d_out <= 0) return invalid("sizes must be positive");
+  if (d_in % 16 || d_out % 16) return unsupported("e4m3 weight quantisation needs d_in, d_out multiples of 16");
+  if (!aligned16(w) || !aligned16(codes_t) || !aligned4(scales)) return invalid("pointers are misaligned");
+  if (d_in > 65536 || d_out > 65536) return unsupported("problem too large");
+  return quantize_weight_e4m3(w, d_in, d_out, codes_t, scales, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_project_w8a8(const uint8_t* a_codes, const float* a_scales, int64_t n_rows,
+                                           int64_t d_in, const uint8_t* w_codes_t, const float* w_scales,
+                                           int64_t d_out, void* y, void* stream) {
+  if (!a_codes || !a_scales || !w_codes_t || !w_scales || !y) return invalid("required pointer is NULL");
+  if (n_rows <= 0 || d_in <= 0 || d_out <= 0) return invalid("sizes must be positive");
+  if (d_in % 16 || d_out % 128)
+    return unsupported("W8A8 projection needs d_in %% 16 == 0 and d_out %% 128 == 0 (got %lld, %lld)",
+                       (long long)d_in, (long long)d_out);
+  if (!aligned16(a_codes) || !aligned16(w_codes_t) || !aligned16(w_scales) || !aligned4(a_scales) || !aligned16(y))
+    return invalid("codes, w_scales and y must be 16-byte aligned, a_scales 4-byte aligned");
+  if (n_rows > INT32_MAX / 2 || d_in > 65536 || d_out > 65536) return unsupported("problem too large");
+  return project_e4m3(a_codes, a_scales, n_rows, d_in, w_codes_t, w_scales, d_out, y,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_local_attention_project_w8a8(
+    const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim, ispa_dtype_t dt,
+    float softmax_scale, const ispa_kv_segment_t* local, int32_t n_local, const uint8_t* w_codes_t,
+    const float* w_scales, void* y, void* a_loc_out, uint8_t* a_codes, float* a_scales, int32_t* dev_status,
+    void* stream) {
+  if (dt != ISPA_DT_BF16) return unsupported("the W8A8 L-layer path takes bf16 activations");
+  if (!w_codes_t || !w_scales || !y || !a_loc_out || !a_codes || !a_scales)
+    return invalid("w_codes_t, w_scales, y, a_loc_out, a_codes and a_scales are required");
+  const int64_t D = (int64_t)n_heads * head_dim;
+  if (D % 128) return unsupported("W8A8 L-layer projection needs D %% 128 == 0");
+  ispa_status_t st = ispa_dual_attention(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local,
+                                         nullptr, 0, nullptr, a_loc_out, nullptr, nullptr, nullptr, dev_status,
+                                         stream);
+  if (st != ISPA_OK) return st;
+  st = ispa_quantize_e4m3_rows(a_loc_out, n_q, D, D, dt, a_codes, a_scales, stream);
+  if (st != ISPA_OK) return st;
+  return ispa_project_w8a8(a_codes, a_scales, n_q, D, w_codes_t, w_scales, D, y, stream);
 }
 
 // ------------------------------------------------------------ bookkeeping

@@ -26,7 +26,8 @@ namespace ispa {
 namespace gemm {
 
 constexpr int kBM = 256;  // two tensor-core M=128 halves
-constexpr int kBK = 64;
+constexpr int kBK = 64;    // K elements per stage for bf16 (128 bytes of a row)
+constexpr int kBK8 = 128;  // K elements per stage for e4m3 (the same 128 bytes)
 constexpr int kThreads = 384;
 
 enum Mode : int { kStoreBf16 = 0, kStoreF32 = 1, kReduceF32 = 2 };
@@ -44,6 +45,8 @@ struct Params {
   int64_t ldc;
   int32_t mode;
   int32_t* status;
+  const float* row_scale;  // e4m3 inputs: y[i, j] = acc[i, j] * row_scale[i] * col_scale[j]
+  const float* col_scale;
 };
 
 template <int BN, int NST>
@@ -63,9 +66,14 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-template <bool A_MN, bool B_MN, int BN, int NST>
-__global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_constant__ Params p) {
+// The body shared by the bf16 kernels and the e4m3 kernel (F8: both operands
+// K-major e4m3, kind::f8f6f4 MMAs with K = 32, the same 128-byte rows and
+// swizzle per stage as bf16, and a scaled bf16 epilogue through TMA).
+template <bool A_MN, bool B_MN, int BN, int NST, bool F8>
+__device__ __forceinline__ void gemm_body(const Params& p) {
   using L = Layout<BN, NST>;
+  static_assert(!F8 || (!A_MN && !B_MN), "e4m3 operands are K-major");
+  constexpr int BK = F8 ? kBK8 : kBK;
   const int n0g = blockIdx.x * BN, m0 = blockIdx.y * kBM;
   const int half_n = n0g >= p.n_split ? 1 : 0;
   const int n0 = n0g - half_n * p.n_split;
@@ -75,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   const int k_begin = blockIdx.z * p.k_per_split;
   const int k_end = min(p.K, k_begin + p.k_per_split);
   if (k_begin >= k_end) return;
-  const int nk = (k_end - k_begin + kBK - 1) / kBK;
+  const int nk = (k_end - k_begin + BK - 1) / BK;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -117,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
       if (kb >= NST && !mbar_wait(&empty[stage], ((kb / NST) - 1) & 1, abort_flag)) break;
       uint8_t* sa = smem + stage * L::kStage;
       uint8_t* sb = sa + L::kABytes;
-      const int k0 = k_begin + kb * kBK;
+      const int k0 = k_begin + kb * BK;
       mbar_arrive_expect_tx(&full[stage], L::kStage);
       if (A_MN) {
 #pragma unroll
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
-    constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN, A_MN, B_MN);
+    constexpr uint32_t kIdesc = F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, A_MN, B_MN);
     const uint32_t base = smem_u32(smem);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -151,14 +159,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
       const uint32_t sa = base + stage * L::kStage;
       const uint32_t sb = sa + L::kABytes;
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk) {
+      for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes of K (16 bf16 or 32 e4m3)
         const uint64_t db = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // rows 128h..128h+127 of the A tile: MN-major blocks 2h, 2h+1 / K-major rows
           const uint64_t da = A_MN ? sdesc_sw128(sa + h * 16384 + kk * 2048, 8192, 1024)
                                    : sdesc_sw128(sa + h * 16384 + kk * 32, 16, 1024);
-          umma_ss(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          if (F8)
+            umma_ss_f8(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          else
+            umma_ss(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
         }
       }
       umma_commit(&empty[stage]);
@@ -191,6 +202,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
         uint32_t r[32];
         tmem_ld32(taddr + 32 * c, r);
         tmem_wait_ld();
+        if (F8) {
+          // per-row and per-column dequantisation scales
+          const float sa = gm < p.M ? __ldg(p.row_scale + gm) : 0.f;
+          const float4* sw4 = reinterpret_cast<const float4*>(p.col_scale + n0 + 32 * c);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 w4 = __ldg(sw4 + j);
+            r[4 * j + 0] = __float_as_uint(__uint_as_float(r[4 * j + 0]) * (sa * w4.x));
+            r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * (sa * w4.y));
+            r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * (sa * w4.z));
+            r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) * (sa * w4.w));
+          }
+        }
         uint8_t* buf = stage_base + (c & 1) * 4096;
         if (c >= 2) {
           if (lane == 0) bulk_wait_read<1>();  // the block staged two steps ago has been read
@@ -229,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
       }
       if (lane == 0) bulk_wait<0>();
       __syncwarp();
-    } else if (ok) {
+    } else if (ok && !F8) {  // outputs the TMA epilogue cannot address (e4m3 callers always use TMA)
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
       const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
@@ -275,6 +299,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
 }
 
+template <bool A_MN, bool B_MN, int BN, int NST>
+__global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_constant__ Params p) {
+  gemm_body<A_MN, B_MN, BN, NST, false>(p);
+}
+
+template <int BN, int NST>
+__global__ void __launch_bounds__(kThreads, 1) gemm_e4m3_kernel(const __grid_constant__ Params p) {
+  gemm_body<false, false, BN, NST, true>(p);
+}
+
 // Output maps for the TMA epilogue: c[0] has inner0 columns, c[1] inner1, both
 // `rows` rows `ld` elements apart.  Outputs whose base or row pitch is not
 // 16-byte aligned keep the per-thread epilogue (c_tma = 0).
@@ -286,6 +320,17 @@ static bool set_out_maps(Params& p, bool f32, int64_t rows, int64_t ld, int64_t 
   if (!encode_map_out_2d(&p.c_map[1], p.c[1], f32, inner1, rows, ld * eb)) return false;
   p.c_tma = 1;
   return true;
+}
+
+template <int BN, int NST>
+static ispa_status_t launch_e4m3(const Params& p, cudaStream_t stream) {
+  using L = Layout<BN, NST>;
+  auto kern = gemm_e4m3_kernel<BN, NST>;
+  ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
+  if (st != ISPA_OK) return st;
+  dim3 grid(p.N / BN, (p.M + kBM - 1) / kBM, 1);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
+  return check_launch("gemm_e4m3_kernel");
 }
 
 template <bool A_MN, bool B_MN, int BN, int NST>
@@ -429,6 +474,35 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   if (d_out % 256 == 0) return launch<false, true, 256, 3>(p, 1, stream);
   if (d_out % 128 == 0) return launch<false, true, 128, 4>(p, 1, stream);
   return unsupported("bf16 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);
+}
+
+// y[n_rows, d_out] (bf16) = diag(a_scale) qa[n_rows, d_in] qw_t[d_out, d_in]^T diag(w_scale):
+// e4m3 codes of the activations (row-major, token rows) and of the weight
+// stored transposed (one row per output channel), fp32 accumulation.
+ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_rows, int64_t d_in,
+                           const uint8_t* qw_t, const float* w_scale, int64_t d_out, void* y, cudaStream_t stream) {
+  using namespace gemm;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  if (!encode_map_u8_2d(&p.a_map, qa, d_in, n_rows, d_in, kBK8, kBM)) return ISPA_ERR_CUDA;
+  const int BN = d_out % 256 == 0 ? 256 : 128;
+  if (!encode_map_u8_2d(&p.b_map[0], qw_t, d_in, d_out, d_in, kBK8, BN)) return ISPA_ERR_CUDA;
+  p.b_map[1] = p.b_map[0];
+  p.M = (int32_t)n_rows;
+  p.N = (int32_t)d_out;
+  p.K = (int32_t)d_in;
+  p.n_split = (int32_t)d_out;
+  p.k_per_split = (int32_t)(((d_in + kBK8 - 1) / kBK8) * kBK8);
+  p.c[0] = y;
+  p.c[1] = y;
+  p.ldc = d_out;
+  p.mode = kStoreBf16;
+  p.row_scale = a_scale;
+  p.col_scale = w_scale;
+  if (!set_out_maps(p, false, n_rows, d_out, d_out, d_out)) return ISPA_ERR_CUDA;
+  if (!p.c_tma) return unsupported("e4m3 projection needs a 16-byte aligned output");
+  if (BN == 256) return launch_e4m3<256, 3>(p, stream);
+  return launch_e4m3<128, 4>(p, stream);
 }
 
 }  // namespace ispa

@@ -82,6 +82,29 @@ bool encode_map_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint
   return true;
 }
 
+bool encode_map_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                      uint32_t box_inner, uint32_t box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn) {
+    set_last_error("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled (8-bit) failed (%d): inner=%llu rows=%llu row_bytes=%llu box=%ux%u",
+                   (int)r, (unsigned long long)inner, (unsigned long long)rows, (unsigned long long)row_bytes,
+                   box_inner, box_rows);
+    return false;
+  }
+  return true;
+}
+
 bool encode_map_out_2d(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t rows,
                        uint64_t row_bytes) {
   auto fn = get_encode_fn();

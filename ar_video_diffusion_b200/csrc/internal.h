@@ -29,6 +29,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 bool encode_map_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
                         uint32_t box_inner, uint32_t box_rows);
 
+// The same for a row-major [rows, inner] matrix of bytes (e4m3 codes).
+bool encode_map_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                      uint32_t box_inner, uint32_t box_rows);
+
 // 2-D TMA map for output tiles of a row-major [rows, inner] matrix (fp32 or
 // bf16): boxes of 32 x 32 elements, 128-byte swizzle for fp32 (one box row is
 // 128 bytes), 64-byte swizzle for bf16.  Used by TMA stores and reductions.

@@ -32,6 +32,8 @@ MAX_SEGMENTS = 8
 EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "ispa_sym_gram_accumulate",
             "ispa_layer_error_workspace_bytes", "ispa_layer_error", "ispa_select_layers", "ispa_absorb_workspace_bytes",
             "ispa_absorb_solve", "ispa_absorb_solve_noalloc", "ispa_project", "ispa_local_attention_project",
+            "ispa_quantize_e4m3_rows", "ispa_quantize_e4m3_weight", "ispa_project_w8a8",
+            "ispa_local_attention_project_w8a8",
             "ispa_chunk_token_ranges", "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
             "ispa_version")
 
@@ -75,6 +77,11 @@ def lib() -> ctypes.CDLL:
             "ispa_project": (i32, [vp, i64, i64, i64, i64, i32, vp, vp, vp]),
             "ispa_local_attention_project": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp, vp,
                                                    vp]),
+            "ispa_quantize_e4m3_rows": (i32, [vp, i64, i64, i64, i32, vp, vp, vp]),
+            "ispa_quantize_e4m3_weight": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+            "ispa_project_w8a8": (i32, [vp, vp, i64, i64, vp, vp, i64, vp, vp]),
+            "ispa_local_attention_project_w8a8": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp,
+                                                        vp, vp, vp, vp, vp]),
             "ispa_chunk_token_ranges": (i32, [i64, i64, i64, i64, c.POINTER(i64)]),
             "ispa_kv_bytes": (i64, [i64, i32, c.c_uint64, i32, i64, i64, i64, i32, i64]),
             "ispa_selftest_wait_timeout": (i32, [c.c_uint32, vp, vp]),
@@ -192,6 +199,27 @@ def ispa_local_attention_project(q, n_q, q_stride, n_heads, head_dim, dt, softma
     _check(lib().ispa_local_attention_project(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local,
                                               n_local, w_new, y, a_loc_out, dev_status, stream),
            "ispa_local_attention_project")
+
+
+def ispa_quantize_e4m3_rows(x, n_rows, k, row_stride, dt, codes, scales, stream):
+    _check(lib().ispa_quantize_e4m3_rows(x, n_rows, k, row_stride, dt, codes, scales, stream),
+           "ispa_quantize_e4m3_rows")
+
+
+def ispa_quantize_e4m3_weight(w, d_in, d_out, dt, codes_t, scales, stream):
+    _check(lib().ispa_quantize_e4m3_weight(w, d_in, d_out, dt, codes_t, scales, stream), "ispa_quantize_e4m3_weight")
+
+
+def ispa_project_w8a8(a_codes, a_scales, n_rows, d_in, w_codes_t, w_scales, d_out, y, stream):
+    _check(lib().ispa_project_w8a8(a_codes, a_scales, n_rows, d_in, w_codes_t, w_scales, d_out, y, stream),
+           "ispa_project_w8a8")
+
+
+def ispa_local_attention_project_w8a8(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local,
+                                      w_codes_t, w_scales, y, a_loc_out, a_codes, a_scales, dev_status, stream):
+    _check(lib().ispa_local_attention_project_w8a8(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local,
+                                                   n_local, w_codes_t, w_scales, y, a_loc_out, a_codes, a_scales,
+                                                   dev_status, stream), "ispa_local_attention_project_w8a8")
 
 
 def ispa_chunk_token_ranges(chunk: int, frame_tokens: int, chunk_frames: int, sink_frames: int = 1):
@@ -356,3 +384,64 @@ def local_attention_project(q: torch.Tensor, local: Sequence[Tuple[torch.Tensor,
                                  softmax_scale, ls, nl, _dev(w_new, "w_new"), _dev(y, "y"), _dev(a_loc, "a_loc"),
                                  _dev(status, "status"), _stream(stream))
     return y, a_loc
+
+
+def quantize_e4m3_rows(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                       scales: Optional[torch.Tensor] = None, stream=None):
+    """Per-row e4m3 codes (uint8 [n, k]) and fp32 scales [n] of bf16 x [n, k]."""
+    n, k = x.shape
+    if codes is None:
+        codes = torch.empty(n, k, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(n, dtype=torch.float32, device=x.device)
+    ispa_quantize_e4m3_rows(_dev(x, "x"), n, k, _row_stride(x, "x"), _dtype_code(x), _dev(codes, "codes"),
+                            _dev(scales, "scales"), _stream(stream))
+    return codes, scales
+
+
+def quantize_e4m3_weight(w: torch.Tensor, codes_t: Optional[torch.Tensor] = None,
+                         scales: Optional[torch.Tensor] = None, stream=None):
+    """Per-output-channel e4m3 codes of bf16 w [d_in, d_out], returned
+    TRANSPOSED (uint8 [d_out, d_in]), and fp32 scales [d_out]."""
+    d_in, d_out = w.shape
+    if codes_t is None:
+        codes_t = torch.empty(d_out, d_in, dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(d_out, dtype=torch.float32, device=w.device)
+    ispa_quantize_e4m3_weight(_dev(w, "w"), d_in, d_out, _dtype_code(w), _dev(codes_t, "codes_t"),
+                              _dev(scales, "scales"), _stream(stream))
+    return codes_t, scales
+
+
+def project_w8a8(a_codes: torch.Tensor, a_scales: torch.Tensor, w_codes_t: torch.Tensor, w_scales: torch.Tensor,
+                 y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 y [n, d_out] of the W8A8 projection from the two sets of codes."""
+    n, d_in = a_codes.shape
+    d_out = w_codes_t.shape[0]
+    if y is None:
+        y = torch.empty(n, d_out, dtype=torch.bfloat16, device=a_codes.device)
+    ispa_project_w8a8(_dev(a_codes, "a_codes"), _dev(a_scales, "a_scales"), n, d_in, _dev(w_codes_t, "w_codes_t"),
+                      _dev(w_scales, "w_scales"), d_out, _dev(y, "y"), _stream(stream))
+    return y
+
+
+def local_attention_project_w8a8(q: torch.Tensor, local: Sequence[Tuple[torch.Tensor, torch.Tensor]],
+                                 w_codes_t: torch.Tensor, w_scales: torch.Tensor, n_heads: int,
+                                 softmax_scale: float = 0.0, out: Optional[dict] = None,
+                                 status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """L-layer with the W8A8 projection: local attention (bf16) -> A_loc ->
+    e4m3 codes -> y.  Returns {"y", "a_loc", "a_codes", "a_scales"}."""
+    n_q, D = q.shape
+    if out is None:
+        dev = q.device
+        out = {"y": torch.empty(n_q, D, dtype=torch.bfloat16, device=dev),
+               "a_loc": torch.empty(n_q, D, dtype=torch.bfloat16, device=dev),
+               "a_codes": torch.empty(n_q, D, dtype=torch.uint8, device=dev),
+               "a_scales": torch.empty(n_q, dtype=torch.float32, device=dev)}
+    ls, nl = _segments(local)
+    ispa_local_attention_project_w8a8(_dev(q, "q"), n_q, _row_stride(q, "q"), n_heads, D // n_heads,
+                                      _dtype_code(q), softmax_scale, ls, nl, _dev(w_codes_t, "w_codes_t"),
+                                      _dev(w_scales, "w_scales"), _dev(out["y"], "y"), _dev(out["a_loc"], "a_loc"),
+                                      _dev(out["a_codes"], "a_codes"), _dev(out["a_scales"], "a_scales"),
+                                      _dev(status, "status"), _stream(stream))
+    return out

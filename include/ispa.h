@@ -249,6 +249,65 @@ ISPA_API ispa_status_t ispa_local_attention_project(const void* q, int64_t n_q, 
                                            const ispa_kv_segment_t* local, int32_t n_local, const void* w_new,
                                            void* y, void* a_loc_out, int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------- W8A8 --
+ * Source: post-training W8A8 quantisation of the projection, which ISPA is
+ * run with in "Instance-Specific Parametric Absorption" (gist.science
+ * technical summary, section 4 "Experimental Results", item "Speedup").  The
+ * page fixes no scheme.  This library's reading:
+ *   - the 8-bit format is e4m3 (bias 7, 3 mantissa bits, largest finite 448,
+ *     no infinity);
+ *   - activations get one fp32 scale per token row, and the weight W
+ *     [d_in, d_out] one per output channel (column): s = amax / 448, or 1 for
+ *     an all-zero row or column;
+ *   - code = e4m3(x / s), round to nearest even, saturating at +-448, with
+ *     amax / 448 and x / s computed as IEEE fp32 divisions;
+ *   - y[i, j] = s_a[i] * s_w[j] * sum_k dec(qa[i, k]) * dec(qw[k, j]), fp32
+ *     accumulation on the tensor cores, bf16 output;
+ *   - the weight is quantised after the absorb, that is W_new = W + dW.
+ * All pointers are device pointers owned by the caller.  Nothing allocates;
+ * everything runs asynchronously on `stream`.
+ *
+ * ispa_quantize_e4m3_rows:
+ *   - x [n_rows, k] bf16, row_stride elements apart;
+ *   - codes [n_rows, k] bytes, dense;
+ *   - scales [n_rows] fp32;
+ *   - k must be a multiple of 16; x, its rows and codes 16-byte aligned.
+ * ispa_quantize_e4m3_weight:
+ *   - w [d_in, d_out] bf16, row-major;
+ *   - codes_t [d_out, d_in] bytes: the codes TRANSPOSED, one row per output
+ *     channel;
+ *   - scales [d_out] fp32;
+ *   - d_in and d_out must be multiples of 16.
+ * ispa_project_w8a8:
+ *   - y [n_rows, d_out] bf16 from a_codes [n_rows, d_in], a_scales [n_rows],
+ *     w_codes_t [d_out, d_in] and w_scales [d_out];
+ *   - d_in % 16 == 0 and d_out % 128 == 0;
+ *   - codes, w_scales and y must be 16-byte aligned.
+ * ispa_local_attention_project_w8a8: the L-layer of ispa_local_attention_project
+ * with the W8A8 projection.  It runs the bf16 local attention into a_loc_out,
+ * quantises A_loc into a_codes [n_q, D] / a_scales [n_q], then projects with the
+ * quantised W_new.
+ * Errors:
+ *   - ISPA_ERR_INVALID_ARG for a NULL or misaligned pointer or a non-positive
+ *     size;
+ *   - ISPA_ERR_UNSUPPORTED for another dtype or sizes off the multiples above;
+ *   - nothing is launched in either case.
+ */
+ISPA_API ispa_status_t ispa_quantize_e4m3_rows(const void* x, int64_t n_rows, int64_t k, int64_t row_stride,
+                                               ispa_dtype_t dt, uint8_t* codes, float* scales, void* stream);
+ISPA_API ispa_status_t ispa_quantize_e4m3_weight(const void* w, int64_t d_in, int64_t d_out, ispa_dtype_t dt,
+                                                 uint8_t* codes_t, float* scales, void* stream);
+ISPA_API ispa_status_t ispa_project_w8a8(const uint8_t* a_codes, const float* a_scales, int64_t n_rows, int64_t d_in,
+                                         const uint8_t* w_codes_t, const float* w_scales, int64_t d_out, void* y,
+                                         void* stream);
+ISPA_API ispa_status_t ispa_local_attention_project_w8a8(const void* q, int64_t n_q, int64_t q_stride,
+                                                         int32_t n_heads, int32_t head_dim, ispa_dtype_t dt,
+                                                         float softmax_scale, const ispa_kv_segment_t* local,
+                                                         int32_t n_local, const uint8_t* w_codes_t,
+                                                         const float* w_scales, void* y, void* a_loc_out,
+                                                         uint8_t* a_codes, float* a_scales, int32_t* dev_status,
+                                                         void* stream);
+
 /* ------------------------------------------------------ host bookkeeping --
  * Streaming bookkeeping of [gist §2.1, §2.3], host-only and exact (integers).
  *

@@ -146,3 +146,23 @@ def test_segment_limit_and_empty_queries_rejected_before_launch(L):
     r = L.ispa_dual_attention(q, 10, 128, 1, 128, 0, 0.0, segs(1, 0), 1, segs(1), 1, out, out, None, None, None, None,
                               None)
     assert r == 1 and "local" in L.ispa_last_error().decode()
+
+
+def test_w8a8_entry_points_reject_before_launch(L):
+    p, odd = ctypes.c_void_p(256), ctypes.c_void_p(264)
+    # activations: fp32 is unsupported, k must be a multiple of 16, NULL codes, misaligned rows
+    assert L.ispa_quantize_e4m3_rows(p, 4, 128, 128, 1, p, p, None) == 2
+    assert L.ispa_quantize_e4m3_rows(p, 4, 120, 120, 0, p, p, None) == 2
+    assert L.ispa_quantize_e4m3_rows(p, 4, 128, 128, 0, None, p, None) == 1
+    assert L.ispa_quantize_e4m3_rows(p, 4, 128, 132, 0, p, p, None) == 1
+    assert L.ispa_quantize_e4m3_rows(odd, 4, 128, 128, 0, p, p, None) == 1
+    # weight: sizes off the multiples, NULL scales
+    assert L.ispa_quantize_e4m3_weight(p, 100, 128, 0, p, p, None) == 2
+    assert L.ispa_quantize_e4m3_weight(p, 128, 128, 0, p, None, None) == 1
+    # projection: d_out % 128, misaligned codes, non-positive rows
+    assert L.ispa_project_w8a8(p, p, 4, 128, p, p, 192, p, None) == 2
+    assert L.ispa_project_w8a8(odd, p, 4, 128, p, p, 128, p, None) == 1
+    assert L.ispa_project_w8a8(p, p, 0, 128, p, p, 128, p, None) == 1
+    # L-layer W8A8: missing code buffers
+    assert L.ispa_local_attention_project_w8a8(p, 4, 128, 1, 128, 0, 0.0, None, 0, p, p, p, p, None, p, None,
+                                               None) == 1
