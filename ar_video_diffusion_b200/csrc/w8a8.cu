@@ -38,8 +38,12 @@ __device__ __forceinline__ uint2 codes8(const float (&x)[8], float s) {
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// One warp per row: the row is read twice (amax, then codes; the second read
-// hits L1/L2), codes go out as 8-byte pieces, consecutive lanes contiguous.
+// One warp per row.  Rows of up to 2048 elements stay in registers (8
+// 16-byte vectors per lane) between the amax and the codes, so each byte of x
+// is read once; longer rows are read twice (the second read hits L1/L2).
+// Codes go out as 8-byte pieces, consecutive lanes contiguous.
+constexpr int kRegVecs = 8;
+
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t n_rows,
                                                             int K, int64_t stride, uint8_t* __restrict__ q,
                                                             float* __restrict__ scale) {
@@ -47,22 +51,48 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16*
   const int nv = K / 8;
   for (int64_t row = (int64_t)blockIdx.x * 8 + warp; row < n_rows; row += (int64_t)gridDim.x * 8) {
     const uint4* src = reinterpret_cast<const uint4*>(x + row * stride);
-    float amax = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-      float f[8];
-      bf16x8(__ldg(src + v), f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = scale_of(amax);
-    if (lane == 0) scale[row] = s;
     uint2* dst = reinterpret_cast<uint2*>(q + row * K);
-    for (int v = lane; v < nv; v += 32) {
-      float f[8];
-      bf16x8(__ldg(src + v), f);
-      dst[v] = codes8(f, s);
+    float amax = 0.f;
+    if (nv <= 32 * kRegVecs) {
+      uint4 buf[kRegVecs];
+#pragma unroll
+      for (int i = 0; i < kRegVecs; ++i) {
+        const int v = lane + 32 * i;
+        buf[i] = v < nv ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+        float f[8];
+        bf16x8(buf[i], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = scale_of(amax);
+      if (lane == 0) scale[row] = s;
+#pragma unroll
+      for (int i = 0; i < kRegVecs; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nv) {
+          float f[8];
+          bf16x8(buf[i], f);
+          dst[v] = codes8(f, s);
+        }
+      }
+    } else {
+      for (int v = lane; v < nv; v += 32) {
+        float f[8];
+        bf16x8(__ldg(src + v), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = scale_of(amax);
+      if (lane == 0) scale[row] = s;
+      for (int v = lane; v < nv; v += 32) {
+        float f[8];
+        bf16x8(__ldg(src + v), f);
+        dst[v] = codes8(f, s);
+      }
     }
   }
 }

@@ -334,6 +334,8 @@ def run_ours(args, rank, world, device):
     # standalone LSE merge over rotating buffer sets larger than L2
     merge_gbs = merge_bench(ispa, w, device)
     long_hist = long_history_bench(ispa, device)
+    pk0, _ = peaks()
+    w8a8 = w8a8_bench(ispa, w, device, pk0["bf16_tflops"], pk0["hbm_gbs"])
 
     rollout = None if args.no_rollout else run_rollout(device)
 
@@ -387,6 +389,7 @@ def run_ours(args, rank, world, device):
         "clocks": clk,
         "gpu_launches": args.steps * (7 + absorb_launches(D)),
         "long_history": long_hist,
+        "w8a8": w8a8,
         "rollout": rollout,
     }
     return res
@@ -416,6 +419,10 @@ def run_profile_case(op: str, reps: int, device):
         ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=True)
     if op == "merge":
         o_hist = ispa.dual_attention(q, [], hist, H, dual=False, status=status)
+    if op in ("project_w8a8", "quantize_rows"):
+        a16 = ispa.dual_attention(q, local, hist, H, status=status)["a_loc"]
+        qwt, sw = ispa.quantize_e4m3_weight(W)
+        qa, sa = ispa.quantize_e4m3_rows(a16)
     if op == "dual":
         out = {"a_loc": torch.empty(n, D, dtype=torch.bfloat16, device=device),
                "a_full": torch.empty(n, D, dtype=torch.bfloat16, device=device),
@@ -437,6 +444,10 @@ def run_profile_case(op: str, reps: int, device):
             ispa.lse_merge(out["a_loc"], out["lse_loc"], o_hist["a_full"], o_hist["lse_full"], H)
         elif op == "absorb":
             ispa.absorb_solve(G, R, W, status=status)
+        elif op == "project_w8a8":
+            ispa.project_w8a8(qa, sa, qwt, sw)
+        elif op == "quantize_rows":
+            ispa.quantize_e4m3_rows(a16, qa, sa)
     torch.cuda.synchronize(device)
     if int(status[0].item()) != 0:
         raise RuntimeError(f"device status {int(status[0].item())}")
@@ -562,6 +573,79 @@ def long_history_bench(ispa, device, iters=5) -> dict:
     return res
 
 
+def _graph_ms(fn, device, iters) -> float:
+    """Device time of fn's launches captured once and replayed iters times."""
+    side = torch.cuda.Stream(device)
+    stream = torch.cuda.current_stream(device)
+    fn()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        fn()
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / iters
+
+
+def w8a8_bench(ispa, w, device, peak_bf16: float, peak_hbm: float, iters=20) -> dict:
+    """The W8A8 variant of the post-transition L-layer (e4m3 projection with
+    per-token and per-output-channel scales) against the bf16 L-layer, both
+    timed as CUDA-graph replays on the same inputs.  The fp8 peak is the
+    measured bf16 peak times the nominal fp8 / bf16 ratio of 2."""
+    H, D, n = w.n_heads, w.d_model, w.n_q
+    x = synth.single_layer_inputs(w, 1)
+
+    def t(a):
+        return torch.from_numpy(a).to(torch.bfloat16).to(device)
+
+    q = t(x["q"])
+    local = [(t(x["k_sink"]), t(x["v_sink"])), (t(x["k_cur"]), t(x["v_cur"]))]
+    W = t(synth.weight(w, 0))
+    status = ispa.new_status(device)
+    y16, a16 = torch.empty(n, D, dtype=torch.bfloat16, device=device), torch.empty(n, D, dtype=torch.bfloat16,
+                                                                                  device=device)
+    qwt, sw = ispa.quantize_e4m3_weight(W)
+    out8 = ispa.local_attention_project_w8a8(q, local, qwt, sw, H, status=status)
+    ispa.local_attention_project(q, local, W, H, y=y16, a_loc=a16, status=status)
+    qa, sa = ispa.quantize_e4m3_rows(a16)
+    yp = torch.empty(n, D, dtype=torch.bfloat16, device=device)
+    ms = {
+        "l_layer_w8a8": _graph_ms(lambda: ispa.local_attention_project_w8a8(q, local, qwt, sw, H, out=out8,
+                                                                            status=status), device, iters),
+        "l_layer_bf16": _graph_ms(lambda: ispa.local_attention_project(q, local, W, H, y=y16, a_loc=a16,
+                                                                       status=status), device, iters),
+        "project_w8a8": _graph_ms(lambda: ispa.project_w8a8(qa, sa, qwt, sw, yp), device, iters),
+        "project_bf16": _graph_ms(lambda: ispa.project(a16, W, yp), device, iters),
+        "quantize_rows": _graph_ms(lambda: ispa.quantize_e4m3_rows(a16, qa, sa), device, iters),
+        "quantize_weight": _graph_ms(lambda: ispa.quantize_e4m3_weight(W, qwt, sw), device, iters),
+    }
+    torch.cuda.synchronize(device)
+    if int(status[0].item()) != 0:
+        raise RuntimeError("device status during the W8A8 benchmark")
+    flops = 2.0 * n * D * D
+    pk8 = 2.0 * peak_bf16
+    q_bytes = n * D * 2 + n * D + n * 4
+    diff = (out8["y"].float() - y16.float()).norm() / y16.float().norm()
+    return {
+        "workload": "wan1.3b L-layer: local attention (4680 queries, 6240 keys) + y = A_loc W_new, "
+                    "W8A8 = e4m3 codes, per-token and per-output-channel fp32 scales",
+        "ms": {k: round(v, 4) for k, v in ms.items()},
+        "project_w8a8_tflops": round(flops / (ms["project_w8a8"] * 1e-3) / 1e12, 1),
+        "project_w8a8_frac_of_fp8_peak": round(flops / (ms["project_w8a8"] * 1e-3) / 1e12 / pk8, 4),
+        "fp8_peak_tflops": round(pk8, 1),
+        "quantize_rows_gbs": round(q_bytes / (ms["quantize_rows"] * 1e-3) / 1e9, 1),
+        "quantize_rows_frac_of_hbm": round(q_bytes / (ms["quantize_rows"] * 1e-3) / 1e9 / peak_hbm, 4),
+        "l_layer_speedup_vs_bf16": round(ms["l_layer_bf16"] / ms["l_layer_w8a8"], 4),
+        "y_rel_diff_vs_bf16": round(float(diff), 5),
+    }
+
+
 def merge_bench(ispa, w, device, sets=4, iters=20) -> float:
     H, D, n = w.n_heads, w.d_model, w.n_q
     g = torch.Generator(device=device).manual_seed(0)
@@ -668,7 +752,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer streaming rollout")
-    ap.add_argument("--profile", choices=["dual", "full", "local", "gram", "project", "merge", "absorb"],
+    ap.add_argument("--profile", choices=["dual", "full", "local", "gram", "project", "merge", "absorb",
+                                          "project_w8a8", "quantize_rows"],
                     help="run only this op --steps times on the wan1.3b shapes (for ncu captures), no timing")
     args = ap.parse_args()
     if args.warmup < 3:
