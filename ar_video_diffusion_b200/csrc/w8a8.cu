@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(256) weight_codes_t_kernel(const __nv_bfloat16
       bf16x8(__ldg(reinterpret_cast<const uint4*>(w + (int64_t)k * N + n)), f);
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        const uint16_t p = cvt_e4m3x2(__fdiv_rn(f[e], __ldg(scale + n + e)), __fdiv_rn(f[e + 1], __ldg(scale + n + e + 1)));
+        const uint16_t p = cvt_e4m3x2(__fdiv_rn(f[e], __ldg(scale + n + e)),
+                                      __fdiv_rn(f[e + 1], __ldg(scale + n + e + 1)));
         c[e] = (uint8_t)(p & 0xFF);
         c[e + 1] = (uint8_t)(p >> 8);
       }
