@@ -358,3 +358,49 @@ def test_synth_bf16_rounding_is_rne():
     assert np.array_equal(r, t)
     y = np.random.default_rng(3).standard_normal(10000).astype(np.float32) * 7
     assert np.array_equal(synth.round_bf16(y), torch.from_numpy(y).to(torch.bfloat16).float().numpy())
+
+
+def _pages_claims():
+    """tests/golden/pages_claims.txt: key = value lines (the comments cite the pages)."""
+    import os
+    vals = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "pages_claims.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = (x.strip() for x in line.split("="))
+                vals[k] = float(v)
+    return vals
+
+
+def test_kv_removal_approaches_but_never_exceeds_the_pages_bound():
+    """Half the layers absorbed: the KV fraction removed grows with the video
+    and tends to the pages' "up to 50%" without reaching it (an L-layer keeps
+    the sink and the current chunk)."""
+    claims = _pages_claims()
+    L = 30
+    K = int(claims["l_layers_fraction"] * L)
+    mask = orc.layer_mask(L, range(0, L, 2))
+    assert bin(mask).count("1") == K
+    prev = 0.0
+    for c in (4, 8, 23, 100, 1000, 10000):
+        all_f = orc.kv_bytes(c, L, 0, True, 1560, 3, 1536, 2)
+        removed = 1 - orc.kv_bytes(c, L, mask, True, 1560, 3, 1536, 2) / all_f
+        assert prev < removed < claims["kv_removed_upper_bound"]
+        prev = removed
+    # closed form: 1/2 * (1 - (sink + chunk) / (frames up to chunk c))
+    c = 10000
+    frames = 3 * (c + 1)
+    assert abs(prev - 0.5 * (1 - (1 + 3) / frames)) < 1e-12
+    assert claims["kv_removed_upper_bound"] - prev < 1e-3
+
+
+def test_warm_up_reading_meets_the_pages_minimum():
+    """The primary reading's warm-up is 4 chunks of 3 latent frames = 12
+    frames, the pages' sufficient minimum, giving 18720 statistics rows per
+    layer at 1560 tokens per frame."""
+    claims = _pages_claims()
+    from ar_video_diffusion_b200 import synth
+    w = synth.WORKLOADS["wan1.3b"]
+    assert w.warm_chunks * w.chunk_frames == claims["t_warm_frames_min"]
+    assert w.warm_chunks * w.n_q == 18720
