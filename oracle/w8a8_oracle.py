@@ -34,6 +34,11 @@ Pinned by tests/test_oracle_w8a8.py:
   * exactness when every scale is 1 and every value lies on the grid;
   * power-of-two equivariance of the row and column scales;
   * the error bound of a 3-bit mantissa.
+The block-scaled (MXFP8) variant at the end of this file is pinned there too:
+  * its exponents against a brute-force search;
+  * its codes against torch's conversion of the exactly scaled values;
+  * exactness on the grid, per-block power-of-two equivariance, the error
+    bound, and plain loops.
 """
 from __future__ import annotations
 
@@ -110,3 +115,77 @@ def project_w8a8(a, w) -> np.ndarray:
     qa, sa = quantize_rows(a)
     qw, sw = quantize_cols(w)
     return project_codes(qa, sa, qw, sw)
+
+
+# ---------------------------------------------------------------------------
+# Block-scaled variant (MXFP8): the planned layout for activation codes written
+# by the attention epilogue.  A CTA there holds one head's 128 channels of a
+# row, so it can scale blocks of 32 consecutive elements along K but not a
+# whole row.  Readings:
+#   * one power-of-two scale 2^e per block of MX_BLOCK = 32 consecutive
+#     elements along K (a row of A, a column of W);
+#   * e is the smallest integer with amax * 2^-e <= 448, so no element
+#     saturates.  An all-zero block gets e = 0.  e is clamped to the ue8m0
+#     range [-127, 127];
+#   * the code is the e4m3 value nearest to x * 2^-e, with ties to even.  The
+#     scaling is exact, so there is no rounding decision before the
+#     conversion;
+#   * y[i, j] = sum over blocks b of 2^(ea[i, b] + ew[b, j])
+#     * sum over k in b of dec(qa[i, k]) * dec(qw[k, j]).
+MX_BLOCK = 32
+
+
+def mx_block_exponents(amax) -> np.ndarray:
+    """Smallest e with amax * 2^-e <= 448 (0 for amax == 0), clamped to ue8m0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))
+    e0 = ex.astype(np.int64) - 1 - 8          # amax * 2^-e0 lies in [256, 512)
+    e = np.where(np.ldexp(amax, -e0) <= E4M3_MAX, e0, e0 + 1)
+    e = np.where(amax > 0, e, 0)
+    return np.clip(e, -127, 127).astype(np.int64)
+
+
+def _mx_blocks(x, axis):
+    """View x with the K axis split into (blocks, MX_BLOCK); K % 32 == 0."""
+    x = np.asarray(x, dtype=np.float32)
+    if axis == 1:
+        n, K = x.shape
+        return x.reshape(n, K // MX_BLOCK, MX_BLOCK)
+    K, N = x.shape
+    return x.reshape(K // MX_BLOCK, MX_BLOCK, N)
+
+
+def mx_quantize_rows(x) -> Tuple[np.ndarray, np.ndarray]:
+    """Codes [n, K] and block exponents [n, K/32] of x [n, K] (blocks along rows)."""
+    xb = _mx_blocks(x, 1).astype(np.float64)
+    e = mx_block_exponents(np.max(np.abs(xb), axis=2))
+    q = e4m3_encode(np.ldexp(xb, -e[:, :, None]).astype(np.float32))
+    return q.reshape(np.shape(x)), e
+
+
+def mx_quantize_cols(w) -> Tuple[np.ndarray, np.ndarray]:
+    """Codes [K, N] and block exponents [K/32, N] of w [K, N] (blocks along columns)."""
+    wb = _mx_blocks(w, 0).astype(np.float64)
+    e = mx_block_exponents(np.max(np.abs(wb), axis=1))
+    q = e4m3_encode(np.ldexp(wb, -e[:, None, :]).astype(np.float32))
+    return q.reshape(np.shape(w)), e
+
+
+def mx_project_codes(qa, ea, qw, ew) -> np.ndarray:
+    """y from MX codes: one exactly scaled partial product per K block (fp64)."""
+    n, K = qa.shape
+    N = qw.shape[1]
+    y = np.zeros((n, N))
+    da, dw = e4m3_decode(qa), e4m3_decode(qw)
+    for b in range(K // MX_BLOCK):
+        ks = slice(b * MX_BLOCK, (b + 1) * MX_BLOCK)
+        part = da[:, ks] @ dw[ks, :]
+        y += np.ldexp(part, ea[:, b][:, None] + ew[b, :][None, :])
+    return y
+
+
+def project_mxfp8(a, w) -> np.ndarray:
+    """The block-scaled W8A8 projection of a [n, K] by w [K, N]."""
+    qa, ea = mx_quantize_rows(a)
+    qw, ew = mx_quantize_cols(w)
+    return mx_project_codes(qa, ea, qw, ew)

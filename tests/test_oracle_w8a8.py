@@ -161,3 +161,99 @@ def test_project_codes_brute_force_loops():
             for k in range(5):
                 acc += w8.e4m3_decode(qa[i, k]) * w8.e4m3_decode(qw[k, j])
             assert got[i, j] == pytest.approx(float(sa[i]) * float(sw[j]) * acc, rel=1e-15, abs=1e-300)
+
+
+# ----------------------------------------------------------- block-scaled (MXFP8)
+def _bf16_normal(rng, shape):
+    """Normal draws rounded to bf16 (round to nearest even), as fp32."""
+    x = rng.standard_normal(shape).astype(np.float32)
+    u = x.view(np.uint32)
+    return ((u + np.uint32(0x7FFF) + ((u >> 16) & 1)) & np.uint32(0xFFFF0000)).view(np.float32)
+
+
+def test_mx_exponent_is_the_smallest_in_range_brute_force():
+    rng = np.random.default_rng(30)
+    amax = np.concatenate([np.exp2(rng.uniform(-30, 30, 500)),
+                           448.0 * np.exp2(np.arange(-5, 6)),              # exactly on the boundary
+                           np.nextafter(448.0 * np.exp2(np.arange(-5, 6)), np.inf)])  # just above it
+    e = w8.mx_block_exponents(amax)
+    for a, ei in zip(amax, e):
+        ok = [k for k in range(-140, 140) if a * 2.0 ** -k <= 448.0]
+        assert ei == min(ok), (a, ei)
+    assert np.array_equal(w8.mx_block_exponents(448.0 * np.exp2(np.arange(-5, 6))), np.arange(-5, 6))
+    assert w8.mx_block_exponents(np.array([0.0]))[0] == 0
+    assert w8.mx_block_exponents(np.array([1e-45]))[0] == -127  # clamped to the ue8m0 range
+
+
+def test_mx_codes_match_torch_on_exactly_scaled_blocks():
+    rng = np.random.default_rng(31)
+    x = _bf16_normal(rng, (37, 96)) * np.exp2(rng.integers(-12, 12, (37, 1))).astype(np.float32)
+    q, e = w8.mx_quantize_rows(x)
+    assert e.shape == (37, 3)
+    scaled = (x.reshape(37, 3, 32) * np.exp2(-e[:, :, None])).reshape(37, 96).astype(np.float32)
+    assert np.all(np.abs(scaled) <= 448.0)
+    ref = torch.from_numpy(scaled).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+    qw, ew = w8.mx_quantize_cols(x.T.copy())
+    assert np.array_equal(qw, q.T) and np.array_equal(ew, e.T)
+
+
+def test_mx_projection_exact_on_grid():
+    """Blocks whose values lie on the e4m3 grid and reach 448 have exponent 0
+    and their codes are the values: the product is exact."""
+    rng = np.random.default_rng(32)
+    grid = w8.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    a = rng.choice(grid, (5, 64)) * rng.choice([-1.0, 1.0], (5, 64))
+    w = rng.choice(grid, (64, 7)) * rng.choice([-1.0, 1.0], (64, 7))
+    a[:, [3, 40]] = 448.0
+    w[[1, 33], :] = -448.0
+    qa, ea = w8.mx_quantize_rows(a)
+    qw, ew = w8.mx_quantize_cols(w)
+    assert np.all(ea == 0) and np.all(ew == 0)
+    assert np.array_equal(w8.project_mxfp8(a, w), a @ w)
+
+
+def test_mx_per_block_power_of_two_equivariance():
+    """Scaling one 32-element block of a row by 2^k moves only that block's
+    exponent by k; the codes and every other output stay exactly the same."""
+    rng = np.random.default_rng(33)
+    a = rng.standard_normal((4, 96)).astype(np.float32)
+    w = rng.standard_normal((96, 5)).astype(np.float32)
+    qa, ea = w8.mx_quantize_rows(a)
+    a2 = a.copy()
+    a2[1, 32:64] *= 16.0
+    qa2, ea2 = w8.mx_quantize_rows(a2)
+    assert np.array_equal(qa2, qa)
+    assert ea2[1, 1] == ea[1, 1] + 4 and np.array_equal(np.delete(ea2.ravel(), 4), np.delete(ea.ravel(), 4))
+    y, y2 = w8.project_mxfp8(a, w), w8.project_mxfp8(a2, w)
+    assert np.array_equal(np.delete(y2, 1, 0), np.delete(y, 1, 0))
+
+
+def test_mx_error_bound_and_no_saturation():
+    rng = np.random.default_rng(34)
+    a = (rng.standard_normal((64, 256)) * np.exp2(rng.uniform(-8, 8, (64, 8))).repeat(32, 1)).astype(np.float32)
+    qa, ea = w8.mx_quantize_rows(a)
+    deq = (w8.e4m3_decode(qa).reshape(64, 8, 32) * np.exp2(ea[:, :, None])).reshape(64, 256)
+    normal = np.abs(a) * np.exp2(-ea.repeat(32, 1)) >= 2.0 ** -6
+    assert (np.abs(deq - a) / np.abs(a))[normal].max() <= 2.0 ** -4 * (1 + 1e-6)
+    assert np.all(qa & 0x7F != 0x7F)  # nothing saturates into the NaN code
+    w = (rng.standard_normal((256, 32)) / 16).astype(np.float32)
+    exact = a.astype(np.float64) @ w.astype(np.float64)
+    err = np.linalg.norm(w8.project_mxfp8(a, w) - exact) / np.linalg.norm(exact)
+    assert 1e-3 < err < 0.05
+
+
+def test_mx_project_codes_brute_force_loops():
+    rng = np.random.default_rng(35)
+    qa = rng.integers(0, 0x7E, (2, 64)).astype(np.uint8)
+    qw = rng.integers(0, 0x7E, (64, 3)).astype(np.uint8) | rng.choice([0, 0x80], (64, 3)).astype(np.uint8)
+    ea = rng.integers(-5, 5, (2, 2))
+    ew = rng.integers(-5, 5, (2, 3))
+    got = w8.mx_project_codes(qa, ea, qw, ew)
+    for i in range(2):
+        for j in range(3):
+            acc = 0.0
+            for k in range(64):
+                b = k // 32
+                acc += w8.e4m3_decode(qa[i, k]) * w8.e4m3_decode(qw[k, j]) * 2.0 ** (ea[i, b] + ew[b, j])
+            assert got[i, j] == pytest.approx(acc, rel=1e-14, abs=1e-300)
