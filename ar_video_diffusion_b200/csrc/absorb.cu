@@ -506,7 +506,8 @@ static void layer_error_impl(const float* G, const float* R, const float* E, con
   const int sms = num_sms();
   symmetrize_kernel<<<sms * 4, 256, 0, st>>>(G, Gs, D);
   symmetrize_kernel<<<sms * 4, 256, 0, st>>>(E, Es, D);
-  cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st);
+  // on failure nothing more is launched; the caller's check_launch reports the error
+  if (cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st) != cudaSuccess) return;
   double* num = num_den;
   double* den = num_den + 1;
   gemm_f32(st, D, D, D, 1.f, Gs, D, 1, dW, D, 1, 0.f, P, D);  // G dW

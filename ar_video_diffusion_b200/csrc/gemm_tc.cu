@@ -359,10 +359,9 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   if (!encode_map_bf16_2d(&p.a_map, a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&p.b_map[0], a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&p.b_map[1], a_delta, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
-  if (overwrite) {
-    cudaMemsetAsync(G, 0, (size_t)D * D * 4, stream);
-    cudaMemsetAsync(R, 0, (size_t)D * D * 4, stream);
-  }
+  if (overwrite && (cudaMemsetAsync(G, 0, (size_t)D * D * 4, stream) != cudaSuccess ||
+                    cudaMemsetAsync(R, 0, (size_t)D * D * 4, stream) != cudaSuccess))
+    return check_launch("cudaMemsetAsync of G, R");
   p.M = (int32_t)D;
   p.N = (int32_t)(2 * D);
   p.K = (int32_t)n_rows;
@@ -402,7 +401,8 @@ ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t ro
   if (!encode_map_bf16_2d(&p.a_map, x, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   p.b_map[0] = p.a_map;
   p.b_map[1] = p.a_map;
-  if (overwrite) cudaMemsetAsync(E, 0, (size_t)D * D * 4, stream);
+  if (overwrite && cudaMemsetAsync(E, 0, (size_t)D * D * 4, stream) != cudaSuccess)
+    return check_launch("cudaMemsetAsync of E");
   p.M = (int32_t)D;
   p.N = (int32_t)D;
   p.K = (int32_t)n_rows;
