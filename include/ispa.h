@@ -17,6 +17,10 @@
  *               K_hist, V_hist and run local attention with W_new = W + dW.
  *   [gist §3]   "Key Contributions" item 2: decomposition grounded in online
  *               softmax.
+ *   [gist sel]  "Dynamic Layer Selection": every layer is ranked by its
+ *               reconstruction error after the warm-up.
+ *   [gist §4]   "Experimental Results", item "Speedup": ISPA combined with
+ *               post-training W8A8 quantisation.
  *
  * Conventions shared by every entry point
  *   - Layout: token-major row-major matrices [n, D] with the heads interleaved,
