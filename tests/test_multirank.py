@@ -110,3 +110,119 @@ def test_reference_arm_rank0_line():
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["value"] > 0
+
+
+# ------------------------------------------------------ sharded hot path (host side)
+def test_query_shard_partitions_whole_tiles():
+    sys.path.insert(0, ROOT)
+    from ar_video_diffusion_b200 import sharded
+    for n in (1, 127, 128, 129, 300, 4680, 18720):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [sharded.query_shard(n, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == n
+            for (b0, e0), (b1, e1) in zip(ranges, ranges[1:]):
+                assert e0 == b1  # contiguous, no overlap
+            sizes_in_tiles = [-(-(e - b) // 128) for b, e in ranges]
+            assert max(sizes_in_tiles) - min(sizes_in_tiles) <= 1
+            for b, e in ranges:
+                # a range starts on a tile boundary (an empty one sits at n) and ends on one or at n
+                assert (b % 128 == 0 or b == e == n) and (e % 128 == 0 or e == n)
+    with pytest.raises(ValueError):
+        sharded.query_shard(10, 2, 2)
+
+
+STATS_CODE = r"""
+import datetime, json, os, sys
+sys.path.insert(0, os.environ["ISPA_ROOT"])
+import numpy as np
+import torch
+import torch.distributed as dist
+from ar_video_diffusion_b200 import sharded
+from oracle import ispa_oracle as orc
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+rank, world = dist.get_rank(), dist.get_world_size()
+rng = np.random.default_rng(5)                      # the same seeded rows on every rank
+n, D = 700, 48
+A = rng.standard_normal((n, D))
+Dl = 0.1 * rng.standard_normal((n, D))
+b, e = sharded.query_shard(n, world, rank)
+# stand-in for the statistics kernel on this rank's rows (CPU, fp64)
+stats = torch.zeros(2, D, D, dtype=torch.float64)
+stats[0] = torch.from_numpy(A[b:e].T @ A[b:e])
+stats[1] = torch.from_numpy(A[b:e].T @ Dl[b:e])
+sharded.allreduce_statistics(stats)
+G, R = orc.gram(A, Dl)
+err = max(float(np.abs(stats[0].numpy() - G).max() / np.abs(G).max()),
+          float(np.abs(stats[1].numpy() - R).max() / np.abs(R).max()))
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "rows": [b, e], "err": err}))
+"""
+
+
+def test_statistics_allreduce_two_gloo_ranks():
+    outs = _run_ranks(STATS_CODE, 2, {})
+    res = []
+    for rc, out, err in outs:
+        assert rc == 0, err[-2000:]
+        res.append(json.loads(out.strip().splitlines()[-1]))
+    rows = sorted(tuple(r["rows"]) for r in res)
+    assert rows[0][0] == 0 and rows[0][1] == rows[1][0] and rows[1][1] == 700
+    for r in res:
+        assert r["err"] < 1e-12  # the sum of the partial Gram matrices is the oracle's Gram
+
+
+ABSORB_CODE = r"""
+import datetime, json, os, sys
+sys.path.insert(0, os.environ["ISPA_ROOT"])
+import numpy as np
+import torch
+import torch.distributed as dist
+from ar_video_diffusion_b200 import sharded
+from oracle import ispa_oracle as orc
+dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+rank, world = dist.get_rank(), dist.get_world_size()
+solved = []
+
+def absorb_solve(G, R, W, lambda_rel=1e-2, workspace=None, status=None):
+    # stand-in for the device solve: the oracle's, on this rank
+    Gn, Rn, Wn = (t.numpy().astype(np.float64) for t in (G, R, W))
+    Gs = np.tril(Gn) + np.tril(Gn, -1).T
+    dW = orc.absorb(Gs, Rn, Wn, orc.ridge_lambda(Gs, lambda_rel))
+    solved.append(len(solved))
+    return torch.from_numpy(dW), torch.from_numpy(Wn + dW)
+
+sharded.ispa.absorb_solve = absorb_solve
+D, layers = 16, [0, 2, 4, 6, 8]
+rng = np.random.default_rng(9)
+stats, W = {}, {}
+for l in layers:
+    A = rng.standard_normal((40, D))
+    Dl = 0.1 * rng.standard_normal((40, D))
+    s = torch.zeros(2, D, D, dtype=torch.float64)
+    s[0] = torch.from_numpy(A.T @ A)
+    s[1] = torch.from_numpy(A.T @ Dl)
+    stats[l] = s
+    W[l] = torch.from_numpy(rng.standard_normal((D, D)) / 4)
+w_new = sharded.absorb_layers(stats, W, world, rank)
+mine = [l for l in layers if sharded.absorb_owner(l, world) == rank]
+out = {"rank": rank, "n_solved": len(solved), "mine": mine,
+       "w_new": {str(l): float(w_new[l].sum()) for l in layers}}
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps(out))
+"""
+
+
+def test_absorb_layers_owned_once_and_broadcast_two_gloo_ranks():
+    outs = _run_ranks(ABSORB_CODE, 2, {})
+    res = []
+    for rc, out, err in outs:
+        assert rc == 0, err[-2000:]
+        res.append(json.loads(out.strip().splitlines()[-1]))
+    # every layer solved exactly once, by its owner; every rank ends with the same W_new
+    owned = sorted(l for r in res for l in r["mine"])
+    assert owned == [0, 2, 4, 6, 8]
+    for r in res:
+        assert r["n_solved"] == len(r["mine"])
+    assert res[0]["w_new"] == res[1]["w_new"]
