@@ -12,8 +12,12 @@
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // library reserves kNoAllocBytes of device memory for it until the process
 // exits.  Its size bounds d_model at kNoAllocMaxD.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 
@@ -32,34 +36,65 @@ constexpr size_t kNoAllocBytes = (size_t)(4 * kNoAllocMaxD * kNoAllocMaxD + 256 
 static __device__ __align__(256) unsigned char g_absorb_scratch[kNoAllocBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_absorb_scratch on the current device, looked up once
-// per device (the lookup must run with that device current).
+std::mutex g_mu;
+// (context id, device address of g_absorb_scratch in that context).  The id
+// that cuCtxGetId returns is unique for the life of the process, so a context
+// that replaced a destroyed one (after cudaDeviceReset, say) never finds the
+// address the old context had.
+std::vector<std::pair<unsigned long long, void*>> g_scratch_by_ctx;
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context; 0 when there is none yet.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  *id = 0;
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  return !ctx || get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_absorb_scratch in the current device's context.  The
+// lookup runs once per context, with that context current (on the first call
+// a context sees); later calls find the cached address.
 ispa_status_t scratch_for_current_device(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    set_last_error("cudaGetDevice failed: %s", cudaGetErrorString(e));
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) {
+    set_last_error("cuCtxGetCurrent / cuCtxGetId are not available from the driver");
     return ISPA_ERR_CUDA;
   }
-  if (dev < 0 || dev >= kMaxDevices) {
-    set_last_error("device index %d out of range", dev);
-    return ISPA_ERR_UNSUPPORTED;
-  }
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_absorb_scratch);
-    if (e != cudaSuccess || !p) {
-      set_last_error("cudaGetSymbolAddress of the absorb scratch failed: %s", cudaGetErrorString(e));
-      return ISPA_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
+  if (id != 0) {
+    for (const auto& e : g_scratch_by_ctx)
+      if (e.first == id) {
+        *out = e.second;
+        return ISPA_OK;
+      }
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_absorb_scratch);
+  if (e != cudaSuccess || !p) {
+    set_last_error("cudaGetSymbolAddress of the absorb scratch failed: %s", cudaGetErrorString(e));
+    return ISPA_ERR_CUDA;
+  }
+  if (id == 0 && !current_context_id(&id)) {  // the lookup made the runtime's context current
+    set_last_error("cuCtxGetId failed");
+    return ISPA_ERR_CUDA;
+  }
+  if (id != 0) g_scratch_by_ctx.emplace_back(id, p);
+  *out = p;
   return ISPA_OK;
 }
 }  // namespace

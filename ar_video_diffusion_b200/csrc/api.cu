@@ -364,6 +364,9 @@ extern "C" ispa_status_t ispa_chunk_token_ranges(int64_t chunk, int64_t frame_to
   if (!out) return invalid("out is NULL");
   if (chunk < 0 || frame_tokens < 0 || chunk_frames < 0 || sink_frames < 0)
     return invalid("sizes must be non-negative");
+  if (chunk > 0 && sink_frames > chunk * chunk_frames)
+    return invalid("the sink (%lld frames) must end before chunk %lld starts (frame %lld)", (long long)sink_frames,
+                   (long long)chunk, (long long)(chunk * chunk_frames));
   const int64_t F = frame_tokens, cf = chunk_frames;
   out[4] = chunk * cf * F;
   out[5] = (chunk + 1) * cf * F;
@@ -385,7 +388,7 @@ extern "C" int64_t ispa_kv_bytes(int64_t chunk, int32_t n_layers, uint64_t l_lay
       elem_bytes <= 0 || sink_frames < 0)
     return -1;
   int64_t r[6];
-  ispa_chunk_token_ranges(chunk, frame_tokens, chunk_frames, sink_frames, r);
+  if (ispa_chunk_token_ranges(chunk, frame_tokens, chunk_frames, sink_frames, r) != ISPA_OK) return -1;
   int64_t total = 0;
   for (int l = 0; l < n_layers; ++l) {
     const bool is_l = (l_layer_mask >> l) & 1u;

@@ -89,8 +89,11 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const uint4* __restrict_
       const int64_t li = (int64_t)h * n_q + r0 + rr;
       const float ll = __ldg(lse_loc + li), lh = __ldg(lse_hist + li);
       const float mx = fmaxf(ll, lh);
-      const float L = mx + logf(expf(ll - mx) + expf(lh - mx));
-      wts[rr][h] = make_float2(expf(ll - L), expf(lh - L));
+      // both branches empty: the union is empty too, so A_full = 0 and
+      // L = -inf (attention over no keys), with both weights 0
+      const bool none = mx == -INFINITY;
+      const float L = none ? -INFINITY : mx + logf(expf(ll - mx) + expf(lh - mx));
+      wts[rr][h] = none ? make_float2(0.f, 0.f) : make_float2(expf(ll - L), expf(lh - L));
       if (lse_full) lse_full[li] = L;
     }
     __syncthreads();

@@ -92,6 +92,7 @@ class Rollout:
         self.R = {l: torch.zeros(D, D, **f32) for l in self.stats_layers}
         self.E = {l: torch.zeros(D, D, **f32) for l in self.stats_layers} if self.rank else {}
         self.eps: List[float] = []      # reconstruction error of every layer (when ranked)
+        self.dW_ranked: Dict[int, torch.Tensor] = {}  # every ranked layer's dW (when ranked)
         self.select_ms = 0.0
         self.transitioned = False
         n_q = self.chunk_tokens
@@ -162,6 +163,7 @@ class Rollout:
             self.mask = 0
             for l in self.absorbed:
                 self.mask |= 1 << l
+        self.dW_ranked = {l: cand[l][0] for l in cand}
         for l in self.absorbed:
             self.dW[l], self.W_new[l] = cand[l]
         self.absorb_ms = [ev[l][0].elapsed_time(ev[l][1]) for l in self.absorbed]

@@ -11,9 +11,15 @@ summary, section 2) shards without changing its arithmetic:
   sums over rows.  Each rank accumulates its rows and one all-reduce (sum) of
   the packed [G | R] buffer gives every rank the full statistics, 2 D^2 fp32
   (18.9 MB at D = 1536).
-* Absorb (stage 2) and modulation (stage 3): layers are independent.  Layer l
-  is solved by rank l mod world, which then broadcasts W_new (D^2 in the
-  weight dtype) to the others, which need it for their rows of the L-layer.
+* Absorb (stage 2) and modulation (stage 3): layers are independent
+  ("Dynamic Layer Selection": the selected layers are absorbed one by one).
+  The i-th absorbed layer in increasing layer order is solved by rank
+  i mod world, so the ranks' shares differ by at most one layer whatever the
+  selected set (the even layers, or an instance-specific choice).  Every rank
+  first solves all of its layers back to back, then the owners broadcast
+  W_new (D^2 in the weight dtype) to the others, which need it for their rows
+  of the L-layer; the broadcasts are issued together and awaited at the end,
+  so no rank's solve waits for another rank's.
 
 Every step on a device runs in libispa's kernels through ``ispa``; this module
 only partitions rows and layers and issues the collectives.  The collectives
@@ -44,9 +50,12 @@ def query_shard(n_q: int, world: int, rank: int, tile: int = Q_TILE) -> Tuple[in
     return min(t0 * tile, n_q), min(t1 * tile, n_q)
 
 
-def absorb_owner(layer: int, world: int) -> int:
-    """The rank that solves layer `layer`'s absorb."""
-    return layer % world
+def absorb_owners(layers: Sequence[int], world: int) -> dict:
+    """layer -> the rank that solves its absorb: the i-th layer of the sorted
+    set goes to rank i mod world (balanced to within one layer)."""
+    if world <= 0:
+        raise ValueError("world must be positive")
+    return {l: i % world for i, l in enumerate(sorted(set(layers)))}
 
 
 def new_statistics(d_model: int, device) -> torch.Tensor:
@@ -89,16 +98,19 @@ def absorb_layers(stats_by_layer, W_by_layer, world: int, rank: int, lambda_rel:
 
     stats_by_layer / W_by_layer: dicts layer -> all-reduced [2, D, D] stats /
     weight [D, D].  Returns a dict layer -> W_new, identical on every rank.
-    Each rank takes the same broadcasts in the same (sorted layer) order."""
+    This rank's solves run back to back first; then every rank takes the same
+    broadcasts in the same (sorted layer) order, issued asynchronously and
+    awaited together."""
+    owners = absorb_owners(stats_by_layer.keys(), world)
     w_new = {}
     for l in sorted(stats_by_layer):
-        W = W_by_layer[l]
-        if absorb_owner(l, world) == rank:
-            _, wn = ispa.absorb_solve(stats_by_layer[l][0], stats_by_layer[l][1], W, lambda_rel=lambda_rel,
-                                      workspace=workspace, status=status)
+        if owners[l] == rank:
+            _, w_new[l] = ispa.absorb_solve(stats_by_layer[l][0], stats_by_layer[l][1], W_by_layer[l],
+                                            lambda_rel=lambda_rel, workspace=workspace, status=status)
         else:
-            wn = torch.empty_like(W)
-        if dist.is_initialized() and world > 1:
-            dist.broadcast(wn, src=absorb_owner(l, world), group=group)
-        w_new[l] = wn
+            w_new[l] = torch.empty_like(W_by_layer[l])
+    if dist.is_initialized() and world > 1:
+        works = [dist.broadcast(w_new[l], src=owners[l], group=group, async_op=True) for l in sorted(w_new)]
+        for wk in works:
+            wk.wait()
     return w_new

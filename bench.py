@@ -337,7 +337,9 @@ def run_ours(args, rank, world, device):
     pk0, _ = peaks()
     w8a8 = w8a8_bench(ispa, w, device, pk0["bf16_tflops"], pk0["hbm_gbs"])
 
+    configs = configs_bench(ispa, device, pk0["bf16_tflops"], pk0["hbm_gbs"])
     rollout = None if args.no_rollout else run_rollout(device)
+    rollout_12warm = None if args.no_rollout else run_rollout_12warm(device)
 
     pk, src = peaks()
     tc_peak = pk["bf16_tflops"]
@@ -389,8 +391,10 @@ def run_ours(args, rank, world, device):
         "clocks": clk,
         "gpu_launches": args.steps * (7 + absorb_launches(D)),
         "long_history": long_hist,
+        "configs": configs,
         "w8a8": w8a8,
         "rollout": rollout,
+        "rollout_12warm": rollout_12warm,
     }
     return res
 
@@ -522,6 +526,177 @@ def run_layer_selection(device) -> dict:
         "rank_ms_per_layer": round(ro.select_ms / w.n_layers, 4),
     }
     assert ro.absorbed == ispa.select_layers(eps, len(even))
+    del ro
+    torch.cuda.empty_cache()
+    return res
+
+
+def _frames_device(w, layer: int, frames, device):
+    """K, V of the listed latent frames from the seeded device generator."""
+    F, D = w.frame_tokens, w.d_model
+    k = torch.empty(len(frames) * F, D, dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    for i, f in enumerate(frames):
+        kf, vf = synth.frame_kv_device(w, 0, f, device)
+        k[i * F:(i + 1) * F].copy_(kf)
+        v[i * F:(i + 1) * F].copy_(vf)
+    return k, v
+
+
+def _single_layer_device(w, device):
+    """One warm-up chunk of a single-layer workload on the device: Q and the
+    sink / history / current K, V (device generator, the host recipe's shapes)."""
+    fr = synth.single_layer_frames(w, 1)
+    ks, vs = _frames_device(w, 0, fr["sink"], device)
+    kh, vh = _frames_device(w, 0, fr["hist"], device)
+    kc, vc = _frames_device(w, 0, fr["cur"], device)
+    q = synth.chunk_q_device(w, 0, 1, device)
+    return q, [(ks, vs), (kc, vc)], [(kh, vh)]
+
+
+def _rows_like(src: torch.Tensor, n_rows: int) -> torch.Tensor:
+    """n_rows rows made of repeats of src's rows (statistics inputs of the
+    workload's size; the values do not change the work)."""
+    reps = (n_rows + src.shape[0] - 1) // src.shape[0]
+    return src.repeat(reps, 1)[:n_rows].contiguous()
+
+
+def configs_bench(ispa, device, peak_bf16: float, peak_hbm: float, iters=10) -> dict:
+    """The other benchmark configurations, each timed as CUDA-graph replays:
+    tiny fp32 (latency of every step), long history (93600 history tokens:
+    dual attention, LSE merge and a 93600-row statistics accumulation) and
+    Wan-14B shapes (dual attention, 18720-row statistics, 5120 x 5120 absorb)."""
+    res = {}
+    status = ispa.new_status(device)
+
+    # ---- tiny fp32: 2 heads x 64, 64 queries, 16 sink + 64 current + 256 history keys, D = 128
+    w = synth.WORKLOADS["tiny_f32"]
+    H, D = w.n_heads, w.d_model
+    x = synth.single_layer_inputs(w, 1)
+    t32 = {k: torch.from_numpy(v).to(device) for k, v in x.items()}
+    loc = [(t32["k_sink"], t32["v_sink"]), (t32["k_cur"], t32["v_cur"])]
+    his = [(t32["k_hist"], t32["v_hist"])]
+    out = ispa.dual_attention(t32["q"], loc, his, H, status=status)
+    oh = ispa.dual_attention(t32["q"], [], his, H, dual=False, status=status)
+    a_rows = _rows_like(out["a_loc"], w.warm_chunks * w.n_q)
+    d_rows = _rows_like(out["a_delta"], w.warm_chunks * w.n_q)
+    G, R = torch.empty(D, D, device=device), torch.empty(D, D, device=device)
+    ispa.gram_accumulate(a_rows, d_rows, G, R, zero_first=True)
+    W = torch.from_numpy(synth.weight(w, 0)).to(device)
+    ws = ispa.absorb_workspace(D, device)
+    dW, Wn = torch.empty(D, D, device=device), torch.empty_like(W)
+    mo = {"a_full": torch.empty_like(out["a_loc"]), "a_delta": torch.empty_like(out["a_loc"]),
+          "lse_full": torch.empty_like(out["lse_loc"])}
+    ms = {
+        "dual_attention": _graph_ms(lambda: ispa.dual_attention(t32["q"], loc, his, H, out=out, status=status),
+                                    device, iters),
+        "lse_merge": _graph_ms(lambda: ispa.lse_merge(out["a_loc"], out["lse_loc"], oh["a_full"], oh["lse_full"], H,
+                                                      out=mo), device, iters),
+        "gram_256_rows": _graph_ms(lambda: ispa.gram_accumulate(a_rows, d_rows, G, R, zero_first=True), device, iters),
+        "absorb_solve": _graph_ms(lambda: ispa.absorb_solve(G, R, W, workspace=ws, status=status, delta_w=dW,
+                                                            w_new=Wn), device, iters),
+    }
+    res["tiny_f32"] = {"workload": "tiny fp32: 2 heads x 64, 64 queries, 16 sink + 64 current + 256 history keys, "
+                                   "256 statistics rows, D = 128 (latency only; fp32 on the CUDA cores)",
+                       "ms": {k: round(v, 4) for k, v in ms.items()},
+                       "step_ms": round(sum(ms.values()), 4)}
+
+    # ---- long history: wan1.3b shapes, 93600 history tokens, 93600-row statistics
+    w = synth.WORKLOADS["long_hist"]
+    H, D = w.n_heads, w.d_model
+    q, loc, his = _single_layer_device(w, device)
+    out = ispa.dual_attention(q, loc, his, H, status=status)
+    oh = ispa.dual_attention(q, [], his, H, dual=False, status=status)
+    n_rows = w.warm_chunks * w.n_q
+    a_rows, d_rows = _rows_like(out["a_loc"], n_rows), _rows_like(out["a_delta"], n_rows)
+    G, R = torch.empty(D, D, device=device), torch.empty(D, D, device=device)
+    t_dual = _graph_ms(lambda: ispa.dual_attention(q, loc, his, H, out=out, status=status), device, iters)
+    mo = {"a_full": torch.empty_like(out["a_loc"]), "a_delta": torch.empty_like(out["a_loc"]),
+          "lse_full": torch.empty_like(out["lse_loc"])}
+    t_merge = _graph_ms(lambda: ispa.lse_merge(out["a_loc"], out["lse_loc"], oh["a_full"], oh["lse_full"], H, out=mo),
+                        device, iters)
+    t_gram = _graph_ms(lambda: ispa.gram_accumulate(a_rows, d_rows, G, R, zero_first=True), device, iters)
+    F_attn = attn_flops(w)
+    merge_bytes = w.n_q * D * 2 * 4 + H * w.n_q * 4 * 3
+    res["long_hist"] = {
+        "workload": "long history: wan1.3b shapes, 1560 sink + 4680 current + 93600 history keys; statistics over "
+                    "93600 rows",
+        "dual_attention_ms": round(t_dual, 4),
+        "dual_attention_tflops": round(F_attn / (t_dual * 1e-3) / 1e12, 1),
+        "dual_attention_frac": round(F_attn / (t_dual * 1e-3) / 1e12 / peak_bf16, 4),
+        "lse_merge_ms": round(t_merge, 4),
+        "lse_merge_gbs": round(merge_bytes / (t_merge * 1e-3) / 1e9, 1),
+        "lse_merge_frac": round(merge_bytes / (t_merge * 1e-3) / 1e9 / peak_hbm, 4),
+        "lse_merge_note": "one launch, inputs partly L2-resident (58.2 MB < 126 MB L2)",
+        "gram_93600_rows_ms": round(t_gram, 4),
+        "gram_tflops": round(gram_flops(w, n_rows) / (t_gram * 1e-3) / 1e12, 1),
+        "gram_frac": round(gram_flops(w, n_rows) / (t_gram * 1e-3) / 1e12 / peak_bf16, 4),
+    }
+    del q, loc, his, out, oh, mo, a_rows, d_rows, G, R
+    torch.cuda.empty_cache()
+
+    # ---- Wan-14B shapes: 40 heads x 128 (D = 5120), 18720 history keys, 18720-row statistics, 5120^2 absorb
+    w = synth.WORKLOADS["wan14b"]
+    H, D = w.n_heads, w.d_model
+    q, loc, his = _single_layer_device(w, device)
+    out = ispa.dual_attention(q, loc, his, H, status=status)
+    n_rows = w.warm_chunks * w.n_q
+    a_rows, d_rows = _rows_like(out["a_loc"], n_rows), _rows_like(out["a_delta"], n_rows)
+    G, R = torch.empty(D, D, device=device), torch.empty(D, D, device=device)
+    ispa.gram_accumulate(a_rows, d_rows, G, R, zero_first=True)
+    W = synth.weight_device(w, 0, device)
+    ws = ispa.absorb_workspace(D, device)
+    dW, Wn = torch.empty(D, D, device=device), torch.empty_like(W)
+    t_dual = _graph_ms(lambda: ispa.dual_attention(q, loc, his, H, out=out, status=status), device, iters)
+    t_gram = _graph_ms(lambda: ispa.gram_accumulate(a_rows, d_rows, G, R, zero_first=True), device, iters)
+    t_abs = _graph_ms(lambda: ispa.absorb_solve(G, R, W, workspace=ws, status=status, delta_w=dW, w_new=Wn),
+                      device, 3)
+    F_attn = attn_flops(w)
+    res["wan14b"] = {
+        "workload": "wan14b: 40 heads x 128 (D = 5120), 4680 queries, 1560 sink + 4680 current + 18720 history "
+                    "keys; statistics over 18720 rows; absorb on 5120 x 5120",
+        "dual_attention_ms": round(t_dual, 4),
+        "dual_attention_tflops": round(F_attn / (t_dual * 1e-3) / 1e12, 1),
+        "dual_attention_frac": round(F_attn / (t_dual * 1e-3) / 1e12 / peak_bf16, 4),
+        "gram_18720_rows_ms": round(t_gram, 4),
+        "gram_tflops": round(gram_flops(w, n_rows) / (t_gram * 1e-3) / 1e12, 1),
+        "gram_frac": round(gram_flops(w, n_rows) / (t_gram * 1e-3) / 1e12 / peak_bf16, 4),
+        "absorb_ms_per_layer": round(t_abs, 3),
+        "absorb_tflops": round(solve_flops(D) / (t_abs * 1e-3) / 1e12, 2),
+        "absorb_frac": round(solve_flops(D) / (t_abs * 1e-3) / 1e12 / peak_bf16, 4),
+    }
+    torch.cuda.synchronize(device)
+    if int(status[0].item()) != 0:
+        raise RuntimeError("device status during the configuration benchmarks")
+    del q, loc, his, out, a_rows, d_rows, G, R, W, ws, dW, Wn
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_rollout_12warm(device) -> dict:
+    """The secondary reading of the rollout's warm-up: 12 warm-up chunks
+    (36 latent frames, 56160 statistics rows per absorbed layer) instead of
+    T_warm = 12 latent frames, then the same 20 chunks."""
+    from ar_video_diffusion_b200.rollout import Rollout
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["rollout"], warm_chunks=12)
+    ro = Rollout(w, device=device)
+    reps = ro.run()
+    post = [r for r in reps if r.phase == "post"]
+    warm = [r for r in reps if r.phase == "warmup"]
+    last = reps[-1]
+    res = {
+        "workload": "rollout, secondary warm-up reading: 30 layers, 1.3B shapes, 12 warm-up chunks (56160 rows) + "
+                    "20 post-transition chunks, even layers absorbed",
+        "chunk_ms": [round(r.gpu_ms, 3) for r in reps],
+        "warmup_chunk_ms_mean": round(sum(r.gpu_ms for r in warm) / len(warm), 3),
+        "post_chunk_ms_first": round(post[0].gpu_ms, 3),
+        "post_chunk_ms_last": round(post[-1].gpu_ms, 3),
+        "absorb_ms_per_layer": round(sum(ro.absorb_ms) / len(ro.absorb_ms), 4),
+        "kv_bytes_last": last.kv_bytes,
+        "kv_bytes_all_f_last": last.kv_bytes_all_f,
+        "kv_removed_frac": round(1 - last.kv_bytes / last.kv_bytes_all_f, 4),
+    }
     del ro
     torch.cuda.empty_cache()
     return res
@@ -713,14 +888,68 @@ def oracle_sample(rows: int):
     return run, flops
 
 
-def cpu_baseline(rows=256):
+def blas_info() -> dict:
+    """BLAS library numpy uses and its thread count."""
+    try:
+        import threadpoolctl
+        info = [i for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return {"vendor": f"{info[0].get('internal_api')} {info[0].get('version')}",
+                    "threads": info[0].get("num_threads")}
+    except Exception:  # noqa: BLE001 - reporting only
+        pass
+    return {"vendor": "unknown", "threads": None}
+
+
+def oracle_tiny_step():
+    """The oracle's whole hot path on the tiny fp32 workload: four warm-up
+    chunks of the dual stream, their statistics, the absorb and an L-layer."""
+    from oracle import ispa_oracle as orc
+    w = synth.WORKLOADS["tiny_f32"]
+    xs = [synth.single_layer_inputs(w, c) for c in range(w.warm_chunks)]
+    W = synth.weight(w, 0)
+
+    def run():
+        a, d = [], []
+        for x in xs:
+            r = orc.dual_stream(x["q"], [(x["k_sink"], x["v_sink"]), (x["k_cur"], x["v_cur"])],
+                                [(x["k_hist"], x["v_hist"])], w.n_heads)
+            a.append(r["a_loc"])
+            d.append(r["delta"])
+        G, R = orc.gram(np.concatenate(a), np.concatenate(d))
+        dW = orc.absorb(G, R, W, orc.ridge_lambda(G))
+        orc.project(a[-1], orc.modulated_weight(W, dW))
+    return run
+
+
+def cpu_baseline(rows=256, rows_1t=32):
+    from threadpoolctl import threadpool_limits
     run, flops = oracle_sample(rows)
     t0 = time.perf_counter()
     run()
     dt = time.perf_counter() - t0
+    run1, flops1 = oracle_sample(rows_1t)
+    tiny = oracle_tiny_step()
+    with threadpool_limits(limits=1, user_api="blas"):
+        t0 = time.perf_counter()
+        run1()
+        dt1 = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        tiny()
+        dt_tiny1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    tiny()
+    dt_tiny = time.perf_counter() - t0
+    blas = blas_info()
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+            "blas": blas["vendor"], "blas_threads": blas["threads"],
             "sample": f"fp64 numpy oracle, {rows} of 4680 query rows of the wan1.3b chunk (local, history and "
-                      f"single-pass full attention), {dt:.2f} s"}
+                      f"single-pass full attention), {dt:.2f} s",
+            "one_thread": {"wan1.3b_tflops": round(flops1 / dt1 / 1e12, 6),
+                           "wan1.3b_sample": f"{rows_1t} query rows, {dt1:.2f} s",
+                           "tiny_f32_step_ms": round(dt_tiny1 * 1e3, 2)},
+            "tiny_f32_step_ms": round(dt_tiny * 1e3, 2),
+            "tiny_f32_step": "4 warm-up chunks of the dual stream, statistics, absorb, one L-layer projection"}
 
 
 def run_reference(args):
@@ -740,6 +969,7 @@ def run_reference(args):
             "config": {"workload": "wan1.3b single layer dual-stream attention; each step a bounded sample of "
                                    f"{rows} query rows", "parallelism": "none (host cores)"},
             "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+                             "blas": blas_info()["vendor"], "blas_threads": blas_info()["threads"],
                              "sample": f"{rows} of 4680 query rows per step"},
             "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -120,7 +120,9 @@ ISPA_API ispa_status_t ispa_dual_attention(const void* q, int64_t n_q, int64_t q
  * stride D); lse_loc, lse_hist [n_heads, n_q] fp32 (lse_hist = -inf marks an
  * empty branch).  Writes a_full = exp(L_loc - L) o_loc + exp(L_hist - L) o_hist,
  * a_delta = a_full - o_loc (nullable) and lse_full = L (nullable), with
- * L = logaddexp(L_loc, L_hist).  Outputs may not alias inputs.
+ * L = logaddexp(L_loc, L_hist).  A (row, head) pair whose two LSEs are both
+ * -inf (both branches empty) gets both weights 0: a_full = 0 and L = -inf, as
+ * attention over the empty union of the key sets.  Outputs may not alias inputs.
  */
 ISPA_API ispa_status_t ispa_lse_merge(const void* o_loc, const float* lse_loc, const void* o_hist, const float* lse_hist,
                              int64_t n_q, int32_t n_heads, int32_t head_dim, ispa_dtype_t dt, void* a_full,
@@ -220,9 +222,10 @@ ISPA_API ispa_status_t ispa_absorb_solve(const float* G, const float* R, const v
  *     ISPA_ERR_UNSUPPORTED without launching.
  *   - No allocation of any kind happens, and nothing needs clearing: each call
  *     writes every working value before reading it.
- *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress); make that first call before any stream
- *     capture.
+ *   - The first call in a CUDA context (normally one per device; a new one
+ *     after cudaDeviceReset) looks up the array's device address in that
+ *     context (cudaGetSymbolAddress) and caches it under the context's unique
+ *     id; make that first call before any stream capture.
  *   - All calls on a device share the one array: calls whose executions overlap
  *     on the GPU (different streams without ordering between them) race and
  *     give undefined results.  Calls on one stream are safe.
@@ -321,7 +324,9 @@ ISPA_API ispa_status_t ispa_local_attention_project_w8a8(const void* q, int64_t 
  * the sink frame inside its own current chunk: no separate sink, no history.
  * Chunk c >= 1: sink = first sink_frames frames, history = the frames between
  * the sink and the current chunk, current = frames [c*chunk_frames,
- * (c+1)*chunk_frames).  Returns ISPA_ERR_INVALID_ARG on negative sizes.
+ * (c+1)*chunk_frames).  Returns ISPA_ERR_INVALID_ARG on negative sizes and,
+ * for chunk >= 1, when the sink does not end before the current chunk starts
+ * (sink_frames > chunk * chunk_frames): the ranges would overlap.
  */
 ISPA_API ispa_status_t ispa_chunk_token_ranges(int64_t chunk, int64_t frame_tokens, int64_t chunk_frames,
                                       int64_t sink_frames, int64_t* out);
@@ -329,7 +334,8 @@ ISPA_API ispa_status_t ispa_chunk_token_ranges(int64_t chunk, int64_t frame_toke
 /* KV bytes held by n_layers layers at chunk `chunk`: bit l of l_layer_mask marks
  * an L-layer; once `transitioned` is non-zero an L-layer keeps only the sink and
  * current tokens, an F-layer keeps every frame up to the current chunk.
- * Returns -1 on invalid arguments. */
+ * Returns -1 on invalid arguments (those ispa_chunk_token_ranges rejects
+ * included). */
 ISPA_API int64_t ispa_kv_bytes(int64_t chunk, int32_t n_layers, uint64_t l_layer_mask, int32_t transitioned,
                       int64_t frame_tokens, int64_t chunk_frames, int64_t d_model, int32_t elem_bytes,
                       int64_t sink_frames);

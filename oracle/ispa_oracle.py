@@ -129,15 +129,19 @@ def lse_merge(o_loc, lse_loc, o_hist, lse_hist, n_heads: int):
 
     With L = log(exp(L_loc) + exp(L_hist)) per (head, row), the full output is
     exp(L_loc - L) * O_loc + exp(L_hist - L) * O_hist.  An empty branch has
-    LSE = -inf and weight 0.  Returns (A_full, delta = A_full - O_loc, L).
+    LSE = -inf and weight 0; when both are empty (L = -inf) both weights are 0,
+    so A_full = 0 and L = -inf, which is attention over the empty union of the
+    two key sets.  Returns (A_full, delta = A_full - O_loc, L).
     """
     o_loc, o_hist = _f64(o_loc), _f64(o_hist)
     lse_loc, lse_hist = _f64(lse_loc), _f64(lse_hist)
     n_q, D = o_loc.shape
     d = D // n_heads
     L = np.logaddexp(lse_loc, lse_hist)                     # [H, n_q]
-    w_loc = np.exp(lse_loc - L)
-    w_hist = np.exp(lse_hist - L)
+    empty = np.isneginf(L)
+    Ls = np.where(empty, 0.0, L)
+    w_loc = np.where(empty, 0.0, np.exp(np.where(empty, 0.0, lse_loc - Ls)))
+    w_hist = np.where(empty, 0.0, np.exp(np.where(empty, 0.0, lse_hist - Ls)))
     w_loc_rows = np.repeat(w_loc.T, d, axis=1)              # [n_q, D], head-major columns
     w_hist_rows = np.repeat(w_hist.T, d, axis=1)
     a_full = w_loc_rows * o_loc + w_hist_rows * o_hist
@@ -219,8 +223,12 @@ def chunk_token_ranges(chunk: int, frame_tokens: int, chunk_frames: int,
     token 0.  Chunk 0 holds the sink frame inside its own current chunk, so it
     has no separate sink and no history; chunk c >= 1 sees sink = the first
     ``sink_frames`` frames, history = the frames between the sink and the
-    current chunk, current = frames [c*chunk_frames, (c+1)*chunk_frames)."""
+    current chunk, current = frames [c*chunk_frames, (c+1)*chunk_frames).  The
+    sink precedes the current chunk, so chunk c >= 1 needs
+    sink_frames <= c*chunk_frames (ValueError otherwise)."""
     F, cf = frame_tokens, chunk_frames
+    if chunk > 0 and sink_frames > chunk * cf:
+        raise ValueError("the sink must end before the current chunk starts")
     cur = (chunk * cf * F, (chunk + 1) * cf * F)
     if chunk == 0:
         return {"sink": (0, 0), "hist": (0, 0), "cur": cur}

@@ -1,5 +1,13 @@
 """Shared helpers of the GPU parity tests: moving seeded numpy inputs to the
-device and the error measures the tolerances are stated in."""
+device and the error measures the tolerances are stated in.
+
+Every call of ``max_rel`` is also recorded, together with the elementwise
+relative error whose denominator is floored at 1e-3 of the reference's largest
+magnitude, and ``tests/conftest.py`` prints the worst of both per test at the
+end of the run (the floored elementwise figure is reported, not bounded: for
+bf16 outputs it reaches O(1) on elements near the floor)."""
+import os
+
 import numpy as np
 import torch
 
@@ -16,6 +24,19 @@ GRAM_REL = 1e-4
 # y = A W: bf16 operands, fp32 accumulation over D terms, bf16 output rounding
 PROJ_MAX_REL = 1e-2
 
+# Chained tolerances: expected values come from the oracle's own chain on the
+# seeded inputs while the GPU chain consumes its own bf16 attention outputs.
+# Each bound is produced by tests/chain_tolerances.py (oracle-only simulation
+# of the GPU's bf16 rounding plus a 2^-9 relative attention error) and checked
+# against it by tests/test_chain_tolerances.py.
+CHAIN_DW_REL = 2e-2      # dW of the small rollout (simulated 4-5e-3)
+CHAIN_EPS_REL = 1e-3     # a layer's reconstruction error (simulated ~1e-4)
+CHAIN_W8A8_FRO = 4e-2    # W8A8 L-layer y, relative Frobenius (simulated 1.4-1.6e-2)
+CHAIN_W8A8_MAX = 5e-2    # W8A8 L-layer y, largest element error / max|y| (simulated 1.6-1.9e-2)
+
+ELEM_FLOOR = 1e-3        # floor of the elementwise relative error, times max|ref|
+REPORT = []              # (test id, max_rel, elementwise relative error with floor)
+
 
 def dev(x: np.ndarray, dtype: str) -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
@@ -27,9 +48,21 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def max_rel(x, ref) -> float:
+def elem_rel(x, ref, floor: float = ELEM_FLOOR) -> float:
+    """max_i |x_i - ref_i| / max(|ref_i|, floor * max|ref|)."""
     ref = np.asarray(ref, np.float64)
-    return float(np.max(np.abs(np.asarray(x, np.float64) - ref)) / max(np.max(np.abs(ref)), 1e-30))
+    den = np.maximum(np.abs(ref), floor * max(float(np.max(np.abs(ref))) if ref.size else 0.0, 1e-30))
+    return float(np.max(np.abs(np.asarray(x, np.float64) - ref) / den)) if ref.size else 0.0
+
+
+def max_rel(x, ref) -> float:
+    """max|x - ref| / max|ref| per tensor (the measure the bounds are stated in);
+    recorded with the floored elementwise error for the end-of-run report."""
+    ref = np.asarray(ref, np.float64)
+    v = float(np.max(np.abs(np.asarray(x, np.float64) - ref)) / max(np.max(np.abs(ref)), 1e-30))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    REPORT.append((test, v, elem_rel(x, ref)))
+    return v
 
 
 def max_abs(x, ref) -> float:

@@ -84,6 +84,21 @@ def test_chunk_token_ranges_bit_exact(L, chunk):
         assert got == orc.chunk_token_ranges(chunk, F, cf, sf)
 
 
+def test_chunk_token_ranges_rejects_a_sink_that_overlaps_the_current_chunk(L):
+    # chunk 1 of 3-frame chunks starts at frame 3: a 4-frame sink would overlap it
+    for args in [(1, 1560, 3, 4), (2, 16, 1, 3), (1, 7, 2, 3)]:
+        with pytest.raises(ispa.IspaError) as e:
+            ispa.ispa_chunk_token_ranges(*args)
+        assert e.value.code == 1
+        with pytest.raises(ValueError):
+            orc.chunk_token_ranges(*args)
+        with pytest.raises(ispa.IspaError):
+            ispa.ispa_kv_bytes(args[0], 4, 0b0101, True, args[1], args[2], 128, 2, args[3])
+    # the boundary case (the sink fills every frame before the chunk) and chunk 0 are valid
+    assert ispa.ispa_chunk_token_ranges(1, 16, 3, 3) == orc.chunk_token_ranges(1, 16, 3, 3)
+    assert ispa.ispa_chunk_token_ranges(0, 16, 3, 9) == orc.chunk_token_ranges(0, 16, 3, 9)
+
+
 def test_kv_bytes_bit_exact(L):
     mask = orc.layer_mask(30, range(0, 30, 2))
     for chunk in range(24):

@@ -173,6 +173,41 @@ def test_lse_merge_matches_oracle():
     assert np.array_equal(host(out["a_full"])[:50, d:2 * d], o_loc[:50, d:2 * d])
 
 
+def test_lse_merge_rows_with_both_branches_empty():
+    """(row, head) pairs whose local and historical branches are both empty
+    (both LSEs -inf; the outputs of those branches are 0, as attention over no
+    keys gives): A_full = 0 and LSE = -inf, as for attention over the empty
+    union, and no NaN anywhere; every other pair as the oracle."""
+    g = np.random.default_rng(6)
+    H, d, n = 2, 64, 131
+    o_loc = synth.round_bf16(g.standard_normal((n, H * d)).astype(np.float32))
+    o_hist = synth.round_bf16(g.standard_normal((n, H * d)).astype(np.float32))
+    l_loc = (g.standard_normal((H, n)) * 3).astype(np.float32)
+    l_hist = (g.standard_normal((H, n)) * 3).astype(np.float32)
+    empty = np.zeros((H, n), bool)
+    empty[0, 10:40] = True
+    empty[1, 100:] = True
+    for h in range(H):
+        r = np.nonzero(empty[h])[0]
+        l_loc[h, r] = l_hist[h, r] = -np.inf
+        o_loc[np.ix_(r, range(h * d, (h + 1) * d))] = 0.0
+        o_hist[np.ix_(r, range(h * d, (h + 1) * d))] = 0.0
+    out = ispa.lse_merge(dev(o_loc, "bf16"), torch.from_numpy(l_loc).cuda(), dev(o_hist, "bf16"),
+                         torch.from_numpy(l_hist).cuda(), H)
+    torch.cuda.synchronize()
+    got = {k: host(v) for k, v in out.items()}
+    a_full, delta, L = orc.lse_merge(o_loc, l_loc, o_hist, l_hist, H)
+    for v in got.values():
+        assert not np.any(np.isnan(v))
+    assert np.array_equal(np.isneginf(got["lse_full"]), empty) and np.array_equal(np.isneginf(L), empty)
+    assert max_abs(got["lse_full"][~empty], L[~empty]) <= LSE_ABS
+    assert max_rel(got["a_full"], a_full) <= ATTN_MAX_REL
+    assert max_rel(got["a_delta"], delta) <= ATTN_MAX_REL
+    for h in range(H):
+        r = np.nonzero(empty[h])[0]
+        assert np.all(got["a_full"][np.ix_(r, range(h * d, (h + 1) * d))] == 0.0)
+
+
 @pytest.mark.parametrize("n_rows,D", [(4680, 1536), (300, 256), (1, 128), (129, 384)])
 def test_gram_bf16_matches_oracle(n_rows, D):
     g = np.random.default_rng(n_rows + D)

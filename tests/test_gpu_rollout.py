@@ -12,12 +12,19 @@ Absorption", gist.science technical summary, section 2, stages 1-3).
 * The 1.3B-shaped rollout (4 layers) is checked where the oracle can follow
   it: the KV bookkeeping bit for bit, the eviction, and sampled rows of
   F-layer outputs, whose weight is the seeded W.
+* Two layers of the 1.3B-shaped rollout at full size, with the absorbed layer
+  chosen by instance selection: the oracle runs its own chain over all 18720
+  warm-up rows of each layer (A_loc and A_full by direct attention, G, R,
+  lambda, dW, eps), and the GPU's dW of both layers, their eps, the choice and
+  sampled rows of the chosen layer's post-transition L-layer output (local
+  attention times the oracle's W_new) are compared with it.
 
-Chained tolerance of dW: the GPU statistics consume bf16 A_loc and delta, and
-the attention outputs differ from the oracle's at the 2^-9 level.  Simulated
-in the oracle (bf16 rounding plus 2^-9 relative noise on A_loc and A_full over
-the small rollout's 1440 warm-up rows), that moves dW by 4.5e-3 relative; the
-bound is 2e-2."""
+Chained tolerance of dW (CHAIN_DW_REL in tests/helpers.py): the GPU statistics
+consume bf16 A_loc and delta, and the attention outputs differ from the
+oracle's at the 2^-9 level.  tests/chain_tolerances.py simulates that in the
+oracle (bf16 rounding plus 2^-9 relative noise on A_loc and A_full over the
+small rollout's 1440 warm-up rows): dW moves by 4-5e-3 relative; the bound is
+2e-2.  The measured chain errors are printed in the run's parity report."""
 import dataclasses
 
 import numpy as np
@@ -28,12 +35,10 @@ from ar_video_diffusion_b200 import build as ispa_build
 from ar_video_diffusion_b200 import ispa, synth
 from ar_video_diffusion_b200.rollout import Rollout
 from oracle import ispa_oracle as orc
-from helpers import (ATTN_MAX_REL, capture_inputs, cat_segments, fro_rel, host, max_rel,
-                     oracle_rollout_statistics)
+from helpers import (ATTN_MAX_REL, CHAIN_DW_REL, CHAIN_EPS_REL, REPORT, capture_inputs, cat_segments, fro_rel,
+                     host, max_rel, oracle_rollout_statistics)
 
 pytestmark = pytest.mark.gpu
-
-CHAIN_DW_REL = 2e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -70,7 +75,9 @@ def test_small_rollout_against_the_oracle_chain():
         a_loc, a_full = oracle_rollout_statistics(w, inputs, l)
         G, R = orc.gram(a_loc, a_full - a_loc)
         dW_ref = orc.absorb(G, R, W[l], orc.ridge_lambda(G))
-        assert fro_rel(host(ro.dW[l]), dW_ref) <= CHAIN_DW_REL, l
+        err = fro_rel(host(ro.dW[l]), dW_ref)
+        REPORT.append((f"small rollout chain: dW of layer {l} (relative Frobenius)", err, err))
+        assert err <= CHAIN_DW_REL, (l, err)
         W_new_ref[l] = synth.round_bf16(orc.modulated_weight(W[l], dW_ref).astype(np.float32))
 
     n_chunks = w.warm_chunks + w.post_chunks
@@ -118,3 +125,69 @@ def test_full_size_rollout_bookkeeping_and_f_layers():
         a, _ = orc.attention(ck["q"], np.concatenate([ck["k_loc"], ck["k_hist"]]),
                              np.concatenate([ck["v_loc"], ck["v_hist"]]), w.n_heads)
         assert max_rel(ck["y"], orc.project(a, ck["W"])) <= ATTN_MAX_REL, (ck["l"], ck["c"])
+
+
+def _f32_segments(segs, i, D):
+    """Host fp32 copy of the concatenated segments (bf16 values are exact in fp32)."""
+    if not segs:
+        return np.zeros((0, D), np.float32)
+    return np.concatenate([s[i].float().cpu().numpy() for s in segs])
+
+
+def test_full_size_rollout_absorbed_layers_against_the_oracle_chain():
+    """Layers 0 and 1 of the 1.3B-shaped rollout (12 heads x 128, 4680 chunk
+    queries, 4 warm-up chunks = 18720 statistics rows, then one chunk), K = 1
+    layer chosen by reconstruction error."""
+    w = dataclasses.replace(synth.WORKLOADS["rollout"], n_layers=2, post_chunks=1)
+    D, H = w.d_model, w.n_heads
+    rows = np.sort(np.random.default_rng(12).choice(w.n_q, 64, replace=False))
+    rows[-1] = w.n_q - 1
+    warm, post = {}, {}
+
+    def on_layer(l, c, info):
+        torch.cuda.synchronize()
+        rec = {"q": info["q"].float().cpu().numpy(), "mode": info["mode"],
+               "k_loc": _f32_segments(info["local"], 0, D), "v_loc": _f32_segments(info["local"], 1, D),
+               "k_hist": _f32_segments(info["hist"], 0, D), "v_hist": _f32_segments(info["hist"], 1, D)}
+        if c < w.warm_chunks:
+            warm[(l, c)] = rec
+        else:
+            rec["y"] = host(info["y"])[rows]
+            rec["q"] = rec["q"][rows]
+            post[l] = rec
+
+    ro = Rollout(w, absorbed=[0], selection="instance", on_layer=on_layer)
+    ro.run()
+    eps_o, dW_o = [], {}
+    for l in range(w.n_layers):
+        a_loc, a_full = [], []
+        for c in range(w.warm_chunks):
+            x = warm[(l, c)]
+            a_loc.append(orc.attention(x["q"], x["k_loc"], x["v_loc"], H)[0])
+            a_full.append(orc.attention(x["q"], np.concatenate([x["k_loc"], x["k_hist"]]),
+                                        np.concatenate([x["v_loc"], x["v_hist"]]), H)[0])
+        a_loc, a_full = np.concatenate(a_loc), np.concatenate(a_full)
+        assert a_loc.shape == (w.warm_chunks * w.n_q, D)
+        W = host(ro.W[l])
+        G, R = orc.gram(a_loc, a_full - a_loc)
+        dW_o[l] = orc.absorb(G, R, W, orc.ridge_lambda(G))
+        eps_o.append(orc.reconstruction_error(a_loc, a_full, W, dW_o[l]))
+        err = fro_rel(host(ro.dW_ranked[l]), dW_o[l])
+        REPORT.append((f"1.3B rollout chain: dW of layer {l} (relative Frobenius)", err, err))
+        assert err <= CHAIN_DW_REL, (l, err)
+        e_err = abs(ro.eps[l] - eps_o[l]) / eps_o[l]
+        REPORT.append((f"1.3B rollout chain: eps of layer {l} (relative)", e_err, e_err))
+        assert e_err <= CHAIN_EPS_REL, (l, ro.eps[l], eps_o[l])
+    # the choice is the oracle's unless the two errors lie within the tolerance of each other
+    if abs(eps_o[0] - eps_o[1]) > 2 * CHAIN_EPS_REL * max(eps_o):
+        assert ro.absorbed == orc.select_layers(eps_o, 1)
+    (chosen,) = ro.absorbed
+    assert ro.k[chosen].shape[0] == w.frame_tokens + w.n_q  # history evicted
+    x = post[chosen]
+    assert x["mode"] == "L" and x["k_hist"].shape[0] == 0
+    assert x["k_loc"].shape[0] == w.frame_tokens + w.n_q
+    W_new_ref = synth.round_bf16(orc.modulated_weight(host(ro.W[chosen]), dW_o[chosen]).astype(np.float32))
+    a, _ = orc.attention(x["q"], x["k_loc"], x["v_loc"], H)
+    assert max_rel(x["y"], orc.project(a, W_new_ref)) <= ATTN_MAX_REL
+    other = post[1 - chosen]
+    assert other["mode"] == "F" and other["k_hist"].shape[0] == (w.warm_chunks * w.chunk_frames - 1) * w.frame_tokens

@@ -11,6 +11,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -205,7 +206,7 @@ for l in layers:
     stats[l] = s
     W[l] = torch.from_numpy(rng.standard_normal((D, D)) / 4)
 w_new = sharded.absorb_layers(stats, W, world, rank)
-mine = [l for l in layers if sharded.absorb_owner(l, world) == rank]
+mine = [l for l, r in sharded.absorb_owners(layers, world).items() if r == rank]
 out = {"rank": rank, "n_solved": len(solved), "mine": mine,
        "w_new": {str(l): float(w_new[l].sum()) for l in layers}}
 dist.barrier()
@@ -225,4 +226,21 @@ def test_absorb_layers_owned_once_and_broadcast_two_gloo_ranks():
     assert owned == [0, 2, 4, 6, 8]
     for r in res:
         assert r["n_solved"] == len(r["mine"])
+    # both ranks solve: the even layers are split 3 / 2, not all to rank 0
+    assert sorted(len(r["mine"]) for r in res) == [2, 3]
     assert res[0]["w_new"] == res[1]["w_new"]
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_absorb_owners_balanced_for_any_layer_set(world):
+    from ar_video_diffusion_b200 import sharded
+    rng = np.random.default_rng(world)
+    sets = [list(range(0, 30, 2)), list(range(1, 30, 2)), list(range(30)),
+            sorted(rng.choice(30, 15, replace=False).tolist()), [4], []]
+    for layers in sets:
+        owners = sharded.absorb_owners(layers, world)
+        assert sorted(owners) == sorted(layers)
+        counts = [sum(1 for r in owners.values() if r == k) for k in range(world)]
+        assert sum(counts) == len(layers)
+        assert max(counts) - min(counts) <= 1, (layers, counts)
+        assert all(0 <= r < world for r in owners.values())

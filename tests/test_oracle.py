@@ -114,6 +114,32 @@ def test_merge_with_empty_history_is_identity():
     assert np.max(np.abs(r["a_full"] - r["a_loc"])) == 0
 
 
+def test_merge_of_two_empty_branches_is_attention_over_no_keys():
+    """A row whose local and historical branches are both empty: the merge
+    must give what attention over the (empty) union gives -- o = 0 and
+    LSE = -inf -- with no NaN; rows with a non-empty branch are unaffected."""
+    H, d, n = 2, 8, 5
+    c = synth.random_case(23, n_q=n, n_heads=H, head_dim=d, seg_tokens=[9, 14], dtype="f32")
+    (kl, vl), (kh, vh) = c["segments"]
+    o_l, l_l = orc.attention(c["q"], kl, vl, H)
+    o_h, l_h = orc.attention(c["q"], kh, vh, H)
+    o_e, l_e = orc.attention(c["q"], np.zeros((0, H * d)), np.zeros((0, H * d)), H)
+    # rows 1 and 3 lose both branches for head 0; row 4 keeps only its history for head 1
+    for r in (1, 3):
+        o_l[r, :d], l_l[0, r] = o_e[r, :d], l_e[0, r]
+        o_h[r, :d], l_h[0, r] = o_e[r, :d], l_e[0, r]
+    o_l[4, d:], l_l[1, 4] = 0.0, -np.inf
+    a_full, delta, L = orc.lse_merge(o_l, l_l, o_h, l_h, H)
+    assert not np.any(np.isnan(a_full)) and not np.any(np.isnan(delta)) and not np.any(np.isnan(L))
+    for r in (1, 3):
+        assert np.all(a_full[r, :d] == o_e[r, :d]) and np.isneginf(L[0, r]) and np.isneginf(l_e[0, r])
+    assert np.array_equal(a_full[4, d:], o_h[4, d:]) and L[1, 4] == l_h[1, 4]
+    ref, _, Lref = orc.lse_merge(orc.attention(c["q"], kl, vl, H)[0], orc.attention(c["q"], kl, vl, H)[1],
+                                 orc.attention(c["q"], kh, vh, H)[0], orc.attention(c["q"], kh, vh, H)[1], H)
+    keep = [0, 2]
+    assert np.array_equal(a_full[keep], ref[keep]) and np.array_equal(L[:, keep], Lref[:, keep])
+
+
 # ---------------------------------------------------------------------- absorb
 def _ridge_case(seed, N, D, Dout=None):
     Dout = D if Dout is None else Dout
@@ -227,6 +253,27 @@ def test_absorb_ols_at_lambda_zero():
     dW = orc.absorb(G, R, W, 0.0)
     ref = np.linalg.lstsq(a_loc, (a_full - a_loc) @ W, rcond=None)[0]
     assert np.linalg.norm(dW - ref) <= 1e-10 * np.linalg.norm(ref)
+
+
+def test_ridge_lambda_hand_values():
+    """lambda = 1e-2 * trace(G) / D, the value every benchmark configuration
+    states ("lambda = 1e-2 * trace(G) / D"; the pages give none), on values
+    worked out by hand.  A wrong divisor (the row count N instead of D), a
+    wrong constant or a missing lambda_abs term fails one of them."""
+    # G = diag(1, 2, 3, 4): trace 10, D = 4 -> 1e-2 * 10 / 4
+    assert orc.ridge_lambda(np.diag([1.0, 2.0, 3.0, 4.0])) == pytest.approx(0.025, rel=1e-15)
+    # G = A^T A with A 7 x 4 (N = 7 rows != D = 4): trace(G) = sum of A's
+    # squares = 1 + 4 + 9 + 4 + 0 + 16 + 1 = 35 -> 1e-2 * 35 / 4 = 0.0875 (N in
+    # the divisor would give 0.05)
+    A = np.array([[1.0, 0, 0, 0], [0, 2, 0, 0], [0, 0, 0, 3], [1, 1, 1, 1], [0, 0, 0, 0], [0, 0, 4, 0],
+                  [0, 0, 0, 1]])
+    assert np.sum(A * A) == 35
+    assert orc.ridge_lambda(A.T @ A) == pytest.approx(0.0875, rel=1e-15)
+    # off-diagonal entries do not enter; lambda_abs adds, lambda_rel scales
+    G = np.array([[2.0, -7.0], [-7.0, 6.0]])  # trace 8, D = 2
+    assert orc.ridge_lambda(G) == pytest.approx(0.04, rel=1e-15)
+    assert orc.ridge_lambda(G, lambda_rel=0.5, lambda_abs=0.25) == pytest.approx(0.25 + 0.5 * 8 / 2, rel=1e-15)
+    assert orc.LAMBDA_REL == 1e-2
 
 
 def test_lambda_reading_is_normalisation_invariant():
