@@ -4,19 +4,22 @@
 // Instance-Specific Parametric Absorption", gist.science technical summary,
 // section 2 stage 2 "Layer Absorb"), then W_new = W + dW (stage 3).
 //
-// fp32 throughout, all on the device, stream ordered:
-//   1. S = R W, written straight into dW (which the solves then update in
-//      place): on the tensor cores as hi(R) W + lo(R) W when W is bf16;
+// All on the device, stream ordered, in two forms.
+// Tensor-core form (bf16 W, D a multiple of 128, D >= 256):
+//   1. S = R W on the tensor cores as hi(R) W + lo(R) W (W is exactly bf16);
 //   2. trace(G) -> lambda (one block, fp64 sum);  M = G + lambda I;
-//   3. right-looking blocked Cholesky M = L L^T with 64 x 64 panels: the
-//      diagonal block is factored in shared memory by one CTA (which also
-//      forms its inverse), the panel below is multiplied by that inverse, and
-//      the trailing lower triangle gets a rank-64 update;
-//   4. L Y = S, then L^T X = Y, block by block with the stored diagonal
-//      inverses and rank-64 updates of the remaining rows;
+//   3. right-looking blocked Cholesky M = L L^T with 64-wide panels, the
+//      right-hand sides [S | I] carried along: per panel the diagonal block
+//      is factored (and its factor inverted) by one CTA, the panel below and
+//      the panel's rows of the right-hand sides are multiplied by that
+//      inverse, and one split-precision tensor-core product updates the
+//      trailing lower triangle and the remaining right-hand-side rows;
+//   4. dW = (L^-1)^T (L^-1 S), one split-precision tensor-core product;
 //   5. W_new = W + dW, rounded to W's dtype.
-// The fp32 GEMM used by steps 2-4 (and by the fp32 activation path of the
-// statistics and the projection) is a 64 x 64-tile CUDA-core kernel with
+// Compact form (every other case, and the no-allocation entry point): the
+// same factorisation with fp32 CUDA-core updates and blocked triangular
+// solves L Y = S, L^T X = Y.  Its fp32 GEMM (also the fp32 activation path of
+// the statistics and the projection) is a 64 x 64-tile CUDA-core kernel with
 // arbitrary strides, so transposed operands are read in place.
 #include <cstring>
 
@@ -379,15 +382,337 @@ __global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ 
 
 }  // namespace simt
 
-size_t absorb_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
+// ------------------------------------------- tensor-core form of the solve
+// For bf16 W and D a multiple of 128 (D >= 256) the solve runs its products on
+// the tensor cores in split precision (hi/lo bf16 pairs, about 2^-17 relative
+// per product), with the right-hand sides carried through the factorisation:
+//   RHS = [S | I] (D x 2D) with S = R W;
+//   for each 64-wide panel k (right-looking):
+//     factor the diagonal block and invert its factor (one CTA);
+//     L21 = A21 L_kk^-T for the rows below, and Y_k = L_kk^-1 RHS_k for the
+//     panel's rows of the right-hand sides (final rows of L^-1 S and L^-1);
+//     one tensor-core update [M22 | RHS_2] -= L21 [L21^T | Y_k];
+//   after the last panel RHS = [L^-1 S | L^-1], and
+//   dW = (L^-1)^T (L^-1 S) = (G + lambda I)^-1 S is one tensor-core product
+//   whose A operand (L^-1)^T is upper triangular.
+namespace simt {
+
+// 32 x 32 Cholesky factor of a lower triangle in shared memory (row stride
+// ld), by one warp: lane r holds row r in registers with the columns rotated
+// (a[0] is the current column), so the loop body is short and its register
+// indices static; the loop itself stays rolled, keeping the code small enough
+// for the instruction cache (an unrolled factorisation run once by one warp is
+// bound by instruction fetch).  L is written over the lower triangle.  A pivot
+// <= 0 or non-finite is replaced by 1 and its index (first only) recorded.
+__device__ __forceinline__ void chol32_rot(float* A, int ld, int lane, int base, int* bad) {
+  float a[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) a[c] = c <= lane ? A[lane * ld + c] : 0.f;
+#pragma unroll 1
+  for (int j = 0; j < 32; ++j) {
+    float d = __shfl_sync(0xffffffffu, a[0], j);
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (lane == 0 && *bad < 0) *bad = base + j;
+      d = 1.f;
+    }
+    const float ljj = sqrtf(d);
+    const float l = lane == j ? ljj : (lane > j ? a[0] / ljj : 0.f);
+    if (lane >= j) A[lane * ld + j] = l;
+    // a[c] holds column j + c: subtract l * L[j + c][j] (lane j + c's l)
+#pragma unroll
+    for (int c = 1; c < 32; ++c) {
+      const float lk = __shfl_sync(0xffffffffu, l, (j + c) & 31);
+      a[c - 1] = a[c] - l * lk;
+    }
+    a[31] = 0.f;
+  }
+}
+
+// Column `lane` of X = L^-1 for the 32 x 32 lower-triangular L in shared memory
+// (row stride ld), by one warp, column-oriented forward elimination with the
+// right-hand side rotated in registers; X[m][lane] written with row stride ldx.
+__device__ __forceinline__ void inv32_rot(const float* L, int ld, float* X, int ldx, int lane) {
+  float b[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
+#pragma unroll 1
+  for (int m = 0; m < 32; ++m) {
+    const float x = b[0] / L[m * ld + m];
+    X[m * ldx + lane] = x;
+#pragma unroll
+    for (int c = 1; c < 32; ++c) {
+      const float lr = m + c < 32 ? L[(m + c) * ld + m] : 0.f;
+      b[c - 1] = b[c] - lr * x;
+    }
+    b[31] = 0.f;
+  }
+}
+
+// Cholesky factor of the 64 x 64 block in A (shared, row stride 65; lower
+// triangle used) and the inverse X of that factor (shared, row stride 65),
+// by the 256 threads of a CTA: L11 = chol(A11) and X11 by warp 0,
+// L21 = A21 X11^T, A22 - L21 L21^T, L22 = chol(.) and X22 by warp 0,
+// X21 = -X22 (L21 X11).  T: 32 x 33 scratch.
+__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], int* bad, int base) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // element (i, j) of a 32 x 32 product: i = tid / 8, j = tid % 8 + 8 b
+  const int pi = tid >> 3, pj = tid & 7;
+  for (int e = tid; e < 64 * 65; e += 256) (&X[0][0])[e] = 0.f;
+  if (warp == 0) {
+    chol32_rot(&A[0][0], 65, lane, base, bad);
+    __syncwarp();
+    inv32_rot(&A[0][0], 65, &X[0][0], 65, lane);
+  }
+  __syncthreads();
+  float acc[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {  // L21 = A21 X11^T
+    const int j = pj + 8 * b;
+    float v = 0.f;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * X[j][m];
+    acc[b] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int b = 0; b < 4; ++b) A[32 + pi][pj + 8 * b] = acc[b];
+  __syncthreads();
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {  // A22 -= L21 L21^T
+    const int j = pj + 8 * b;
+    float v = 0.f;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * A[32 + j][m];
+    A[32 + pi][32 + j] -= v;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    chol32_rot(&A[32][32], 65, lane, base + 32, bad);
+    __syncwarp();
+    inv32_rot(&A[32][32], 65, &X[32][32], 65, lane);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {  // T = L21 X11
+    const int j = pj + 8 * b;
+    float v = 0.f;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * X[m][j];
+    T[pi][j] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {  // X21 = -X22 T
+    const int j = pj + 8 * b;
+    float v = 0.f;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) v += X[32 + pi][32 + m] * T[m][j];
+    X[32 + pi][j] = -v;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void split_store(float v, __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t i) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[i] = h;
+  lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// Panel k, with the factorisation of its diagonal block.  Every CTA factors
+// the 64 x 64 diagonal block of M itself (it is small, and the copies run in
+// parallel, so no separate launch or global round trip sits on the chain;
+// CTA 0 records a bad pivot).  Then:
+//   blocks [0, rest): one 64-row block r below the diagonal,
+//     L_rk = A_rk L_kk^-T, written back to M, plus its split operands: -hi/-lo
+//     as K-major [rows, 64] (a_hi, a_lo, local row index) and hi/lo
+//     transposed as [64, ld_t] (lt_hi, lt_lo);
+//   blocks [rest, rest + ncb): one 64-column block of the panel's
+//     right-hand-side rows, Y = L_kk^-1 RHS_k, written back to RHS, plus hi/lo
+//     [64, ld_y] (y_hi, y_lo).
+// Each CTA loads its own block into registers before the factorisation, so
+// the load overlaps it.
+__global__ void __launch_bounds__(256) panel_factor_kernel(float* M, int D, int k, int rest, float* RHS,
+                                                           int64_t rhs_ld, int rhs_cols, __nv_bfloat16* a_hi,
+                                                           __nv_bfloat16* a_lo, __nv_bfloat16* lt_hi,
+                                                           __nv_bfloat16* lt_lo, int64_t ld_t, __nv_bfloat16* y_hi,
+                                                           __nv_bfloat16* y_lo, int64_t ld_y, int32_t* status) {
+  __shared__ float A[kT][kT + 1];  // the diagonal block, then this CTA's block
+  __shared__ float X[kT][kT + 1];  // L_kk^-1
+  __shared__ float T[32][33];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  const bool row_block = (int)blockIdx.x < rest;
+  const int c0 = row_block ? 0 : ((int)blockIdx.x - rest) * kT;
+  const float* own = row_block ? M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)k * kT
+                               : RHS + (int64_t)k * kT * rhs_ld + c0;
+  const int64_t own_ld = row_block ? D : rhs_ld;
+  float pre[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q, i = e >> 6, j = e & 63;
+    pre[q] = (row_block || c0 + j < rhs_cols) ? own[(int64_t)i * own_ld + j] : 0.f;
+  }
+  const float* dblk = M + (int64_t)k * kT * D + (int64_t)k * kT;
+  for (int e = tid; e < kT * kT; e += 256) A[e >> 6][e & 63] = dblk[(int64_t)(e >> 6) * D + (e & 63)];
+  if (tid == 0) bad = -1;
+  __syncthreads();
+  factor_diag64(A, X, T, &bad, k * kT);
+  if (blockIdx.x == 0 && tid == 0 && bad >= 0 && status) {
+    if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    A[e >> 6][e & 63] = pre[q];
+  }
+  __syncthreads();
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+  if (row_block) {
+    mm64(A, X, false, true, acc);  // A_rk L_kk^-T
+    float* blk = M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)k * kT;
+    const int64_t row0 = (int64_t)blockIdx.x * kT;  // local row of the trailing block
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int i = ty + 16 * a, j = tx + 16 * b;
+        const float v = acc[a][b];
+        blk[(int64_t)i * D + j] = v;
+        split_store(-v, a_hi, a_lo, (row0 + i) * 64 + j);
+        split_store(v, lt_hi, lt_lo, (int64_t)j * ld_t + row0 + i);
+      }
+  } else {
+    mm64(X, A, false, false, acc);  // L_kk^-1 RHS_k
+    float* blk = RHS + (int64_t)k * kT * rhs_ld + c0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int i = ty + 16 * a, j = tx + 16 * b;
+        if (c0 + j >= rhs_cols) continue;
+        blk[(int64_t)i * rhs_ld + j] = acc[a][b];
+        split_store(acc[a][b], y_hi, y_lo, (int64_t)i * ld_y + c0 + j);
+      }
+  }
+}
+
+// RHS = [0 | I] (D x 2D fp32, 16-byte vectors)
+__global__ void init_rhs_kernel(float* __restrict__ RHS, int D) {
+  const int64_t n4 = (int64_t)D * 2 * D / 4;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = (e * 4) / (2 * D), j0 = (e * 4) % (2 * D) - D;  // column within the identity part
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t off = i - j0;
+    v.x = off == 0 ? 1.f : 0.f;
+    v.y = off == 1 ? 1.f : 0.f;
+    v.z = off == 2 ? 1.f : 0.f;
+    v.w = off == 3 ? 1.f : 0.f;
+    reinterpret_cast<float4*>(RHS)[e] = v;
+  }
+}
+
+// [Y | X] (D x 2D fp32) -> hi/lo of Y and of X, each D x D bf16
+__global__ void split_rhs_kernel(const float* __restrict__ RHS, int D, __nv_bfloat16* __restrict__ yh,
+                                 __nv_bfloat16* __restrict__ yl, __nv_bfloat16* __restrict__ xh,
+                                 __nv_bfloat16* __restrict__ xl) {
+  const int64_t n = (int64_t)D * 2 * D;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / (2 * D), j = e % (2 * D);
+    if (j < D)
+      split_store(RHS[e], yh, yl, i * D + j);
+    else
+      split_store(RHS[e], xh, xl, i * D + j - D);
+  }
+}
+
+}  // namespace simt
+
+// workspace of the tensor-core form: M (4 D^2) | RHS (8 D^2) | split area (4 D^2) |
+// Linv (256 D) | A hi/lo (256 D) | L21^T hi/lo (256 D) | Y_k hi/lo (512 D) | lambda
+static bool tc_eligible(ispa_dtype_t w_dt, int64_t D) { return w_dt == ISPA_DT_BF16 && D % 128 == 0 && D >= 256; }
+static size_t tc_workspace_bytes(int64_t D) { return (size_t)(16 * D * D + 1280 * D + 256); }
+static size_t compact_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
+
+size_t absorb_workspace_bytes(int64_t D) { return D % 128 == 0 && D >= 256 ? tc_workspace_bytes(D) : compact_workspace_bytes(D); }
+size_t absorb_compact_workspace_bytes(int64_t D) { return compact_workspace_bytes(D); }
+
+ispa_status_t absorb_step_update(int64_t rows, const void* a_hi, const void* a_lo, const void* lt_hi,
+                                 const void* lt_lo, int64_t lt_ld, const void* y_hi, const void* y_lo, int64_t y_ld,
+                                 int64_t rhs_cols, float* m_sub, int64_t m_ld, float* rhs_sub, int64_t rhs_ld,
+                                 cudaStream_t stream);
+ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const void* x_lo, int64_t x_ld,
+                               const void* y_hi, const void* y_lo, int64_t y_ld, float* c, int64_t ldc,
+                               cudaStream_t stream);
+ispa_status_t gemm_hilo_w(int64_t M, int64_t K, const void* a_hi, const void* a_lo, const void* w, int64_t N,
+                          float* c, int64_t ldc, cudaStream_t stream);
+
+static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_bfloat16* W, int64_t D64,
+                                    double lam_abs, double lam_rel, float* dW, __nv_bfloat16* w_new, void* workspace,
+                                    int32_t* status, cudaStream_t st) {
+  using namespace simt;
+  const int D = (int)D64;
+  const int nb = D / kT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* M = reinterpret_cast<float*>(ws);
+  float* RHS = reinterpret_cast<float*>(ws + 4 * D64 * D64);
+  uint8_t* split = ws + 12 * D64 * D64;
+  __nv_bfloat16* a_hi = reinterpret_cast<__nv_bfloat16*>(ws + 16 * D64 * D64 + 256 * D64);
+  __nv_bfloat16* a_lo = a_hi + 64 * D64;
+  __nv_bfloat16* lt_hi = a_lo + 64 * D64;
+  __nv_bfloat16* lt_lo = lt_hi + 64 * D64;
+  __nv_bfloat16* y_hi = lt_lo + 64 * D64;
+  __nv_bfloat16* y_lo = y_hi + 128 * D64;
+  double* lam = reinterpret_cast<double*>(ws + 16 * D64 * D64 + 1280 * D64);
+  const int sms = num_sms();
+  const int64_t rhs_ld = 2 * D64;
+
+  // S = R W into RHS[:, :D], RHS[:, D:] = I
+  __nv_bfloat16* r_hi = reinterpret_cast<__nv_bfloat16*>(split);
+  __nv_bfloat16* r_lo = r_hi + D64 * D64;
+  split_bf16_kernel<<<sms * 4, 256, 0, st>>>(R, r_hi, r_lo, D64 * D64);
+  init_rhs_kernel<<<sms * 4, 256, 0, st>>>(RHS, D);
+  ispa_status_t s1 = gemm_hilo_w(D, D, r_hi, r_lo, W, D, RHS, rhs_ld, st);
+  if (s1 != ISPA_OK) return s1;
+  trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
+  shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
+  for (int k = 0; k < nb; ++k) {
+    const int rest = nb - k - 1;
+    const int off = (k + 1) * kT;
+    const int rhs_cols = D + off;  // nonzero columns of the panel's rows of [L^-1 S | L^-1]
+    panel_factor_kernel<<<rest + (rhs_cols + kT - 1) / kT, 256, 0, st>>>(
+        M, D, k, rest, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, status);
+    if (rest > 0) {
+      s1 = absorb_step_update(D - off, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, rhs_cols,
+                              M + (int64_t)off * D + off, D64, RHS + (int64_t)off * rhs_ld, rhs_ld, st);
+      if (s1 != ISPA_OK) return s1;
+    }
+  }
+  // dW = (L^-1)^T (L^-1 S): hi/lo of L^-1 S into M's storage, of L^-1 into the split area
+  __nv_bfloat16* yh = reinterpret_cast<__nv_bfloat16*>(M);
+  __nv_bfloat16* yl = yh + D64 * D64;
+  __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(split);
+  __nv_bfloat16* xl = xh + D64 * D64;
+  split_rhs_kernel<<<sms * 4, 256, 0, st>>>(RHS, D, yh, yl, xh, xl);
+  if (cudaMemsetAsync(dW, 0, (size_t)D64 * D64 * 4, st) != cudaSuccess) return check_launch("cudaMemsetAsync of dW");
+  s1 = gemm_split3_xt_y(D, D, xh, xl, D64, yh, yl, D64, dW, D64, st);
+  if (s1 != ISPA_OK) return s1;
+  if (w_new) wnew_kernel<<<sms * 4, 256, 0, st>>>(W, dW, w_new, D64 * D64);
+  return check_launch("absorb_solve");
+}
 
 // C[M, N] (= | +=) A[M, K] W[K, N] on the tensor cores (bf16 operands, fp32 C).
 ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_stride, const void* w, int64_t N,
                                float* c, int64_t ldc, bool accumulate, cudaStream_t stream);
 
-ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D64,
-                                  double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
-                                  int32_t* status, cudaStream_t st) {
+// Compact form of the solve (workspace 4 D^2 + 256 D + 256 bytes): the same
+// factorisation with its updates and triangular solves on the CUDA cores in
+// fp32.  Used for fp32 W (whose 1e-3 accuracy the split-precision products do
+// not keep for ill-conditioned statistics), for D that the tensor-core form
+// does not tile, and by the no-allocation entry point.
+ispa_status_t absorb_solve_compact(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D64,
+                                   double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
+                                   int32_t* status, cudaStream_t st) {
   using namespace simt;
   const int D = (int)D64;
   const int nb = D / kT;
@@ -450,6 +775,15 @@ ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W,
       wnew_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(W), dW, static_cast<float*>(w_new), n);
   }
   return check_launch("absorb_solve");
+}
+
+ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D,
+                                  double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
+                                  int32_t* status, cudaStream_t st) {
+  if (tc_eligible(w_dt, D))
+    return absorb_solve_tc(G, R, static_cast<const __nv_bfloat16*>(W), D, lam_abs, lam_rel, dW,
+                           static_cast<__nv_bfloat16*>(w_new), workspace, status, st);
+  return absorb_solve_compact(G, R, W, w_dt, D, lam_abs, lam_rel, dW, w_new, workspace, status, st);
 }
 
 // ------------------------------------------------------- layer selection

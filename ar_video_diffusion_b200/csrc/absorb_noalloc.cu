@@ -23,10 +23,10 @@
 
 namespace ispa {
 
-size_t absorb_workspace_bytes(int64_t D);
-ispa_status_t absorb_solve_launch(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D,
-                                  double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
-                                  int32_t* status, cudaStream_t st);
+size_t absorb_compact_workspace_bytes(int64_t D);
+ispa_status_t absorb_solve_compact(const float* G, const float* R, const void* W, ispa_dtype_t w_dt, int64_t D,
+                                   double lam_abs, double lam_rel, float* dW, void* w_new, void* workspace,
+                                   int32_t* status, cudaStream_t st);
 
 constexpr int64_t kNoAllocMaxD = 2048;
 constexpr size_t kNoAllocBytes = (size_t)(4 * kNoAllocMaxD * kNoAllocMaxD + 256 * kNoAllocMaxD + 256);
@@ -116,12 +116,14 @@ extern "C" ispa_status_t ispa_absorb_solve_noalloc(const float* G, const float* 
     return invalid("lambda_abs and lambda_rel must be finite and >= 0");
   for (const void* p : {(const void*)G, (const void*)R, W, (const void*)delta_w, (const void*)w_new})
     if (p && !aligned16(p)) return invalid("matrices must be 16-byte aligned");
-  if (absorb_workspace_bytes(d_model) > kNoAllocBytes) return unsupported("scratch too small for d_model");
+  if (absorb_compact_workspace_bytes(d_model) > kNoAllocBytes) return unsupported("scratch too small for d_model");
   void* scratch = nullptr;
   ispa_status_t st = scratch_for_current_device(&scratch);
   if (st != ISPA_OK) return st;
-  // Every working matrix of the solve is written before it is read, so the
-  // stale contents left by an earlier call need no clearing.
-  return absorb_solve_launch(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, scratch, dev_status,
-                             static_cast<cudaStream_t>(stream));
+  // The compact form of the solve (working matrices 4 d^2 + 256 d + 256
+  // bytes) keeps the array small.  Every working matrix of it is written
+  // before it is read, so the stale contents left by an earlier call need no
+  // clearing.
+  return absorb_solve_compact(G, R, W, w_dt, d_model, lambda_abs, lambda_rel, delta_w, w_new, scratch, dev_status,
+                              static_cast<cudaStream_t>(stream));
 }

@@ -14,28 +14,33 @@
 //               released once S(j) is done, a V tile after PV(j));
 //   warp 1      tcgen05 issuer, the whole warp converged, one elected lane
 //               issuing: S(j) = Q K(j)^T (both operands K-major in shared
-//               memory) and O_w += P(j) V(j) (P from tensor memory, V
-//               MN-major in shared memory);
+//               memory) and O += P(j) V(j) (P from tensor memory, V MN-major
+//               in shared memory);
 //   warp 2      allocates / frees the 512 tensor-memory columns;
-//   warps 4-11  softmax: two warpgroups; warpgroup w owns the key tiles
+//   warps 4-11  softmax: two warpgroups; warpgroup w takes the key tiles
 //               j = w mod 2; thread = query row = TMEM lane.
-// Tensor memory: one S buffer and one O accumulator per warpgroup
-// (2 x 128 + 2 x head_dim columns).  Each warpgroup runs its own online
-// softmax (running maximum and sum) over its tiles; the two are merged once,
-// when a result is normalised.  The issue order S(0), S(1), PV(0), S(2),
-// PV(1), ... lets one warpgroup exponentiate while the other's products run.
-// A softmax thread holds the whole 128-key row of S in registers (the
-// warpgroups' register budget is raised with setmaxnreg) and writes the bf16
-// P into the first 64 columns of its S buffer.  Online softmax in the log2
-// domain with a lazily updated maximum: O_w is rescaled only when the
-// running maximum grows by more than 2^16 (P <= 2^16 is exact-range in bf16
-// and keeps the fp32 sums far from overflow; relative precision does not
-// depend on the scale).
-// Dual mode: before its first history tile each warpgroup takes a local
-// checkpoint; warpgroup 0 merges both accumulators and writes A_loc, LSE_loc,
-// and both restart; the epilogue fuses the history result with A_loc
-// (logaddexp of the two LSEs).  Single-pass mode runs one softmax over every
-// tile.
+// Tensor memory: three S buffers (tile j uses buffer j mod 3) and ONE O
+// accumulator (head_dim columns) that both warpgroups' products add into.
+// With three S buffers, S(j+3) is issued right after PV(j) (the product that
+// reads P(j) out of the same columns), so a warpgroup's next S is computed
+// while it is still exponentiating: the tensor core runs PV(j), S(j+3) while
+// the softmax of tile j+1 runs, and neither waits for the other's chain.
+// Online softmax in the log2 domain with one running maximum per row shared
+// by the two warpgroups: the warpgroup of tile j reads the maximum m(j-1)
+// that tile j-1 used (a per-row value in shared memory, published through one
+// mbarrier per warp quarter), decides m(j), publishes it before its
+// exponentials, and computes P(j) = 2^(s scale log2e - m(j)).  The maximum is
+// raised lazily: only when a tile's maximum exceeds m(j-1) by more than 2^16
+// (P <= 2^16 is exact-range in bf16 and keeps the fp32 sums far from
+// overflow), and then O -- holding sum_{i<j} P(i) V(i) -- is rescaled by the
+// warpgroup of tile j once PV(j-1) has completed and before it hands P(j)
+// over, so every product lands on the right scale.  Each warpgroup keeps its
+// own partial row sum, brought to the current maximum when it next uses it.
+// Dual mode: once PV of the last local tile has completed, both warpgroups
+// normalise O (each writes half of the channels of A_loc) and LSE_loc is
+// written; the first history product then restarts O and the maximum chain
+// restarts.  The epilogue fuses the history result with A_loc (logaddexp of
+// the two LSEs).  Single-pass mode runs one softmax over every tile.
 #include <cstring>
 
 #include "internal.h"
@@ -51,8 +56,9 @@ constexpr int kMaxSeg = ISPA_MAX_SEGMENTS;
 constexpr float kRescaleLog2 = 16.0f;  // lazy rescale threshold (log2)
 constexpr float kLn2 = 0.69314718055994530942f;
 // tensor-memory column map
-constexpr uint32_t kTmS = 0;    // S buffers: warpgroup w at kTmS + 128 w
-constexpr uint32_t kTmO = 256;  // O accumulators: warpgroup w at kTmO + w * head_dim
+constexpr int kNS = 3;          // S buffers: tile j uses buffer j mod 3 at kTmS + 128 (j mod 3)
+constexpr uint32_t kTmS = 0;
+constexpr uint32_t kTmO = 384;  // the O accumulator (head_dim columns)
 // bit j set: column pair j (mod 8) of a score row takes 2^x from the FMA-pipe
 // polynomial (exp2_fma2) instead of the special-function unit
 constexpr uint32_t kEmuPairs = 0x00u;
@@ -87,10 +93,12 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + NST * kTileBytes;
-  static constexpr int kXs = kV + NST * kTileBytes;  // warpgroup 1's (m, l) per row at the local checkpoint
-  static constexpr int kBars = kXs + 2 * kBM * 4;
-  // kv_full[NST], kv_empty[NST], q_full, s_full[2], p_full[2], pv_done[2], ck_done, xsum[2], teardown
-  static constexpr int kNumBars = 4 * NST + 1 + 2 + 2 + 2 + 1 + 2 + 1;
+  static constexpr int kXs = kV + NST * kTileBytes;  // local checkpoint exchange: (m, l) per row
+  static constexpr int kMref = kXs + 2 * kBM * 4;     // the shared running maximum, one float per row
+  static constexpr int kBars = kMref + kBM * 4;
+  // kv_full, kv_empty, v_full, v_empty [NST]; q_full; s_full, p_full, pv_done [3]; mref_full[4];
+  // ck_ready, ck_done, fin_ready; xsum[3]; teardown
+  static constexpr int kNumBars = 4 * NST + 1 + 3 * kNS + 4 + 3 + 3 + 1;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -176,12 +184,35 @@ __device__ void producer(const Params& p, uint8_t* smem, bool v_side, uint64_t* 
 }
 
 // ------------------------------------------------------------- MMA issuer
-// The whole warp runs the loop; one elected lane issues.  Key tile i belongs to softmax
-// warpgroup i & 1, whose S buffer and O accumulator it uses.
+// The whole warp runs the loop; one elected lane issues.  Tile j's S goes to
+// S buffer j mod 3 and its P is read from there by PV(j); every PV adds into
+// the one O accumulator.  Issue order: S(0), S(1), S(2), then per tile j:
+// PV(j), S(j + 3) (into the buffer PV(j) has just read: tcgen05 MMAs of one
+// thread execute in issue order).
+// The CTA's mbarriers, at fixed offsets from one base (so that an address
+// costs one add, not a live register).
+template <int NST>
+struct Bars {
+  uint64_t* base;
+  __device__ __forceinline__ uint64_t* kv_full(int i) const { return base + i; }
+  __device__ __forceinline__ uint64_t* kv_empty(int i) const { return base + NST + i; }
+  __device__ __forceinline__ uint64_t* v_full(int i) const { return base + 2 * NST + i; }
+  __device__ __forceinline__ uint64_t* v_empty(int i) const { return base + 3 * NST + i; }
+  __device__ __forceinline__ uint64_t* q_full() const { return base + 4 * NST; }
+  __device__ __forceinline__ uint64_t* s_full(int b) const { return base + 4 * NST + 1 + b; }     // per S buffer
+  __device__ __forceinline__ uint64_t* p_full(int b) const { return base + 4 * NST + 4 + b; }
+  __device__ __forceinline__ uint64_t* pv_done(int b) const { return base + 4 * NST + 7 + b; }
+  __device__ __forceinline__ uint64_t* mref_full(int q) const { return base + 4 * NST + 10 + q; }  // per warp quarter
+  __device__ __forceinline__ uint64_t* ck_ready() const { return base + 4 * NST + 14; }
+  __device__ __forceinline__ uint64_t* ck_done() const { return base + 4 * NST + 15; }
+  __device__ __forceinline__ uint64_t* fin_ready() const { return base + 4 * NST + 16; }
+  __device__ __forceinline__ uint64_t* xsum(int k) const { return base + 4 * NST + 17 + k; }
+  __device__ __forceinline__ uint64_t* teardown() const { return base + 4 * NST + 20; }
+  static constexpr int kCount = 4 * NST + 21;
+};
+
 template <int HD, int NST>
-__device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uint64_t* kv_full, uint64_t* kv_empty,
-                           uint64_t* v_full, uint64_t* v_empty, uint64_t* s_full, uint64_t* p_full, uint64_t* pv_done, uint64_t* ck_done,
-                           uint64_t* teardown, volatile int* abort_flag, uint32_t tmem) {
+__device__ void mma_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, volatile int* abort_flag, uint32_t tmem) {
   using L = Layout<HD, NST>;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
@@ -195,171 +226,167 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, uint64_t* q_full, uin
   };
   auto issue_s = [&](int j) -> bool {
     const int stage = j % NST;
-    if (!wait(&kv_full[stage], (j / NST) & 1)) return false;
+    if (!wait(B.kv_full(stage), (j / NST) & 1)) return false;
     tc_fence_after();
     const uint32_t kb = sK + stage * L::kTileBytes;
-    const uint32_t d = tmem + kTmS + (j & 1) * 128;
+    const uint32_t d = tmem + kTmS + (j % kNS) * 128;
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
       umma_ss_warp(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
                    kk > 0 ? 1u : 0u);
     }
-    umma_commit_warp(&s_full[j & 1]);
-    umma_commit_warp(&kv_empty[stage]);
+    umma_commit_warp(B.s_full(j % kNS));
+    umma_commit_warp(B.kv_empty(stage));
     return true;
   };
 
-  bool ok = wait(q_full, 0);
+  bool ok = wait(B.q_full(), 0);
   tc_fence_after();
-  if (ok && T > 0) ok = issue_s(0);
-  if (ok && T > 1) ok = issue_s(1);
-  bool ck_seen = false;
+  for (int j = 0; ok && j < kNS && j < T; ++j) ok = issue_s(j);
   for (int i = 0; ok && i < T; ++i) {
-    const int w = i & 1;
-    const bool first_hist = ck && i >= n_loc && i - 2 < n_loc;
-    const bool fresh = i < 2 || first_hist;
-    if (first_hist && !ck_seen) {
-      // the first history products overwrite the accumulators; the local
-      // result must have been read out of them first
-      if (!wait(ck_done, 0)) break;
-      ck_seen = true;
-    }
+    const int b = i % kNS;
+    const bool first_hist = ck && i == n_loc;
+    const bool fresh = i == 0 || first_hist;
+    // the first history product overwrites O: the local result must have
+    // been read out of it first
+    if (first_hist && !wait(B.ck_done(), 0)) break;
     const int stage = i % NST;
     const uint32_t vb = sV + stage * L::kTileBytes;
-    const uint32_t pb = tmem + kTmS + w * 128;
-    // p_full[w] completes once per tile of warpgroup w; its next phase needs
-    // S(i + 2), issued below, so the parity is unambiguous
-    if (!wait(&v_full[stage], (i / NST) & 1)) break;
-    if (!wait(&p_full[w], (i >> 1) & 1)) break;
+    const uint32_t pb = tmem + kTmS + b * 128;
+    if (!wait(B.v_full(stage), (i / NST) & 1)) break;
+    // p_full[b] completes once per use of buffer b; its next phase needs
+    // S(i + 3), issued below, so the parity is unambiguous
+    if (!wait(B.p_full(b), (i / kNS) & 1)) break;
     tc_fence_after();
-    // O_w += P V: P (bf16, 128 keys) in the first 64 columns of the S buffer
+    // O += P V: P (bf16, 128 keys) in the first 64 columns of S buffer b
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      umma_ts_warp(tmem + kTmO + w * HD, pb + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024), kIdescPV,
+      umma_ts_warp(tmem + kTmO, pb + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024), kIdescPV,
                    (kk > 0 || !fresh) ? 1u : 0u);
-    umma_commit_warp(&v_empty[stage]);
-    umma_commit_warp(&pv_done[w]);
-    if (i + 2 < T) ok = issue_s(i + 2);
+    umma_commit_warp(B.v_empty(stage));
+    umma_commit_warp(B.pv_done(b));
+    if (ck && i == n_loc - 1) umma_commit_warp(B.ck_ready());
+    if (i == T - 1) umma_commit_warp(B.fin_ready());
+    if (i + kNS < T) ok = issue_s(i + kNS);
   }
   // every MMA must have completed before tensor memory is released
-  umma_commit_warp(teardown);
-  mbar_wait_drain(teardown, 0, 100000000ull);
+  umma_commit_warp(B.teardown());
+  mbar_wait_drain(B.teardown(), 0, 100000000ull);
   __syncwarp();
 }
 
 // ------------------------------------------------------------------ softmax
-// bf16 pair from two non-negative floats, rounded to nearest (ties away from
-// zero) with integer ALU operations, so the conversion does not compete with
-// the exponentials for the special-function pipe.
-__device__ __forceinline__ uint32_t pack_p_bf16x2(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
 
 struct Row {
-  int wg, lane, row, grow;
+  int wg, lane, row, grow, quarter;
   bool row_ok;
   uint32_t lane_base;
 };
 
-// Merged, normalised accumulator for channels [32 cc, 32 cc + 32) of this
-// row: (O_0 w0 + O_1 w1) / lt.  A weight of 0 means that accumulator holds
-// nothing of this result (it may hold stale data) and is not read.
-template <int HD>
-__device__ __forceinline__ void load_merged(const Row& r, int cc, float w0, float w1, float inv, float (&x)[32]) {
-  uint32_t a[32], b[32];
+// Normalised accumulator for channels [32 cc, 32 cc + 32) of this row: O / l.
+__device__ __forceinline__ void load_o(const Row& r, int cc, float inv, float (&x)[32]) {
+  uint32_t a[32];
   tmem_ld32(r.lane_base + kTmO + 32 * cc, a);
-  tmem_ld32(r.lane_base + kTmO + HD + 32 * cc, b);
   tmem_wait_ld();
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float u = w0 != 0.f ? __uint_as_float(a[j]) * w0 : 0.f;
-    const float v = w1 != 0.f ? __uint_as_float(b[j]) * w1 : 0.f;
-    x[j] = (u + v) * inv;
-  }
+  for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(a[j]) * inv;
 }
 
-// Waits (all lanes) for the product of warpgroup w's tile number k (counted
-// per warpgroup) to have completed.
-__device__ __forceinline__ bool wait_pv(uint64_t* pv_done, int w, int k, volatile int* abort_flag) {
-  if (k < 0) return true;
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[w], k & 1, abort_flag));
-  tc_fence_after();
-  return ok;
+// Combined row sum of the two warpgroups, each (m, l) relative to its own
+// maximum: returns (m, l) relative to the larger one.
+__device__ __forceinline__ float2 combine(float m0, float l0, float m1, float l1) {
+  const float mm = fmaxf(m0, m1);
+  const float a = l0 > 0.f ? l0 * ex2(m0 - mm) : 0.f;
+  const float b = l1 > 0.f ? l1 * ex2(m1 - mm) : 0.f;
+  return make_float2(mm, a + b);
 }
 
 template <int HD, int NST>
-__device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t* s_full, uint64_t* p_full,
-                        uint64_t* pv_done, uint64_t* ck_done, uint64_t* xsum, volatile int* abort_flag, int q0,
-                        int head) {
+__device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bars<NST>& B, volatile int* abort_flag,
+                        int q0, int head) {
   using L = Layout<HD, NST>;
-  float* xck = reinterpret_cast<float*>(smem + L::kXs);  // checkpoint: warpgroup 1's (m, l) per row
-  float* xfin = reinterpret_cast<float*>(smem + L::kQ);  // final: [wg][m, l, lse_loc][row]; Q is dead by then
+  float* xck = reinterpret_cast<float*>(smem + L::kXs);  // checkpoint exchange [m | l][row]
+  float* mref = reinterpret_cast<float*>(smem + L::kMref);
+  float* xfin = reinterpret_cast<float*>(smem + L::kQ);  // final: [wg][m, l][row]; Q is dead by then
   Row r;
   const int warp = threadIdx.x >> 5;
   r.wg = (warp - 4) >> 2;
+  r.quarter = warp & 3;
   r.lane = threadIdx.x & 31;
-  r.row = (warp & 3) * 32 + r.lane;
+  r.row = r.quarter * 32 + r.lane;
   r.grow = q0 + r.row;
   r.row_ok = r.grow < p.n_q;
-  r.lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  r.lane_base = tmem + ((uint32_t)(r.quarter * 32) << 16);
   const int w = r.wg;
-  const uint32_t o_own = r.lane_base + kTmO + w * HD;
-  const uint32_t sbuf = r.lane_base + kTmS + w * 128;
+  const uint32_t o_row = r.lane_base + kTmO;
   const float sl2 = p.scale_log2;
   const int T = p.n_tiles, n_loc = p.n_local_tiles;
   const bool dual = p.dual != 0;
   const bool ck = dual && n_loc > 0 && n_loc < T;
   bool ck_pending = ck;
   bool ok = true;
+  auto all = [&](bool v) { return __all_sync(0xffffffffu, v); };
 
-  float m_used = -INFINITY, l = 0.f, lse_loc2 = 0.f;
-  bool o_live = false;  // O_w holds products of the current accumulation
+  // this warpgroup's partial row sum l, relative to the maximum m_l it last used
+  float m_l = -INFINITY, l = 0.f, lse_loc2 = 0.f;
 
-  // local result: the two warpgroups' accumulators are merged, normalised and
-  // written (A_loc, LSE_loc) by warpgroup 0; then both restart
-  auto checkpoint = [&](int k_next) -> bool {
-    if (!wait_pv(pv_done, w, k_next - 1, abort_flag)) return false;  // own last local product
+  // local result: O / l written as A_loc (warpgroup w writes channels
+  // [w HD/2, (w + 1) HD/2)), LSE_loc by warpgroup 0; then a fresh accumulation
+  auto checkpoint = [&]() -> bool {
+    if (!all(mbar_wait(B.ck_ready(), 0, abort_flag))) return false;  // PV of the last local tile complete
+    tc_fence_after();
+    float mf, lt;
     if (w == 1) {
-      xck[r.row] = m_used;
+      xck[r.row] = m_l;
       xck[kBM + r.row] = l;
-      mbar_arrive(&xsum[0]);
+      mbar_arrive(B.xsum(0));
+      if (!all(mbar_wait(B.xsum(1), 0, abort_flag))) return false;
+      mf = xck[r.row];
+      lt = xck[kBM + r.row];
     } else {
-      if (!wait_pv(pv_done, 1, (n_loc >> 1) - 1, abort_flag)) return false;  // warpgroup 1's last local product
-      if (!__all_sync(0xffffffffu, mbar_wait(&xsum[0], 0, abort_flag))) return false;
-      const float m1 = xck[r.row], l1 = xck[kBM + r.row];
-      const float mm = fmaxf(m_used, m1);
-      const float w0 = l > 0.f ? ex2(m_used - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
-      const float lt = l * w0 + l1 * w1;
-      const float inv = 1.0f / lt;
-      __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD;
-#pragma unroll 1
-      for (int cc = 0; cc < HD / 32; ++cc) {
-        float x[32];
-        load_merged<HD>(r, cc, w0, w1, inv, x);
-        if (r.row_ok) store_bf16x32(dst + 32 * cc, x);
-      }
-      lse_loc2 = mm + log2f(lt);
-      if (r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
-      tc_fence_before();
-      __syncwarp();
-      if (r.lane == 0) mbar_arrive(ck_done);
+      if (!all(mbar_wait(B.xsum(0), 0, abort_flag))) return false;
+      const float2 c = combine(m_l, l, xck[r.row], xck[kBM + r.row]);
+      mf = c.x;
+      lt = c.y;
+      xck[r.row] = mf;
+      xck[kBM + r.row] = lt;
+      mbar_arrive(B.xsum(1));
     }
-    m_used = -INFINITY;
+    const float inv = 1.0f / lt;
+    __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD + w * (HD / 2);
+#pragma unroll 1
+    for (int kc = 0; kc < HD / 64; ++kc) {
+      float x[32];
+      load_o(r, w * (HD / 64) + kc, inv, x);
+      if (r.row_ok) store_bf16x32(dst + 32 * kc, x);
+    }
+    lse_loc2 = mf + log2f(lt);
+    if (w == 0 && r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
+    tc_fence_before();
+    __syncwarp();
+    if (r.lane == 0) mbar_arrive(B.ck_done());
+    m_l = -INFINITY;
     l = 0.f;
-    o_live = false;
     return true;
   };
 
 #pragma unroll 1
   for (int i = w; i < T; i += 2) {
-    const int k = i >> 1;  // this warpgroup's tile count
+    const int b = i % kNS;
     if (ck_pending && i >= n_loc) {
       ck_pending = false;
-      if (!(ok = checkpoint(k))) break;
+      if (!(ok = checkpoint())) break;
     }
-    ok = __all_sync(0xffffffffu, mbar_wait(&s_full[w], k & 1, abort_flag));
-    if (!ok) break;
+    // the maximum tile i - 1 used (none at the start of an accumulation),
+    // read before the scores occupy the registers
+    const bool first_acc = i == 0 || (ck && i == n_loc);
+    float m_prev = -INFINITY;
+    if (!first_acc) {
+      if (!(ok = all(mbar_wait(B.mref_full(r.quarter), (i - 1) & 1, abort_flag)))) break;
+      m_prev = mref[r.row];
+    }
+    if (!(ok = all(mbar_wait(B.s_full(b), (i / kNS) & 1, abort_flag)))) break;
     tc_fence_after();
     int valid = kBN;
 #pragma unroll
@@ -367,6 +394,7 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
       if (i == p.seg_last_tile[q]) valid = p.seg_last_valid[q];
 
     // the whole 128-key row of S in registers
+    const uint32_t sbuf = r.lane_base + kTmS + b * 128;
     uint32_t s[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, s[c]);
@@ -378,9 +406,31 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
         for (int j = 0; j < 32; ++j)
           if (c * 32 + j >= valid) s[c][j] = __float_as_uint(-INFINITY);
     }
+    // tile maximum (scaled, log2 domain; -inf if every key is masked)
+    float m_tile;
+    {
+      float mc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* v = &s[q >> 1][(q & 1) * 16];
+        mc[q] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+#pragma unroll
+        for (int j = 1; j < 8; ++j) mc[q] = fmax3(mc[q], __uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+      }
+      const float a = fmax3(mc[0], mc[1], mc[2]), bb = fmax3(mc[3], mc[4], mc[5]), c = fmaxf(mc[6], mc[7]);
+      m_tile = fmax3(a, bb, c) * sl2;
+    }
+    const bool fin_prev = m_prev != -INFINITY;
+    const bool grow = __any_sync(0xffffffffu, fin_prev && m_tile > m_prev + kRescaleLog2);
+    const float m_i = !fin_prev ? m_tile : (grow ? fmaxf(m_prev, m_tile) : m_prev);
+    mref[r.row] = m_i;
+    mbar_arrive(B.mref_full(r.quarter));
+
     // P = 2^(s * scale_log2 - m) as bf16 into the first 64 columns of the S
-    // buffer (whose values are all in registers by now); returns the sum of P
-    auto exponentiate = [&](float m) -> float {
+    // buffer (whose values are all in registers by now); the sum of P
+    float psum;
+    {
+      const float m = m_i == -INFINITY ? 0.f : m_i;
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
       float2 sum2[4];
 #pragma unroll
@@ -393,83 +443,52 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
               ffma2(make_float2(__uint_as_float(s[c][2 * j]), __uint_as_float(s[c][2 * j + 1])), sc2, nm2);
           const float2 pv = (kEmuPairs & (1u << (j & 7))) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
           sum2[c] = fadd2(sum2[c], pv);
-          pk[j] = pack_p_bf16x2(pv.x, pv.y);
+          pk[j] = pack_bf16x2(pv.x, pv.y);  // one packed round-to-nearest-even conversion
         }
         tmem_st16(sbuf + 16 * c, pk);
       }
       const float2 st2 = fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3]));
-      return st2.x + st2.y;
-    };
-    auto tile_max = [&]() -> float {
-      float mc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t* v = &s[q >> 1][(q & 1) * 16];
-        mc[q] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
-#pragma unroll
-        for (int j = 1; j < 8; ++j) mc[q] = fmax3(mc[q], __uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-      }
-      const float a = fmax3(mc[0], mc[1], mc[2]), b = fmax3(mc[3], mc[4], mc[5]), c = fmaxf(mc[6], mc[7]);
-      return fmax3(a, b, c) * sl2;  // -inf if all masked
-    };
-    // exponentials with the running maximum straight away, the tile maximum
-    // alongside; a growth beyond 2^16 (rare, and always at the start of an
-    // accumulation) rescales what was accumulated and redoes the tile.  O_w
-    // is quiescent here: S(i) was issued after this warpgroup's previous
-    // product, and its completion implies that product's.
-    const bool first = __any_sync(0xffffffffu, m_used == -INFINITY);
-    float psum = first ? 0.f : exponentiate(m_used);
-    const float m_tile = tile_max();
-    if (first || __any_sync(0xffffffffu, m_tile > m_used + kRescaleLog2)) {
-      const float m_new = fmaxf(m_used, m_tile);
-      // rows whose keys are all masked so far keep m = -inf: their P is exactly 0
-      const float f = (m_used == -INFINITY || m_new == -INFINITY) ? 0.f : ex2(m_used - m_new);
-      if (o_live) {
-#pragma unroll 1
-        for (int cc = 0; cc < HD / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(o_own + 32 * cc, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-          tmem_st32(o_own + 32 * cc, o);
-        }
-      }
-      tmem_wait_st();  // the first pass's P stores complete before they are overwritten
-      l *= f;
-      m_used = m_new;
-      psum = exponentiate(m_used == -INFINITY ? 0.f : m_used);
+      psum = st2.x + st2.y;
     }
+    if (l > 0.f && m_i != m_l) l *= ex2(m_l - m_i);
     l += psum;
-    if (!ok) break;
+    if (m_i != -INFINITY) m_l = m_i;
+
+    // a raised maximum: O (every product before tile i) moves to the new
+    // scale once PV(i - 1) has completed; PV(i) waits for p_full below
+    const bool rescale_row = fin_prev && m_i > m_prev;
+    if (__any_sync(0xffffffffu, rescale_row)) {
+      if (!(ok = all(mbar_wait(B.pv_done((i - 1) % kNS), ((i - 1) / kNS) & 1, abort_flag)))) break;
+      tc_fence_after();
+      const float f = rescale_row ? ex2(m_prev - m_i) : 1.f;
+#pragma unroll 1
+      for (int cc = 0; cc < HD / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(o_row + 32 * cc, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+        tmem_st32(o_row + 32 * cc, o);
+      }
+    }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (r.lane == 0) mbar_arrive(&p_full[w]);
-    o_live = true;
+    if (r.lane == 0) mbar_arrive(B.p_full(b));
   }
   if (!ok || *abort_flag) return;
-  if (ck_pending) {  // no history tile fell to this warpgroup
-    if (!checkpoint((T - w + 1) >> 1)) return;
-  }
-  // both accumulators final (own first, so the other is at most one phase behind)
-  const int n_own = (T - w + 1) >> 1, n_other = (T - (1 - w) + 1) >> 1;
-  if (!wait_pv(pv_done, w, n_own - 1, abort_flag)) return;
-  if (!wait_pv(pv_done, 1 - w, n_other - 1, abort_flag)) return;
-  // final merge of the two warpgroups' statistics (the Q tile is no longer read)
-  xfin[(w * 3 + 0) * kBM + r.row] = m_used;
-  xfin[(w * 3 + 1) * kBM + r.row] = l;
-  xfin[(w * 3 + 2) * kBM + r.row] = lse_loc2;
-  mbar_arrive(&xsum[1]);
-  if (!__all_sync(0xffffffffu, mbar_wait(&xsum[1], 0, abort_flag))) return;
-  const float m0 = xfin[r.row], l0 = xfin[kBM + r.row];
-  const float m1 = xfin[3 * kBM + r.row], l1 = xfin[4 * kBM + r.row];
-  lse_loc2 = xfin[2 * kBM + r.row];  // computed by warpgroup 0 at the checkpoint
-  const float mm = fmaxf(m0, m1);
-  const float w0 = l0 > 0.f ? ex2(m0 - mm) : 0.f, w1 = l1 > 0.f ? ex2(m1 - mm) : 0.f;
-  const float lt = l0 * w0 + l1 * w1;
-  const float inv = 1.0f / lt;
-  const float lse2 = mm + log2f(lt);
+  if (ck_pending && !checkpoint()) return;  // no history tile fell to this warpgroup
+  // the last product complete: O final
+  if (!all(mbar_wait(B.fin_ready(), 0, abort_flag))) return;
+  tc_fence_after();
+  // final row sums of the two warpgroups (the Q tile is no longer read)
+  xfin[(w * 2 + 0) * kBM + r.row] = m_l;
+  xfin[(w * 2 + 1) * kBM + r.row] = l;
+  mbar_arrive(B.xsum(2));
+  if (!all(mbar_wait(B.xsum(2), 0, abort_flag))) return;
+  const float2 cmb = combine(xfin[r.row], xfin[kBM + r.row], xfin[2 * kBM + r.row], xfin[3 * kBM + r.row]);
+  const float inv = 1.0f / cmb.y;
+  const float lse2 = cmb.x + log2f(cmb.y);
   const int64_t li = (int64_t)head * p.n_q + r.grow;
   const int64_t base = (int64_t)r.grow * p.out_stride + head * HD + w * (HD / 2);
   const int c_first = w * (HD / 64);  // this warpgroup's 32-channel blocks
@@ -478,7 +497,7 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
 #pragma unroll 1
     for (int kc = 0; kc < HD / 64; ++kc) {
       float x[32];
-      load_merged<HD>(r, c_first + kc, w0, w1, inv, x);
+      load_o(r, c_first + kc, inv, x);
       if (!r.row_ok) continue;
       store_bf16x32(p.a_full + base + 32 * kc, x);
       if (dual) {
@@ -497,14 +516,15 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, uint64_t*
     }
     return;
   }
-  // fuse the history result with the checkpointed local result
+  // fuse the history result with the checkpointed local result (this
+  // warpgroup wrote the same channels of A_loc itself)
   const float mx = fmaxf(lse_loc2, lse2);
   const float lse_full2 = mx + log2f(exp2f(lse_loc2 - mx) + exp2f(lse2 - mx));
   const float wgt = exp2f(lse2 - lse_full2);
 #pragma unroll 1
   for (int kc = 0; kc < HD / 64; ++kc) {
     float oh[32];
-    load_merged<HD>(r, c_first + kc, w0, w1, inv, oh);
+    load_o(r, c_first + kc, inv, oh);
     if (!r.row_ok) continue;
     float a[32], full[32], dl[32];
     unpack_bf16x32(reinterpret_cast<const uint4*>(p.a_loc + base + 32 * kc), a);
@@ -526,17 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = kv_full + NST;
-  uint64_t* v_full = kv_empty + NST;
-  uint64_t* v_empty = v_full + NST;
-  uint64_t* q_full = v_empty + NST;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* ck_done = pv_done + 2;
-  uint64_t* xsum = ck_done + 1;
-  uint64_t* teardown = xsum + 2;
+  Bars<NST> B{bars};
+  static_assert(Bars<NST>::kCount == L::kNumBars, "barrier count");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -545,21 +556,25 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
+      mbar_init(B.kv_full(i), 1);
+      mbar_init(B.kv_empty(i), 1);
+      mbar_init(B.v_full(i), 1);
+      mbar_init(B.v_empty(i), 1);
     }
-    mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
+    mbar_init(B.q_full(), 1);
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(B.s_full(i), 1);
+      mbar_init(B.p_full(i), 4);  // the four warps of the tile's warpgroup
+      mbar_init(B.pv_done(i), 1);
     }
-    mbar_init(ck_done, 4);
-    mbar_init(&xsum[0], 128);
-    mbar_init(&xsum[1], 256);
-    mbar_init(teardown, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(B.mref_full(i), 32);  // the 32 rows of one warp
+    mbar_init(B.ck_ready(), 1);
+    mbar_init(B.ck_done(), 8);
+    mbar_init(B.fin_ready(), 1);
+    mbar_init(B.xsum(0), 128);
+    mbar_init(B.xsum(1), 128);
+    mbar_init(B.xsum(2), 256);
+    mbar_init(B.teardown(), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -577,16 +592,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   // 128 x 88 + 256 x 208 = 384 x 168, the launch budget
   if (warp >= 4) {
     regs_inc<208>();
-    softmax<HD, NST>(p, smem, tmem, s_full, p_full, pv_done, ck_done, xsum, abort_flag, q0, head);
+    softmax<HD, NST>(p, smem, tmem, B, abort_flag, q0, head);
   } else {
     regs_dec<88>();
     if (warp == 0) {
-      if (lane == 0) producer<HD, NST>(p, smem, false, q_full, kv_full, kv_empty, abort_flag, q0, head);
+      if (lane == 0) producer<HD, NST>(p, smem, false, B.q_full(), B.kv_full(0), B.kv_empty(0), abort_flag, q0, head);
     } else if (warp == 1) {
-      mma_issuer<HD, NST>(p, smem, q_full, kv_full, kv_empty, v_full, v_empty, s_full, p_full, pv_done, ck_done, teardown, abort_flag,
-                          tmem);
+      mma_issuer<HD, NST>(p, smem, B, abort_flag, tmem);
     } else if (warp == 3) {
-      if (lane == 0) producer<HD, NST>(p, smem, true, nullptr, v_full, v_empty, abort_flag, q0, head);
+      if (lane == 0) producer<HD, NST>(p, smem, true, nullptr, B.v_full(0), B.v_empty(0), abort_flag, q0, head);
     }
   }
 

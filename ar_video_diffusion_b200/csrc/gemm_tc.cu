@@ -32,14 +32,22 @@ constexpr int kThreads = 384;
 
 enum Mode : int { kStoreBf16 = 0, kStoreF32 = 1, kReduceF32 = 2 };
 
+constexpr int kMaxPairs = 3;  // operand pairs summed into one accumulator
+
 struct Params {
-  CUtensorMap a_map;
-  CUtensorMap b_map[2];
+  // C = sum_{q < n_pairs} A_q B_q: the K loop runs over the pairs, q-major, so
+  // every pair lands in the same tensor-memory accumulator (split-precision
+  // products: hi(A) hi(B) + hi(A) lo(B) + lo(A) hi(B))
+  CUtensorMap a_map[kMaxPairs];
+  CUtensorMap b_map[2][kMaxPairs];  // [column range][pair]
   CUtensorMap c_map[2];  // output maps (32 x 32 boxes) for the TMA epilogue, when c_tma
   int32_t c_tma;
   int32_t M, N, K;
   int32_t n_split;      // columns [0, n_split) come from b_map[0] / c[0], the rest from b_map[1] / c[1]
+  int32_t n_cols[2];    // valid columns of each range (outputs beyond are not written)
+  int32_t n_pairs;
   int32_t lower_only0;  // skip tiles of the first column range that lie strictly above the diagonal
+  int32_t a_upper;      // A(m, k) = 0 for k < m: a row block skips the K steps before it
   int32_t k_per_split;  // K rows per blockIdx.z, a multiple of kBK
   void* c[2];
   int64_t ldc;
@@ -80,10 +88,12 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
   // whole-CTA early exit (before any barrier or tensor-memory use): a tile of
   // a lower-triangular output that lies strictly above the diagonal
   if (half_n == 0 && p.lower_only0 && n0 > m0 + kBM - 1) return;
-  const int k_begin = blockIdx.z * p.k_per_split;
+  int k_begin = blockIdx.z * p.k_per_split;
   const int k_end = min(p.K, k_begin + p.k_per_split);
+  if (p.a_upper) k_begin = max(k_begin, (m0 / BK) * BK);
   if (k_begin >= k_end) return;
   const int nk = (k_end - k_begin + BK - 1) / BK;
+  const int steps = p.n_pairs * nk;  // K steps over every pair
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,22 +126,26 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA
-    const CUtensorMap* bm = &p.b_map[half_n];
-    tma_prefetch_desc(&p.a_map);
-    tma_prefetch_desc(bm);
+    for (int q = 0; q < p.n_pairs; ++q) {
+      tma_prefetch_desc(&p.a_map[q]);
+      tma_prefetch_desc(&p.b_map[half_n][q]);
+    }
     int kb = 0;
-    for (; kb < nk; ++kb) {
+    for (; kb < steps; ++kb) {
       const int stage = kb % NST;
       if (kb >= NST && !mbar_wait(&empty[stage], ((kb / NST) - 1) & 1, abort_flag)) break;
       uint8_t* sa = smem + stage * L::kStage;
       uint8_t* sb = sa + L::kABytes;
-      const int k0 = k_begin + kb * BK;
+      const int q = kb / nk;
+      const int k0 = k_begin + (kb - q * nk) * BK;
+      const CUtensorMap* am = &p.a_map[q];
+      const CUtensorMap* bm = &p.b_map[half_n][q];
       mbar_arrive_expect_tx(&full[stage], L::kStage);
       if (A_MN) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_load_2d(sa + c * 8192, &p.a_map, &full[stage], m0 + 64 * c, k0);
+        for (int c = 0; c < 4; ++c) tma_load_2d(sa + c * 8192, am, &full[stage], m0 + 64 * c, k0);
       } else {
-        tma_load_2d(sa, &p.a_map, &full[stage], k0, m0);
+        tma_load_2d(sa, am, &full[stage], k0, m0);
       }
       if (B_MN) {
 #pragma unroll
@@ -140,7 +154,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
         tma_load_2d(sb, bm, &full[stage], k0, n0);
       }
     }
-    if (kb < nk) {  // unwinding after a timeout
+    if (kb < steps) {  // unwinding after a timeout
       for (int j = kb > NST ? kb - NST : 0; j < kb; ++j)
         mbar_wait_drain(&full[j % NST], (j / NST) & 1, 100000000ull);
     }
@@ -149,7 +163,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     constexpr uint32_t kIdesc = F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, A_MN, B_MN);
     const uint32_t base = smem_u32(smem);
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    for (int kb = 0; kb < steps; ++kb) {
       const int stage = kb % NST;
       if (!mbar_wait(&full[stage], (kb / NST) & 1, abort_flag)) {
         ok = false;
@@ -187,7 +201,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     if (ok && p.c_tma) {
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
-      const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
+      const int n_cols = p.n_cols[half_n];
       // The operand ring is idle once acc_full has fired (every MMA that read
       // it has completed).  Each warp stages its 32 rows in 32 x 32 blocks
       // there, double-buffered (2 x 4 KB per warp), in the swizzled layout of
@@ -256,7 +270,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     } else if (ok && !F8) {  // outputs the TMA epilogue cannot address (e4m3 callers always use TMA)
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + h * BN;
-      const int n_cols = p.n_split < p.N ? (half_n ? p.N - p.n_split : p.n_split) : p.N;
+      const int n_cols = p.n_cols[half_n];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -328,7 +342,7 @@ static ispa_status_t launch_e4m3(const Params& p, cudaStream_t stream) {
   auto kern = gemm_e4m3_kernel<BN, NST>;
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
-  dim3 grid(p.N / BN, (p.M + kBM - 1) / kBM, 1);
+  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM, 1);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
   return check_launch("gemm_e4m3_kernel");
 }
@@ -339,7 +353,7 @@ static ispa_status_t launch(const Params& p, int k_splits, cudaStream_t stream) 
   auto kern = gemm_bf16_kernel<A_MN, B_MN, BN, NST>;
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
-  dim3 grid(p.N / BN, (p.M + kBM - 1) / kBM, k_splits);
+  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM, k_splits);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
   return check_launch("gemm_bf16_kernel");
 }
@@ -356,9 +370,9 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   Params p;
   memset(&p, 0, sizeof(p));
   // A operand: element (i, n) = A_loc[n, i]  -> [K = n_rows rows, M = D contiguous]
-  if (!encode_map_bf16_2d(&p.a_map, a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
-  if (!encode_map_bf16_2d(&p.b_map[0], a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
-  if (!encode_map_bf16_2d(&p.b_map[1], a_delta, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.a_map[0], a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.b_map[0][0], a_loc, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.b_map[1][0], a_delta, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
   if (overwrite && (cudaMemsetAsync(G, 0, (size_t)D * D * 4, stream) != cudaSuccess ||
                     cudaMemsetAsync(R, 0, (size_t)D * D * 4, stream) != cudaSuccess))
     return check_launch("cudaMemsetAsync of G, R");
@@ -366,6 +380,9 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   p.N = (int32_t)(2 * D);
   p.K = (int32_t)n_rows;
   p.n_split = (int32_t)D;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)(D);
+  p.n_cols[1] = p.N - p.n_cols[0];
   p.lower_only0 = 1;
   p.c[0] = G;
   p.c[1] = R;
@@ -398,15 +415,18 @@ ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t ro
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_bf16_2d(&p.a_map, x, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
-  p.b_map[0] = p.a_map;
-  p.b_map[1] = p.a_map;
+  if (!encode_map_bf16_2d(&p.a_map[0], x, D, n_rows, row_stride * 2, 64, 64)) return ISPA_ERR_CUDA;
+  p.b_map[0][0] = p.a_map[0];
+  p.b_map[1][0] = p.a_map[0];
   if (overwrite && cudaMemsetAsync(E, 0, (size_t)D * D * 4, stream) != cudaSuccess)
     return check_launch("cudaMemsetAsync of E");
   p.M = (int32_t)D;
   p.N = (int32_t)D;
   p.K = (int32_t)n_rows;
   p.n_split = (int32_t)D;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)(D);
+  p.n_cols[1] = p.N - p.n_cols[0];
   p.lower_only0 = 1;
   p.c[0] = E;
   p.c[1] = E;
@@ -435,13 +455,16 @@ ispa_status_t gemm_rm_bf16_f32(const void* a, int64_t M, int64_t K, int64_t a_st
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_bf16_2d(&p.a_map, a, K, M, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
-  if (!encode_map_bf16_2d(&p.b_map[0], w, N, K, N * 2, 64, 64)) return ISPA_ERR_CUDA;
-  p.b_map[1] = p.b_map[0];
+  if (!encode_map_bf16_2d(&p.a_map[0], a, K, M, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.b_map[0][0], w, N, K, N * 2, 64, 64)) return ISPA_ERR_CUDA;
+  p.b_map[1][0] = p.b_map[0][0];
   p.M = (int32_t)M;
   p.N = (int32_t)N;
   p.K = (int32_t)K;
   p.n_split = (int32_t)N;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)(N);
+  p.n_cols[1] = p.N - p.n_cols[0];
   p.k_per_split = (int32_t)(((K + kBK - 1) / kBK) * kBK);
   p.c[0] = c;
   p.c[1] = c;
@@ -458,13 +481,16 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_bf16_2d(&p.a_map, a, d_in, n_rows, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
-  if (!encode_map_bf16_2d(&p.b_map[0], w, d_out, d_in, d_out * 2, 64, 64)) return ISPA_ERR_CUDA;
-  p.b_map[1] = p.b_map[0];
+  if (!encode_map_bf16_2d(&p.a_map[0], a, d_in, n_rows, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&p.b_map[0][0], w, d_out, d_in, d_out * 2, 64, 64)) return ISPA_ERR_CUDA;
+  p.b_map[1][0] = p.b_map[0][0];
   p.M = (int32_t)n_rows;
   p.N = (int32_t)d_out;
   p.K = (int32_t)d_in;
   p.n_split = (int32_t)d_out;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)(d_out);
+  p.n_cols[1] = p.N - p.n_cols[0];
   p.k_per_split = (int32_t)(((d_in + kBK - 1) / kBK) * kBK);
   p.c[0] = y;
   p.c[1] = y;
@@ -484,14 +510,17 @@ ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_ro
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_u8_2d(&p.a_map, qa, d_in, n_rows, d_in, kBK8, kBM)) return ISPA_ERR_CUDA;
+  if (!encode_map_u8_2d(&p.a_map[0], qa, d_in, n_rows, d_in, kBK8, kBM)) return ISPA_ERR_CUDA;
   const int BN = d_out % 256 == 0 ? 256 : 128;
-  if (!encode_map_u8_2d(&p.b_map[0], qw_t, d_in, d_out, d_in, kBK8, BN)) return ISPA_ERR_CUDA;
-  p.b_map[1] = p.b_map[0];
+  if (!encode_map_u8_2d(&p.b_map[0][0], qw_t, d_in, d_out, d_in, kBK8, BN)) return ISPA_ERR_CUDA;
+  p.b_map[1][0] = p.b_map[0][0];
   p.M = (int32_t)n_rows;
   p.N = (int32_t)d_out;
   p.K = (int32_t)d_in;
   p.n_split = (int32_t)d_out;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)(d_out);
+  p.n_cols[1] = p.N - p.n_cols[0];
   p.k_per_split = (int32_t)(((d_in + kBK8 - 1) / kBK8) * kBK8);
   p.c[0] = y;
   p.c[1] = y;
@@ -503,6 +532,136 @@ ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_ro
   if (!p.c_tma) return unsupported("e4m3 projection needs a 16-byte aligned output");
   if (BN == 256) return launch_e4m3<256, 3>(p, stream);
   return launch_e4m3<128, 4>(p, stream);
+}
+
+}  // namespace ispa
+
+// ------------------------------------------------------- absorb products
+// Split-precision products of the absorb solve.  An fp32 operand x is held as
+// two bf16 matrices hi = bf16(x), lo = bf16(x - hi); a product of two such
+// operands is summed in one accumulator as hi(A) hi(B) + hi(A) lo(B) +
+// lo(A) hi(B) (the dropped lo(A) lo(B) and the representation error are about
+// 2^-17 of |A| |B|).
+namespace ispa {
+
+// One trailing update of the blocked Cholesky with its right-hand sides
+// (panel width 64, rows and columns from `off`):
+//   M[off:, off:] (lower tiles) += A  [L^T]      A = -L21 (rows x 64),
+//   RHS[off:, :rhs_cols]        += A  Y_k        Y_k (64 x rhs_cols),
+// A given as K-major hi/lo [rows, 64]; L21^T as MN-major hi/lo [64, rows]
+// with row stride lt_ld; Y_k as MN-major hi/lo [64, rhs_cols] with row stride
+// y_ld.  M has row stride D, RHS row stride rhs_ld (fp32, reduced in L2).
+ispa_status_t absorb_step_update(int64_t rows, const void* a_hi, const void* a_lo, const void* lt_hi,
+                                 const void* lt_lo, int64_t lt_ld, const void* y_hi, const void* y_lo, int64_t y_ld,
+                                 int64_t rhs_cols, float* m_sub, int64_t m_ld, float* rhs_sub, int64_t rhs_ld,
+                                 cudaStream_t stream) {
+  using namespace gemm;
+  constexpr int BN = 128;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  CUtensorMap ah, al, bh0, bl0, bh1, bl1;
+  if (!encode_map_bf16_2d(&ah, a_hi, 64, rows, 128, 64, kBM) || !encode_map_bf16_2d(&al, a_lo, 64, rows, 128, 64, kBM))
+    return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&bh0, lt_hi, rows, 64, lt_ld * 2, 64, 64) ||
+      !encode_map_bf16_2d(&bl0, lt_lo, rows, 64, lt_ld * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&bh1, y_hi, rhs_cols, 64, y_ld * 2, 64, 64) ||
+      !encode_map_bf16_2d(&bl1, y_lo, rhs_cols, 64, y_ld * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  p.a_map[0] = ah, p.a_map[1] = ah, p.a_map[2] = al;
+  p.b_map[0][0] = bh0, p.b_map[0][1] = bl0, p.b_map[0][2] = bh0;
+  p.b_map[1][0] = bh1, p.b_map[1][1] = bl1, p.b_map[1][2] = bh1;
+  p.n_pairs = 3;
+  if (!encode_map_out_2d(&p.c_map[0], m_sub, true, rows, rows, m_ld * 4) ||
+      !encode_map_out_2d(&p.c_map[1], rhs_sub, true, rhs_cols, rows, rhs_ld * 4))
+    return ISPA_ERR_CUDA;
+  p.c_tma = 1;
+  p.c[0] = m_sub;
+  p.c[1] = rhs_sub;
+  p.M = (int32_t)rows;
+  p.K = 64;
+  p.k_per_split = 64;
+  p.n_split = (int32_t)((rows + BN - 1) / BN * BN);  // range 0 padded to whole tiles
+  p.N = p.n_split + (int32_t)rhs_cols;
+  p.n_cols[0] = (int32_t)rows;
+  p.n_cols[1] = (int32_t)rhs_cols;
+  p.lower_only0 = 1;
+  p.mode = kReduceF32;
+  return launch<false, true, BN, 4>(p, 1, stream);
+}
+
+// C[D, N] += sum of split-precision pairs of A^T B, A = X [K, D] lower
+// triangular (so A^T is upper: a row block of C skips the K rows above it),
+// B [K, N]; hi/lo bf16 row-major with row strides x_ld, y_ld; C fp32 (ldc),
+// which the caller zeroes (the K range is split across CTAs, reduced in L2).
+ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const void* x_lo, int64_t x_ld,
+                               const void* y_hi, const void* y_lo, int64_t y_ld, float* c, int64_t ldc,
+                               cudaStream_t stream) {
+  using namespace gemm;
+  constexpr int BN = 128;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  CUtensorMap xh, xl, yh, yl;
+  if (!encode_map_bf16_2d(&xh, x_hi, D, D, x_ld * 2, 64, 64) || !encode_map_bf16_2d(&xl, x_lo, D, D, x_ld * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&yh, y_hi, N, D, y_ld * 2, 64, 64) || !encode_map_bf16_2d(&yl, y_lo, N, D, y_ld * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  p.a_map[0] = xh, p.a_map[1] = xh, p.a_map[2] = xl;
+  p.b_map[0][0] = yh, p.b_map[0][1] = yl, p.b_map[0][2] = yh;
+  for (int q = 0; q < 3; ++q) p.b_map[1][q] = p.b_map[0][q];
+  p.n_pairs = 3;
+  p.a_upper = 1;
+  p.c[0] = c;
+  p.c[1] = c;
+  p.ldc = ldc;
+  p.M = (int32_t)D;
+  p.N = (int32_t)N;
+  p.K = (int32_t)D;
+  p.n_split = (int32_t)N;
+  p.n_cols[0] = (int32_t)N;
+  p.mode = kReduceF32;
+  if (!encode_map_out_2d(&p.c_map[0], c, true, N, D, ldc * 4)) return ISPA_ERR_CUDA;
+  p.c_map[1] = p.c_map[0];
+  p.c_tma = 1;
+  // two K halves per tile: the 6 x 12 tiles of D = 1536 then fill the GPU
+  const int64_t k_blocks = (D + kBK - 1) / kBK;
+  const int64_t per = (k_blocks + 1) / 2;
+  p.k_per_split = (int32_t)(per * kBK);
+  return launch<true, true, BN, 4>(p, (int)((k_blocks + per - 1) / per), stream);
+}
+
+// C[M, N] += (a_hi + a_lo) W, W exactly bf16 [K, N] row-major; a_hi / a_lo
+// bf16 [M, K] row-major; C fp32 (ldc), zeroed by the caller.  Two K halves
+// per tile, reduced in L2.
+ispa_status_t gemm_hilo_w(int64_t M, int64_t K, const void* a_hi, const void* a_lo, const void* w, int64_t N,
+                          float* c, int64_t ldc, cudaStream_t stream) {
+  using namespace gemm;
+  constexpr int BN = 128;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  if (!encode_map_bf16_2d(&p.a_map[0], a_hi, K, M, K * 2, 64, kBM) ||
+      !encode_map_bf16_2d(&p.a_map[1], a_lo, K, M, K * 2, 64, kBM) ||
+      !encode_map_bf16_2d(&p.b_map[0][0], w, N, K, N * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  p.b_map[0][1] = p.b_map[0][0];
+  p.b_map[1][0] = p.b_map[1][1] = p.b_map[0][0];
+  p.n_pairs = 2;
+  p.c[0] = c;
+  p.c[1] = c;
+  p.ldc = ldc;
+  p.M = (int32_t)M;
+  p.N = (int32_t)N;
+  p.K = (int32_t)K;
+  p.n_split = (int32_t)N;
+  p.n_cols[0] = (int32_t)N;
+  p.mode = kReduceF32;
+  if (!encode_map_out_2d(&p.c_map[0], c, true, N, M, ldc * 4)) return ISPA_ERR_CUDA;
+  p.c_map[1] = p.c_map[0];
+  p.c_tma = 1;
+  const int64_t k_blocks = (K + kBK - 1) / kBK;
+  const int64_t per = (k_blocks + 1) / 2;
+  p.k_per_split = (int32_t)(per * kBK);
+  return launch<false, true, BN, 4>(p, (int)((k_blocks + per - 1) / per), stream);
 }
 
 }  // namespace ispa

@@ -17,7 +17,10 @@ section 2):
     ||A_full W||^2, evaluated from G, R, E without its activations;
   * later chunks (stage 3): selected layers (L-layers) attend to sink +
     current only and project with W_new; the others (F-layers) attend to the
-    whole growing cache and project with W.
+    whole growing cache and project with W.  With ``precision="w8a8"`` the
+    L-layers project with the post-training W8A8 reading of the same page's
+    "Speedup" item: W_new quantised to e4m3 once, after the absorb, and each
+    chunk's A_loc quantised per token.
 Chunk 0 holds the sink frame inside its own current chunk, so it has no
 separate sink and no history.  Every step runs in libispa's kernels; this
 module only owns the device buffers (torch tensors), the chunk schedule and the
@@ -47,13 +50,17 @@ class Rollout:
     def __init__(self, w: synth.Workload, absorbed: Optional[Sequence[int]] = None, device="cuda",
                  lambda_rel: float = 1e-2,
                  on_layer: Optional[Callable[[int, int, dict], None]] = None,
-                 selection: str = "fixed", rank_all: bool = False):
+                 selection: str = "fixed", rank_all: bool = False, precision: str = "bf16"):
         """``absorbed``: the fixed L-layer set (default: even layers); with
         ``selection="instance"`` only its size K is used and the K layers of
         lowest reconstruction error are chosen at the transition.
         ``rank_all``: rank every layer (eps of each) even for a fixed set."""
         if selection not in ("fixed", "instance"):
             raise ValueError("selection must be 'fixed' or 'instance'")
+        if precision not in ("bf16", "w8a8"):
+            raise ValueError("precision must be 'bf16' or 'w8a8'")
+        self.precision = precision
+        self.w8: Dict[int, tuple] = {}  # L-layer -> (e4m3 codes of W_new, transposed; per-channel scales)
         self.w = w
         self.device = torch.device(device)
         self.L = w.n_layers
@@ -101,6 +108,11 @@ class Rollout:
                     "a_delta": torch.empty(n_q, D, **bf), "lse_loc": torch.empty(w.n_heads, n_q, **f32),
                     "lse_full": torch.empty(w.n_heads, n_q, **f32)}
         self.y = torch.empty(n_q, D, **bf)
+        self.w8_out = None
+        if precision == "w8a8":
+            self.w8_out = {"y": self.y, "a_loc": self.out["a_loc"],
+                           "a_codes": torch.empty(n_q, D, dtype=torch.uint8, device=self.device),
+                           "a_scales": torch.empty(n_q, dtype=torch.float32, device=self.device)}
         self.status = ispa.new_status(self.device)
         self.workspace = ispa.absorb_workspace(D, self.device)
         self.reports: List[ChunkReport] = []
@@ -190,6 +202,9 @@ class Rollout:
             k_small[:sink].copy_(self.k[l][:sink])
             v_small[:sink].copy_(self.v[l][:sink])
             self.k[l], self.v[l] = k_small, v_small
+        if self.precision == "w8a8":
+            for l in self.absorbed:
+                self.w8[l] = ispa.quantize_e4m3_weight(self.W_new[l])
         torch.cuda.synchronize(self.device)
         if not self.rank:
             self.absorb_ms = [a.elapsed_time(b) for a, b in events]
@@ -210,8 +225,13 @@ class Rollout:
             if self.is_l_layer(l):
                 n_loc = self.w.sink_frames * self.F + self.chunk_tokens
                 local = [(k[:n_loc], v[:n_loc])]
-                y, _ = ispa.local_attention_project(self.q[l], local, self.W_new[l], H, y=self.y,
-                                                    a_loc=self.out["a_loc"], status=self.status)
+                if self.precision == "w8a8":
+                    qwt, sw = self.w8[l]
+                    ispa.local_attention_project_w8a8(self.q[l], local, qwt, sw, H, out=self.w8_out,
+                                                      status=self.status)
+                else:
+                    ispa.local_attention_project(self.q[l], local, self.W_new[l], H, y=self.y,
+                                                 a_loc=self.out["a_loc"], status=self.status)
                 info = {"mode": "L", "local": local, "hist": [], "W": self.W_new[l]}
             else:
                 cb, ce = r["cur"]

@@ -97,10 +97,12 @@ def replica_tflops(flop_per_step: float, steps: int, world: int, t_max_ms: float
 
 
 def absorb_launches(D: int) -> int:
+    """Kernel launches of one tensor-core absorb solve (bf16 W, D % 128 == 0):
+    split of R, [0 | I] fill, S = R W, trace, shift, one panel kernel per
+    64-wide panel, one update product per panel but the last, the split of
+    [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new."""
     nb = D // 64
-    # split of R, two tensor-core products for R W, trace, shift, W_new,
-    # 3nb-2 Cholesky launches and 2(2nb-1) triangular-solve launches
-    return 7 * nb + 2
+    return 5 + nb + (nb - 1) + 3
 
 
 def cores() -> int:
@@ -498,8 +500,31 @@ def run_rollout(device) -> dict:
     }
     del ro
     torch.cuda.empty_cache()
+    res["w8a8"] = run_rollout_w8a8(device, res)
     res["layer_selection"] = run_layer_selection(device)
     return res
+
+
+def run_rollout_w8a8(device, bf16_res: dict) -> dict:
+    """The same rollout with W8A8 L-layers (W_new quantised to e4m3 once after
+    the absorb, A_loc per token every chunk), post-transition chunks timed
+    the same way as the bf16 rollout's."""
+    from ar_video_diffusion_b200.rollout import Rollout
+    w = synth.WORKLOADS["rollout"]
+    ro = Rollout(w, device=device, precision="w8a8")
+    reps = ro.run()
+    post = [r for r in reps if r.phase == "post"]
+    g_first = ro.chunk_graph_ms(w.warm_chunks)
+    g_last = ro.chunk_graph_ms(reps[-1].chunk)
+    if int(ro.status[0].item()) != 0:
+        raise RuntimeError("device status during the W8A8 rollout")
+    del ro
+    torch.cuda.empty_cache()
+    return {"workload": "the rollout above with W8A8 L-layers (e4m3 W_new per output channel, A_loc per token)",
+            "post_chunk_ms_first": round(post[0].gpu_ms, 3), "post_chunk_ms_last": round(post[-1].gpu_ms, 3),
+            "post_chunk_graph_ms_first": round(g_first, 3), "post_chunk_graph_ms_last": round(g_last, 3),
+            "speedup_vs_bf16_graph_first": round(bf16_res["post_chunk_graph_ms_first"] / g_first, 4),
+            "speedup_vs_bf16_graph_last": round(bf16_res["post_chunk_graph_ms_last"] / g_last, 4)}
 
 
 def run_layer_selection(device) -> dict:

@@ -194,8 +194,12 @@ ISPA_API size_t ispa_absorb_workspace_bytes(int64_t d_model);
 /*
  * ispa_absorb_solve -- closed-form weight modulation [gist §2.2, §2.3].
  * lambda = lambda_abs + lambda_rel * trace(G) / d_model (computed on the device);
- * delta_w = (G + lambda I)^-1 R W by a blocked Cholesky factorisation (fp32)
- * and two triangular solves; w_new = W + delta_w rounded to w_dt (nullable).
+ * delta_w = (G + lambda I)^-1 R W by a blocked Cholesky factorisation and
+ * triangular solves; w_new = W + delta_w rounded to w_dt (nullable).  With a
+ * bf16 W and d_model a multiple of 128 (>= 256) the products run on the tensor
+ * cores in split precision (bf16 hi/lo pairs, about 2^-17 relative per
+ * product) and the solves are carried through the factorisation; otherwise
+ * (fp32 W, other sizes) the updates run on the CUDA cores in fp32.
  * G, R fp32 [D, D] (G symmetric; only its lower triangle is read), W and w_new
  * [D, D] in w_dt, delta_w fp32 [D, D].  workspace: device buffer of at least
  * ispa_absorb_workspace_bytes(d_model) bytes, 256-byte aligned.  dev_status
@@ -217,7 +221,9 @@ ISPA_API ispa_status_t ispa_absorb_solve(const float* G, const float* R, const v
  * Here the working matrices live in a device array owned by the library
  * (4 d^2 + 256 d + 256 bytes for d = 2048, about 17.3 MB), which every GPU that
  * loads libispa holds until the process exits.  The caller still passes G, R,
- * W and the outputs, exactly as for ispa_absorb_solve.
+ * W and the outputs, exactly as for ispa_absorb_solve.  To keep the array that
+ * small it always runs the compact form of the solve (fp32 CUDA-core updates),
+ * whose dW agrees with ispa_absorb_solve's within the solve's accuracy.
  *   - d_model must be a multiple of 64 and at most 2048; larger sizes return
  *     ISPA_ERR_UNSUPPORTED without launching.
  *   - No allocation of any kind happens, and nothing needs clearing: each call

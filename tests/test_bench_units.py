@@ -31,10 +31,10 @@ def test_solve_flops_and_launch_count():
     assert bench.solve_flops(D) == pytest.approx(D ** 3 / 3 + 2 * D ** 3 + 2 * D ** 3)
     assert bench.solve_flops(D) == pytest.approx(15.7e9, rel=3e-3)
     nb = D // 64
-    # Cholesky: nb diagonal factorisations, nb-1 panels, nb-1 trailing updates;
-    # two triangular solves: nb diagonal applications and nb-1 updates each;
-    # plus split, two tensor-core products, trace, shift and W_new
-    assert bench.absorb_launches(D) == (3 * nb - 2) + 2 * (2 * nb - 1) + 6 == 170
+    # tensor-core form: split of R, [0 | I] fill, S = R W, trace, shift;
+    # nb panel kernels (each factoring its diagonal block) and nb-1 update
+    # products; the split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new
+    assert bench.absorb_launches(D) == 5 + nb + (nb - 1) + 3 == 55
 
 
 def test_chunk_rooflines_are_the_tensor_time_of_their_contractions():

@@ -191,3 +191,39 @@ def test_full_size_rollout_absorbed_layers_against_the_oracle_chain():
     assert max_rel(x["y"], orc.project(a, W_new_ref)) <= ATTN_MAX_REL
     other = post[1 - chosen]
     assert other["mode"] == "F" and other["k_hist"].shape[0] == (w.warm_chunks * w.chunk_frames - 1) * w.frame_tokens
+
+
+def test_small_rollout_w8a8_l_layers_against_the_oracle_chain():
+    """The small rollout with W8A8 L-layers: after the absorb, W_new is
+    quantised once (e4m3, per output channel) and every post-transition chunk
+    quantises A_loc per token before the e4m3 projection.  Expected values: the
+    oracle's own chain (its dW from its own dual stream over the warm-up rows),
+    then its W8A8 reading of y = A_loc W_new; bounds CHAIN_W8A8_FRO / _MAX
+    (tests/chain_tolerances.py)."""
+    from oracle import w8a8_oracle as w8
+    from helpers import CHAIN_W8A8_FRO, CHAIN_W8A8_MAX
+    w = synth.WORKLOADS["rollout_small"]
+    absorbed = [0, 2]
+    inputs = {}
+    ro = Rollout(w, absorbed=absorbed, on_layer=capture_inputs(w, inputs), precision="w8a8")
+    reports = ro.run()
+    _check_bookkeeping(w, ro, reports, absorbed)
+    W = {l: host(ro.W[l]) for l in range(w.n_layers)}
+    W_new_ref = {}
+    for l in absorbed:
+        a_loc, a_full = oracle_rollout_statistics(w, inputs, l)
+        G, R = orc.gram(a_loc, a_full - a_loc)
+        dW_ref = orc.absorb(G, R, W[l], orc.ridge_lambda(G))
+        W_new_ref[l] = synth.round_bf16(orc.modulated_weight(W[l], dW_ref).astype(np.float32))
+    n_l = 0
+    for (l, c), x in sorted(inputs.items()):
+        if x["mode"] != "L":
+            continue
+        n_l += 1
+        a, _ = orc.attention(x["q"], x["k_loc"], x["v_loc"], w.n_heads)
+        y_ref = w8.project_w8a8(synth.round_bf16(a.astype(np.float32)), W_new_ref[l])
+        err = fro_rel(x["y"], y_ref)
+        REPORT.append((f"small rollout W8A8 chain: y of layer {l} chunk {c} (relative Frobenius)", err, err))
+        assert err <= CHAIN_W8A8_FRO, (l, c, err)
+        assert np.max(np.abs(x["y"] - y_ref)) <= CHAIN_W8A8_MAX * np.max(np.abs(y_ref)), (l, c)
+    assert n_l == len(absorbed) * w.post_chunks
