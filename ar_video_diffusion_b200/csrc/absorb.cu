@@ -518,6 +518,27 @@ __device__ __forceinline__ void split_store(float v, __nv_bfloat16* hi, __nv_bfl
   lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+// 16 consecutive values (times `sign`) as bf16 hi and lo halves, two 16-byte
+// stores each (hi and lo 32-byte aligned)
+__device__ __forceinline__ void split_store16(const float (&v)[16], float sign, __nv_bfloat16* hi,
+                                              __nv_bfloat16* lo) {
+  uint32_t h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float a = sign * v[2 * e], b = sign * v[2 * e + 1];
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(a - __low2float(hh), b - __high2float(hh));
+    h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[e] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  uint4* h4 = reinterpret_cast<uint4*>(hi);
+  uint4* l4 = reinterpret_cast<uint4*>(lo);
+  h4[0] = make_uint4(h[0], h[1], h[2], h[3]);
+  h4[1] = make_uint4(h[4], h[5], h[6], h[7]);
+  l4[0] = make_uint4(l[0], l[1], l[2], l[3]);
+  l4[1] = make_uint4(l[4], l[5], l[6], l[7]);
+}
+
 // Panel k, with the factorisation of its diagonal block.  Every CTA factors
 // the 64 x 64 diagonal block of M itself (it is small, and the copies run in
 // parallel, so no separate launch or global round trip sits on the chain;
@@ -568,32 +589,39 @@ __global__ void __launch_bounds__(256) panel_factor_kernel(float* M, int D, int 
   __syncthreads();
   const int tx = tid & 15, ty = tid >> 4;
   float acc[4][4];
-  if (row_block) {
+  if (row_block)
     mm64(A, X, false, true, acc);  // A_rk L_kk^-T
-    float* blk = M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)k * kT;
-    const int64_t row0 = (int64_t)blockIdx.x * kT;  // local row of the trailing block
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int i = ty + 16 * a, j = tx + 16 * b;
-        const float v = acc[a][b];
-        blk[(int64_t)i * D + j] = v;
-        split_store(-v, a_hi, a_lo, (row0 + i) * 64 + j);
-        split_store(v, lt_hi, lt_lo, (int64_t)j * ld_t + row0 + i);
-      }
-  } else {
+  else
     mm64(X, A, false, false, acc);  // L_kk^-1 RHS_k
-    float* blk = RHS + (int64_t)k * kT * rhs_ld + c0;
+  __syncthreads();
+  // the 64 x 64 result through shared memory, so that every global store
+  // below is a 16-byte vector of one row
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int i = ty + 16 * a, j = tx + 16 * b;
-        if (c0 + j >= rhs_cols) continue;
-        blk[(int64_t)i * rhs_ld + j] = acc[a][b];
-        split_store(acc[a][b], y_hi, y_lo, (int64_t)i * ld_y + c0 + j);
-      }
+    for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] = acc[a][b];
+  __syncthreads();
+  const int ri = tid >> 2, c16 = (tid & 3) * 16;  // this thread: row (or column) ri, 16 values from c16
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = A[ri][c16 + e];
+  if (row_block) {
+    const int64_t row0 = (int64_t)blockIdx.x * kT;  // local row of the trailing block
+    float4* dst = reinterpret_cast<float4*>(M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)ri * D +
+                                            (int64_t)k * kT + c16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    split_store16(v, -1.f, a_hi + (row0 + ri) * 64 + c16, a_lo + (row0 + ri) * 64 + c16);
+    // L21^T: row ri of the transpose is column ri of the block
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = A[c16 + e][ri];
+    split_store16(v, 1.f, lt_hi + (int64_t)ri * ld_t + row0 + c16, lt_lo + (int64_t)ri * ld_t + row0 + c16);
+  } else {
+    // rhs_cols and c0 are multiples of 64: the block lies wholly inside
+    float4* dst = reinterpret_cast<float4*>(RHS + (int64_t)k * kT * rhs_ld + (int64_t)ri * rhs_ld + c0 + c16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    split_store16(v, 1.f, y_hi + (int64_t)ri * ld_y + c0 + c16, y_lo + (int64_t)ri * ld_y + c0 + c16);
   }
 }
 

@@ -12,19 +12,19 @@
 //   warps 0, 3  TMA producers: Q and the K tiles (warp 0), the V tiles
 //               (warp 3), each into its own NST-stage ring (a K tile is
 //               released once S(j) is done, a V tile after PV(j));
-//   warp 1      tcgen05 issuer, the whole warp converged, one elected lane
-//               issuing: S(j) = Q K(j)^T (both operands K-major in shared
-//               memory) and O += P(j) V(j) (P from tensor memory, V MN-major
-//               in shared memory);
-//   warp 2      allocates / frees the 512 tensor-memory columns;
+//   warps 1, 2  tcgen05 issuers, each converged with one elected lane
+//               issuing: warp 2 S(j) = Q K(j)^T (both operands K-major in
+//               shared memory), warp 1 O += P(j) V(j) (P from tensor memory,
+//               V MN-major in shared memory); warp 2 also allocates and frees
+//               the 512 tensor-memory columns;
 //   warps 4-11  softmax: two warpgroups; warpgroup w takes the key tiles
 //               j = w mod 2; thread = query row = TMEM lane.
 // Tensor memory: three S buffers (tile j uses buffer j mod 3) and ONE O
 // accumulator (head_dim columns) that both warpgroups' products add into.
-// With three S buffers, S(j+3) is issued right after PV(j) (the product that
-// reads P(j) out of the same columns), so a warpgroup's next S is computed
-// while it is still exponentiating: the tensor core runs PV(j), S(j+3) while
-// the softmax of tile j+1 runs, and neither waits for the other's chain.
+// With three S buffers, S(j+3) is issued as soon as PV(j) (the product that
+// reads P(j) out of the same columns) has completed, so a warpgroup's next S
+// is computed while it is still exponentiating, and the two issuers keep the
+// tensor core fed independently.
 // Online softmax in the log2 domain with one running maximum per row shared
 // by the two warpgroups: the warpgroup of tile j reads the maximum m(j-1)
 // that tile j-1 used (a per-row value in shared memory, published through one
@@ -97,8 +97,8 @@ struct Layout {
   static constexpr int kMref = kXs + 2 * kBM * 4;     // the shared running maximum, one float per row
   static constexpr int kBars = kMref + kBM * 4;
   // kv_full, kv_empty, v_full, v_empty [NST]; q_full; s_full, p_full, pv_done [3]; mref_full[4];
-  // ck_ready, ck_done, fin_ready; xsum[3]; teardown
-  static constexpr int kNumBars = 4 * NST + 1 + 3 * kNS + 4 + 3 + 3 + 1;
+  // ck_ready, ck_done, fin_ready; xsum[3]; teardown[2]
+  static constexpr int kNumBars = 4 * NST + 1 + 3 * kNS + 4 + 3 + 3 + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -207,44 +207,63 @@ struct Bars {
   __device__ __forceinline__ uint64_t* ck_done() const { return base + 4 * NST + 15; }
   __device__ __forceinline__ uint64_t* fin_ready() const { return base + 4 * NST + 16; }
   __device__ __forceinline__ uint64_t* xsum(int k) const { return base + 4 * NST + 17 + k; }
-  __device__ __forceinline__ uint64_t* teardown() const { return base + 4 * NST + 20; }
-  static constexpr int kCount = 4 * NST + 21;
+  __device__ __forceinline__ uint64_t* teardown(int w) const { return base + 4 * NST + 20 + w; }  // per issuer
+  static constexpr int kCount = 4 * NST + 22;
 };
 
+// Two issuing warps, each converged with one elected lane issuing:
+//   warp 2 issues S(j) = Q K(j)^T into S buffer j mod 3 once K(j) has arrived
+//   and PV(j - 3) -- the product that reads P(j - 3) out of that buffer -- has
+//   completed;
+//   warp 1 issues O += P(i) V(i) in tile order once P(i) and V(i) are there.
+// Each waits only for its own operands, so the tensor core is fed from one
+// while the other waits (a single issuer interleaving both spent a third of
+// every tile period in waits while the MMA queue ran dry).
 template <int HD, int NST>
-__device__ void mma_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, volatile int* abort_flag, uint32_t tmem) {
+__device__ void s_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, volatile int* abort_flag, uint32_t tmem) {
   using L = Layout<HD, NST>;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false, false);
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
-  const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-  const int T = p.n_tiles, n_loc = p.n_local_tiles;
-  const bool ck = p.dual && n_loc > 0 && n_loc < T;  // a local result is taken between the tiles
-
-  // the whole warp runs the loop and every wait; the elected lane issues
+  const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK);
+  const int T = p.n_tiles;
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
   };
-  auto issue_s = [&](int j) -> bool {
-    const int stage = j % NST;
-    if (!wait(B.kv_full(stage), (j / NST) & 1)) return false;
+  bool ok = wait(B.q_full(), 0);
+  for (int j = 0; ok && j < T; ++j) {
+    const int stage = j % NST, b = j % kNS;
+    // buffer b still holds P(j - 3) until PV(j - 3) has completed
+    if (j >= kNS && !(ok = wait(B.pv_done(b), ((j - kNS) / kNS) & 1))) break;
+    if (!(ok = wait(B.kv_full(stage), (j / NST) & 1))) break;
     tc_fence_after();
     const uint32_t kb = sK + stage * L::kTileBytes;
-    const uint32_t d = tmem + kTmS + (j % kNS) * 128;
+    const uint32_t d = tmem + kTmS + b * 128;
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
       umma_ss_warp(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
                    kk > 0 ? 1u : 0u);
     }
-    umma_commit_warp(B.s_full(j % kNS));
+    umma_commit_warp(B.s_full(b));
     umma_commit_warp(B.kv_empty(stage));
-    return true;
-  };
+  }
+  // every MMA must have completed before tensor memory is released
+  umma_commit_warp(B.teardown(1));
+  mbar_wait_drain(B.teardown(1), 0, 100000000ull);
+  __syncwarp();
+}
 
-  bool ok = wait(B.q_full(), 0);
-  tc_fence_after();
-  for (int j = 0; ok && j < kNS && j < T; ++j) ok = issue_s(j);
-  for (int i = 0; ok && i < T; ++i) {
+template <int HD, int NST>
+__device__ void pv_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, volatile int* abort_flag,
+                          uint32_t tmem) {
+  using L = Layout<HD, NST>;
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, false, true);
+  const uint32_t sV = smem_u32(smem + L::kV);
+  const int T = p.n_tiles, n_loc = p.n_local_tiles;
+  const bool ck = p.dual && n_loc > 0 && n_loc < T;  // a local result is taken between the tiles
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+  };
+  for (int i = 0; i < T; ++i) {
     const int b = i % kNS;
     const bool first_hist = ck && i == n_loc;
     const bool fresh = i == 0 || first_hist;
@@ -256,7 +275,7 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, v
     const uint32_t pb = tmem + kTmS + b * 128;
     if (!wait(B.v_full(stage), (i / NST) & 1)) break;
     // p_full[b] completes once per use of buffer b; its next phase needs
-    // S(i + 3), issued below, so the parity is unambiguous
+    // S(i + 3), which waits for PV(i), so the parity is unambiguous
     if (!wait(B.p_full(b), (i / kNS) & 1)) break;
     tc_fence_after();
     // O += P V: P (bf16, 128 keys) in the first 64 columns of S buffer b
@@ -268,11 +287,10 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, v
     umma_commit_warp(B.pv_done(b));
     if (ck && i == n_loc - 1) umma_commit_warp(B.ck_ready());
     if (i == T - 1) umma_commit_warp(B.fin_ready());
-    if (i + kNS < T) ok = issue_s(i + kNS);
   }
   // every MMA must have completed before tensor memory is released
-  umma_commit_warp(B.teardown());
-  mbar_wait_drain(B.teardown(), 0, 100000000ull);
+  umma_commit_warp(B.teardown(0));
+  mbar_wait_drain(B.teardown(0), 0, 100000000ull);
   __syncwarp();
 }
 
@@ -574,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
     mbar_init(B.xsum(0), 128);
     mbar_init(B.xsum(1), 128);
     mbar_init(B.xsum(2), 256);
-    mbar_init(B.teardown(), 1);
+    mbar_init(B.teardown(0), 1);
+    mbar_init(B.teardown(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -598,7 +617,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
     if (warp == 0) {
       if (lane == 0) producer<HD, NST>(p, smem, false, B.q_full(), B.kv_full(0), B.kv_empty(0), abort_flag, q0, head);
     } else if (warp == 1) {
-      mma_issuer<HD, NST>(p, smem, B, abort_flag, tmem);
+      pv_issuer<HD, NST>(p, smem, B, abort_flag, tmem);
+    } else if (warp == 2) {
+      s_issuer<HD, NST>(p, smem, B, abort_flag, tmem);
     } else if (warp == 3) {
       if (lane == 0) producer<HD, NST>(p, smem, true, nullptr, B.v_full(0), B.v_empty(0), abort_flag, q0, head);
     }
