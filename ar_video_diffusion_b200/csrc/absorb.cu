@@ -398,13 +398,15 @@ __global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ 
 namespace simt {
 
 // 32 x 32 Cholesky factor of a lower triangle in shared memory (row stride
-// ld), by one warp: lane r holds row r in registers with the columns rotated
+// ld), by one warp.  Lane r holds row r in registers with the columns rotated
 // (a[0] is the current column), so the loop body is short and its register
-// indices static; the loop itself stays rolled, keeping the code small enough
-// for the instruction cache (an unrolled factorisation run once by one warp is
-// bound by instruction fetch).  L is written over the lower triangle.  A pivot
-// <= 0 or non-finite is replaced by 1 and its index (first only) recorded.
-__device__ __forceinline__ void chol32_rot(float* A, int ld, int lane, int base, int* bad) {
+// indices static, and the loop stays rolled (an unrolled factorisation run
+// once by one warp is bound by instruction fetch).  Column j of L goes to the
+// lower triangle of A and, shifted, to row j of Ls (Ls[j][c] = L[j + c][j],
+// zero beyond the matrix), so the column is read back as eight 16-byte
+// vectors instead of 31 shuffles.  A pivot <= 0 or non-finite is replaced by
+// 1 and its index (first only) recorded.
+__device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], int lane, int base, int* bad) {
   float a[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) a[c] = c <= lane ? A[lane * ld + c] : 0.f;
@@ -418,32 +420,43 @@ __device__ __forceinline__ void chol32_rot(float* A, int ld, int lane, int base,
     const float ljj = sqrtf(d);
     const float l = lane == j ? ljj : (lane > j ? a[0] / ljj : 0.f);
     if (lane >= j) A[lane * ld + j] = l;
-    // a[c] holds column j + c: subtract l * L[j + c][j] (lane j + c's l)
+    Ls[j][(lane - j) & 31] = lane >= j ? l : 0.f;  // lanes < j zero the tail
+    __syncwarp();
+    const float4* col = reinterpret_cast<const float4*>(Ls[j]);
+    float lk[32];
 #pragma unroll
-    for (int c = 1; c < 32; ++c) {
-      const float lk = __shfl_sync(0xffffffffu, l, (j + c) & 31);
-      a[c - 1] = a[c] - l * lk;
+    for (int q = 0; q < 8; ++q) {
+      const float4 v = col[q];
+      lk[4 * q] = v.x, lk[4 * q + 1] = v.y, lk[4 * q + 2] = v.z, lk[4 * q + 3] = v.w;
     }
+    // a[c] holds column j + c: subtract l * L[j + c][j]
+#pragma unroll
+    for (int c = 1; c < 32; ++c) a[c - 1] = a[c] - l * lk[c];
     a[31] = 0.f;
   }
 }
 
-// Column `lane` of X = L^-1 for the 32 x 32 lower-triangular L in shared memory
-// (row stride ld), by one warp, column-oriented forward elimination with the
-// right-hand side rotated in registers; X[m][lane] written with row stride ldx.
-__device__ __forceinline__ void inv32_rot(const float* L, int ld, float* X, int ldx, int lane) {
+// Column `lane` of X = L^-1 for the 32 x 32 lower-triangular L whose columns
+// chol32_rot left shifted in Ls, by one warp: column-oriented forward
+// elimination with the right-hand side rotated in registers; X[m][lane]
+// written with row stride ldx.
+__device__ __forceinline__ void inv32_rot(const float (*Ls)[32], float* X, int ldx, int lane) {
   float b[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
 #pragma unroll 1
   for (int m = 0; m < 32; ++m) {
-    const float x = b[0] / L[m * ld + m];
+    const float4* col = reinterpret_cast<const float4*>(Ls[m]);
+    float lr[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 v = col[q];
+      lr[4 * q] = v.x, lr[4 * q + 1] = v.y, lr[4 * q + 2] = v.z, lr[4 * q + 3] = v.w;
+    }
+    const float x = b[0] / lr[0];  // lr[0] = L[m][m]
     X[m * ldx + lane] = x;
 #pragma unroll
-    for (int c = 1; c < 32; ++c) {
-      const float lr = m + c < 32 ? L[(m + c) * ld + m] : 0.f;
-      b[c - 1] = b[c] - lr * x;
-    }
+    for (int c = 1; c < 32; ++c) b[c - 1] = b[c] - lr[c] * x;
     b[31] = 0.f;
   }
 }
@@ -452,16 +465,21 @@ __device__ __forceinline__ void inv32_rot(const float* L, int ld, float* X, int 
 // triangle used) and the inverse X of that factor (shared, row stride 65),
 // by the 256 threads of a CTA: L11 = chol(A11) and X11 by warp 0,
 // L21 = A21 X11^T, A22 - L21 L21^T, L22 = chol(.) and X22 by warp 0,
-// X21 = -X22 (L21 X11).  T: 32 x 33 scratch.
-__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], int* bad, int base) {
+// X21 = -X22 (L21 X11).  T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned.
+__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], float (*Ls)[32], int* bad,
+                              int base) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // element (i, j) of a 32 x 32 product: i = tid / 8, j = tid % 8 + 8 b
   const int pi = tid >> 3, pj = tid & 7;
-  for (int e = tid; e < 64 * 65; e += 256) (&X[0][0])[e] = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {  // the upper right quarter of X is zero
+    const int e = tid + 256 * q;
+    X[e >> 5][32 + (e & 31)] = 0.f;
+  }
   if (warp == 0) {
-    chol32_rot(&A[0][0], 65, lane, base, bad);
+    chol32_rot(&A[0][0], 65, Ls, lane, base, bad);
     __syncwarp();
-    inv32_rot(&A[0][0], 65, &X[0][0], 65, lane);
+    inv32_rot(Ls, &X[0][0], 65, lane);
   }
   __syncthreads();
   float acc[4];
@@ -487,9 +505,9 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], in
   }
   __syncthreads();
   if (warp == 0) {
-    chol32_rot(&A[32][32], 65, lane, base + 32, bad);
+    chol32_rot(&A[32][32], 65, Ls, lane, base + 32, bad);
     __syncwarp();
-    inv32_rot(&A[32][32], 65, &X[32][32], 65, lane);
+    inv32_rot(Ls, &X[32][32], 65, lane);
   }
   __syncthreads();
 #pragma unroll
@@ -560,6 +578,7 @@ __global__ void __launch_bounds__(256) panel_factor_kernel(float* M, int D, int 
   __shared__ float A[kT][kT + 1];  // the diagonal block, then this CTA's block
   __shared__ float X[kT][kT + 1];  // L_kk^-1
   __shared__ float T[32][33];
+  __shared__ __align__(16) float Ls[32][32];
   __shared__ int bad;
   const int tid = threadIdx.x;
   const bool row_block = (int)blockIdx.x < rest;
@@ -574,10 +593,20 @@ __global__ void __launch_bounds__(256) panel_factor_kernel(float* M, int D, int 
     pre[q] = (row_block || c0 + j < rhs_cols) ? own[(int64_t)i * own_ld + j] : 0.f;
   }
   const float* dblk = M + (int64_t)k * kT * D + (int64_t)k * kT;
-  for (int e = tid; e < kT * kT; e += 256) A[e >> 6][e & 63] = dblk[(int64_t)(e >> 6) * D + (e & 63)];
+  float dg[16];  // all loads in flight before the first use
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    dg[q] = dblk[(int64_t)(e >> 6) * D + (e & 63)];
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    A[e >> 6][e & 63] = dg[q];
+  }
   if (tid == 0) bad = -1;
   __syncthreads();
-  factor_diag64(A, X, T, &bad, k * kT);
+  factor_diag64(A, X, T, Ls, &bad, k * kT);
   if (blockIdx.x == 0 && tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
   }
@@ -640,17 +669,24 @@ __global__ void init_rhs_kernel(float* __restrict__ RHS, int D) {
   }
 }
 
-// [Y | X] (D x 2D fp32) -> hi/lo of Y and of X, each D x D bf16
+// [Y | X] (D x 2D fp32) -> hi/lo of Y and of X, each D x D bf16; four
+// elements per thread and step (16-byte loads, 8-byte stores)
 __global__ void split_rhs_kernel(const float* __restrict__ RHS, int D, __nv_bfloat16* __restrict__ yh,
                                  __nv_bfloat16* __restrict__ yl, __nv_bfloat16* __restrict__ xh,
                                  __nv_bfloat16* __restrict__ xl) {
-  const int64_t n = (int64_t)D * 2 * D;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t i = e / (2 * D), j = e % (2 * D);
-    if (j < D)
-      split_store(RHS[e], yh, yl, i * D + j);
-    else
-      split_store(RHS[e], xh, xl, i * D + j - D);
+  const int64_t n4 = (int64_t)D * 2 * D / 4;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(RHS)[e];
+    const int64_t i = (e * 4) / (2 * D), j = (e * 4) % (2 * D);  // j multiple of 4: never straddles D
+    __nv_bfloat16* hi = j < D ? yh + i * D + j : xh + i * D + j - D;
+    __nv_bfloat16* lo = j < D ? yl + i * D + j : xl + i * D + j - D;
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
+    const __nv_bfloat162 l0 = __floats2bfloat162_rn(v.x - __low2float(h0), v.y - __high2float(h0));
+    const __nv_bfloat162 l1 = __floats2bfloat162_rn(v.z - __low2float(h1), v.w - __high2float(h1));
+    *reinterpret_cast<uint2*>(hi) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+    *reinterpret_cast<uint2*>(lo) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
   }
 }
 
