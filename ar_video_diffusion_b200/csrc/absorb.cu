@@ -21,7 +21,10 @@
 // solves L Y = S, L^T X = Y.  Its fp32 GEMM (also the fp32 activation path of
 // the statistics and the projection) is a 64 x 64-tile CUDA-core kernel with
 // arbitrary strides, so transposed operands are read in place.
+#include <cudaTypedefs.h>
+
 #include <cstring>
+#include <vector>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -403,23 +406,30 @@ namespace simt {
 // indices static, and the loop stays rolled (an unrolled factorisation run
 // once by one warp is bound by instruction fetch).  Column j of L goes to the
 // lower triangle of A and, shifted, to row j of Ls (Ls[j][c] = L[j + c][j],
-// zero beyond the matrix), so the column is read back as eight 16-byte
-// vectors instead of 31 shuffles.  A pivot <= 0 or non-finite is replaced by
-// 1 and its index (first only) recorded.
-__device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], int lane, int base, int* bad) {
+// zero beyond the matrix), read back as eight 16-byte vectors for the update
+// of the remaining columns.  The next pivot does not wait for that round
+// trip: lane j + 1 updates its own diagonal entry with its own l and passes it
+// on with one shuffle, so the chain per column is shuffle, reciprocal square
+// root, two multiply-adds.  rinv[j] = 1 / L[j][j].  A pivot <= 0 or
+// non-finite is replaced by 1 and its index (first only) recorded.
+__device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], float* rinv, int lane, int base,
+                                           int* bad) {
   float a[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) a[c] = c <= lane ? A[lane * ld + c] : 0.f;
+  float d = __shfl_sync(0xffffffffu, a[0], 0);
 #pragma unroll 1
   for (int j = 0; j < 32; ++j) {
-    float d = __shfl_sync(0xffffffffu, a[0], j);
     if (!(d > 0.f) || !isfinite(d)) {
       if (lane == 0 && *bad < 0) *bad = base + j;
       d = 1.f;
     }
-    const float ljj = sqrtf(d);
-    const float l = lane == j ? ljj : (lane > j ? a[0] / ljj : 0.f);
+    const float r = rsqrtf(d);
+    const float l = lane == j ? d * r : (lane > j ? a[0] * r : 0.f);
+    // the next pivot: lane j + 1's entry (j + 1, j + 1) less its own l squared
+    const float dn = __shfl_sync(0xffffffffu, a[1] - l * l, (j + 1) & 31);
     if (lane >= j) A[lane * ld + j] = l;
+    if (lane == 0) rinv[j] = r;
     Ls[j][(lane - j) & 31] = lane >= j ? l : 0.f;  // lanes < j zero the tail
     __syncwarp();
     const float4* col = reinterpret_cast<const float4*>(Ls[j]);
@@ -433,14 +443,15 @@ __device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], in
 #pragma unroll
     for (int c = 1; c < 32; ++c) a[c - 1] = a[c] - l * lk[c];
     a[31] = 0.f;
+    d = dn;
   }
 }
 
 // Column `lane` of X = L^-1 for the 32 x 32 lower-triangular L whose columns
-// chol32_rot left shifted in Ls, by one warp: column-oriented forward
-// elimination with the right-hand side rotated in registers; X[m][lane]
-// written with row stride ldx.
-__device__ __forceinline__ void inv32_rot(const float (*Ls)[32], float* X, int ldx, int lane) {
+// chol32_rot left shifted in Ls (rinv: reciprocals of its diagonal), by one
+// warp: column-oriented forward elimination with the right-hand side rotated
+// in registers; X[m][lane] written with row stride ldx.
+__device__ __forceinline__ void inv32_rot(const float (*Ls)[32], const float* rinv, float* X, int ldx, int lane) {
   float b[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
@@ -453,7 +464,7 @@ __device__ __forceinline__ void inv32_rot(const float (*Ls)[32], float* X, int l
       const float4 v = col[q];
       lr[4 * q] = v.x, lr[4 * q + 1] = v.y, lr[4 * q + 2] = v.z, lr[4 * q + 3] = v.w;
     }
-    const float x = b[0] / lr[0];  // lr[0] = L[m][m]
+    const float x = b[0] * rinv[m];
     X[m * ldx + lane] = x;
 #pragma unroll
     for (int c = 1; c < 32; ++c) b[c - 1] = b[c] - lr[c] * x;
@@ -465,9 +476,10 @@ __device__ __forceinline__ void inv32_rot(const float (*Ls)[32], float* X, int l
 // triangle used) and the inverse X of that factor (shared, row stride 65),
 // by the 256 threads of a CTA: L11 = chol(A11) and X11 by warp 0,
 // L21 = A21 X11^T, A22 - L21 L21^T, L22 = chol(.) and X22 by warp 0,
-// X21 = -X22 (L21 X11).  T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned.
-__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], float (*Ls)[32], int* bad,
-                              int base) {
+// X21 = -X22 (L21 X11).  T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned;
+// rinv: 32 floats.
+__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], float (*Ls)[32], float* rinv,
+                              int* bad, int base) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // element (i, j) of a 32 x 32 product: i = tid / 8, j = tid % 8 + 8 b
   const int pi = tid >> 3, pj = tid & 7;
@@ -477,9 +489,9 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
     X[e >> 5][32 + (e & 31)] = 0.f;
   }
   if (warp == 0) {
-    chol32_rot(&A[0][0], 65, Ls, lane, base, bad);
+    chol32_rot(&A[0][0], 65, Ls, rinv, lane, base, bad);
     __syncwarp();
-    inv32_rot(Ls, &X[0][0], 65, lane);
+    inv32_rot(Ls, rinv, &X[0][0], 65, lane);
   }
   __syncthreads();
   float acc[4];
@@ -505,9 +517,9 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
   }
   __syncthreads();
   if (warp == 0) {
-    chol32_rot(&A[32][32], 65, Ls, lane, base + 32, bad);
+    chol32_rot(&A[32][32], 65, Ls, rinv, lane, base + 32, bad);
     __syncwarp();
-    inv32_rot(Ls, &X[32][32], 65, lane);
+    inv32_rot(Ls, rinv, &X[32][32], 65, lane);
   }
   __syncthreads();
 #pragma unroll
@@ -557,63 +569,105 @@ __device__ __forceinline__ void split_store16(const float (&v)[16], float sign, 
   l4[1] = make_uint4(l[4], l[5], l[6], l[7]);
 }
 
-// Panel k, with the factorisation of its diagonal block.  Every CTA factors
-// the 64 x 64 diagonal block of M itself (it is small, and the copies run in
-// parallel, so no separate launch or global round trip sits on the chain;
-// CTA 0 records a bad pivot).  Then:
+// Factorisation of diagonal block k (one CTA): the block is Dsrc (row stride
+// ld_src) minus Lrow Lrow^T when Lrow (the 64 x 64 block of L to its left in
+// the same block row, row stride D) is given -- the last trailing update,
+// applied here so that the factorisation of block k + 1 can run beside the
+// update product of panel k; the inverse of its Cholesky factor goes to
+// Linv (64 x 64 row-major).  A bad pivot records ISPA_ERR_NOT_SPD and its row.
+__global__ void __launch_bounds__(256) diag_factor_kernel(const float* __restrict__ Dsrc, int64_t ld_src,
+                                                          const float* __restrict__ Lrow, int D, int k,
+                                                          float* __restrict__ Linv, int32_t* status) {
+  __shared__ float A[kT][kT + 1];
+  __shared__ float X[kT][kT + 1];
+  __shared__ float T[32][33];
+  __shared__ __align__(16) float Ls[32][32];
+  __shared__ float rinv[32];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  float dg[16], lr[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    dg[q] = Dsrc[(int64_t)(e >> 6) * ld_src + (e & 63)];
+    lr[q] = Lrow ? Lrow[(int64_t)(e >> 6) * D + (e & 63)] : 0.f;
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    A[e >> 6][e & 63] = dg[q];
+    X[e >> 6][e & 63] = lr[q];
+  }
+  if (tid == 0) bad = -1;
+  __syncthreads();
+  if (Lrow) {  // A -= Lrow Lrow^T
+    float acc[4][4];
+    mm64(X, X, false, true, acc);
+    __syncthreads();
+    const int tx = tid & 15, ty = tid >> 4;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] -= acc[a][b];
+    __syncthreads();
+  }
+  factor_diag64(A, X, T, Ls, rinv, &bad, k * kT);
+  if (tid == 0 && bad >= 0 && status) {
+    if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = tid + 256 * q;
+    Linv[e] = X[e >> 6][e & 63];
+  }
+}
+
+// Panel k with L_kk^-1 given (Linv, from diag_factor_kernel):
 //   blocks [0, rest): one 64-row block r below the diagonal,
 //     L_rk = A_rk L_kk^-T, written back to M, plus its split operands: -hi/-lo
 //     as K-major [rows, 64] (a_hi, a_lo, local row index) and hi/lo
-//     transposed as [64, ld_t] (lt_hi, lt_lo);
+//     transposed as [64, ld_t] (lt_hi, lt_lo); block 0 (row block k + 1)
+//     also copies the diagonal block (k + 1, k + 1), as the earlier updates
+//     left it, to dnext before the update product of this panel changes it;
 //   blocks [rest, rest + ncb): one 64-column block of the panel's
 //     right-hand-side rows, Y = L_kk^-1 RHS_k, written back to RHS, plus hi/lo
 //     [64, ld_y] (y_hi, y_lo).
-// Each CTA loads its own block into registers before the factorisation, so
-// the load overlaps it.
-__global__ void __launch_bounds__(256) panel_factor_kernel(float* M, int D, int k, int rest, float* RHS,
-                                                           int64_t rhs_ld, int rhs_cols, __nv_bfloat16* a_hi,
-                                                           __nv_bfloat16* a_lo, __nv_bfloat16* lt_hi,
-                                                           __nv_bfloat16* lt_lo, int64_t ld_t, __nv_bfloat16* y_hi,
-                                                           __nv_bfloat16* y_lo, int64_t ld_y, int32_t* status) {
-  __shared__ float A[kT][kT + 1];  // the diagonal block, then this CTA's block
+__global__ void __launch_bounds__(256) panel_apply_kernel(float* M, int D, int k, int rest, const float* __restrict__ Linv,
+                                                          float* __restrict__ dnext, float* RHS, int64_t rhs_ld,
+                                                          int rhs_cols, __nv_bfloat16* a_hi, __nv_bfloat16* a_lo,
+                                                          __nv_bfloat16* lt_hi, __nv_bfloat16* lt_lo, int64_t ld_t,
+                                                          __nv_bfloat16* y_hi, __nv_bfloat16* y_lo, int64_t ld_y) {
+  __shared__ float A[kT][kT + 1];  // this CTA's block, then its result
   __shared__ float X[kT][kT + 1];  // L_kk^-1
-  __shared__ float T[32][33];
-  __shared__ __align__(16) float Ls[32][32];
-  __shared__ int bad;
   const int tid = threadIdx.x;
   const bool row_block = (int)blockIdx.x < rest;
   const int c0 = row_block ? 0 : ((int)blockIdx.x - rest) * kT;
   const float* own = row_block ? M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)k * kT
                                : RHS + (int64_t)k * kT * rhs_ld + c0;
   const int64_t own_ld = row_block ? D : rhs_ld;
-  float pre[16];
+  float pre[16], li[16];
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const int e = tid + 256 * q, i = e >> 6, j = e & 63;
-    pre[q] = (row_block || c0 + j < rhs_cols) ? own[(int64_t)i * own_ld + j] : 0.f;
+    pre[q] = own[(int64_t)i * own_ld + j];
+    li[q] = Linv[e];
   }
-  const float* dblk = M + (int64_t)k * kT * D + (int64_t)k * kT;
-  float dg[16];  // all loads in flight before the first use
+  if (row_block && blockIdx.x == 0) {  // the next diagonal block, before this panel's update reaches it
+    const float* dsrc = M + (int64_t)(k + 1) * kT * D + (int64_t)(k + 1) * kT;
+    float dv[16];
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q;
-    dg[q] = dblk[(int64_t)(e >> 6) * D + (e & 63)];
-  }
+    for (int q = 0; q < 16; ++q) {
+      const int e = tid + 256 * q;
+      dv[q] = dsrc[(int64_t)(e >> 6) * D + (e & 63)];
+    }
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q;
-    A[e >> 6][e & 63] = dg[q];
-  }
-  if (tid == 0) bad = -1;
-  __syncthreads();
-  factor_diag64(A, X, T, Ls, &bad, k * kT);
-  if (blockIdx.x == 0 && tid == 0 && bad >= 0 && status) {
-    if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
+    for (int q = 0; q < 16; ++q) dnext[tid + 256 * q] = dv[q];
   }
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const int e = tid + 256 * q;
     A[e >> 6][e & 63] = pre[q];
+    X[e >> 6][e & 63] = li[q];
   }
   __syncthreads();
   const int tx = tid & 15, ty = tid >> 4;
@@ -693,9 +747,10 @@ __global__ void split_rhs_kernel(const float* __restrict__ RHS, int D, __nv_bflo
 }  // namespace simt
 
 // workspace of the tensor-core form: M (4 D^2) | RHS (8 D^2) | split area (4 D^2) |
-// Linv (256 D) | A hi/lo (256 D) | L21^T hi/lo (256 D) | Y_k hi/lo (512 D) | lambda
+// Linv (256 D) | A hi/lo (256 D) | L21^T hi/lo (256 D) | Y_k hi/lo (512 D) | lambda (256) |
+// next diagonal block (16 KB)
 static bool tc_eligible(ispa_dtype_t w_dt, int64_t D) { return w_dt == ISPA_DT_BF16 && D % 128 == 0 && D >= 256; }
-static size_t tc_workspace_bytes(int64_t D) { return (size_t)(16 * D * D + 1280 * D + 256); }
+static size_t tc_workspace_bytes(int64_t D) { return (size_t)(16 * D * D + 1280 * D + 256 + 64 * 64 * 4); }
 static size_t compact_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
 
 size_t absorb_workspace_bytes(int64_t D) { return D % 128 == 0 && D >= 256 ? tc_workspace_bytes(D) : compact_workspace_bytes(D); }
@@ -710,6 +765,52 @@ ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const voi
                                cudaStream_t stream);
 ispa_status_t gemm_hilo_w(int64_t M, int64_t K, const void* a_hi, const void* a_lo, const void* w, int64_t N,
                           float* c, int64_t ldc, cudaStream_t stream);
+
+// One side stream and two events per host thread and CUDA context, created on
+// the first tensor-core solve there (make that first call before any stream
+// capture) and kept until the process exits.
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+struct SideStream {
+  unsigned long long ctx;
+  cudaStream_t stream;
+  cudaEvent_t fork, join;
+};
+thread_local std::vector<SideStream> t_side;
+}  // namespace
+
+static ispa_status_t side_stream_for_current_context(cudaStream_t* s, cudaEvent_t* fork, cudaEvent_t* join) {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) {
+    set_last_error("no current CUDA context for the absorb solve's side stream");
+    return ISPA_ERR_CUDA;
+  }
+  for (const auto& e : t_side)
+    if (e.ctx == id) {
+      *s = e.stream, *fork = e.fork, *join = e.join;
+      return ISPA_OK;
+    }
+  SideStream e{id, nullptr, nullptr, nullptr};
+  if (cudaStreamCreateWithFlags(&e.stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&e.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&e.join, cudaEventDisableTiming) != cudaSuccess)
+    return check_launch("creating the absorb solve's side stream");
+  t_side.push_back(e);
+  *s = e.stream, *fork = e.fork, *join = e.join;
+  return ISPA_OK;
+}
 
 static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_bfloat16* W, int64_t D64,
                                     double lam_abs, double lam_rel, float* dW, __nv_bfloat16* w_new, void* workspace,
@@ -728,8 +829,14 @@ static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_
   __nv_bfloat16* y_hi = lt_lo + 64 * D64;
   __nv_bfloat16* y_lo = y_hi + 128 * D64;
   double* lam = reinterpret_cast<double*>(ws + 16 * D64 * D64 + 1280 * D64);
+  float* Linv = reinterpret_cast<float*>(ws + 16 * D64 * D64);
+  float* dnext = reinterpret_cast<float*>(ws + 16 * D64 * D64 + 1280 * D64 + 256);
   const int sms = num_sms();
   const int64_t rhs_ld = 2 * D64;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  ispa_status_t s0 = side_stream_for_current_context(&side, &ev_fork, &ev_join);
+  if (s0 != ISPA_OK) return s0;
 
   // S = R W into RHS[:, :D], RHS[:, D:] = I
   __nv_bfloat16* r_hi = reinterpret_cast<__nv_bfloat16*>(split);
@@ -740,16 +847,26 @@ static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_
   if (s1 != ISPA_OK) return s1;
   trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
   shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
+  // the first diagonal block; each later one is factored on the side stream
+  // while the previous panel's update product runs (one-panel look-ahead)
+  diag_factor_kernel<<<1, 256, 0, st>>>(M, D64, nullptr, D, 0, Linv, status);
   for (int k = 0; k < nb; ++k) {
     const int rest = nb - k - 1;
     const int off = (k + 1) * kT;
     const int rhs_cols = D + off;  // nonzero columns of the panel's rows of [L^-1 S | L^-1]
-    panel_factor_kernel<<<rest + (rhs_cols + kT - 1) / kT, 256, 0, st>>>(
-        M, D, k, rest, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, status);
+    float* Lk = Linv + (int64_t)k * kT * kT;
+    panel_apply_kernel<<<rest + (rhs_cols + kT - 1) / kT, 256, 0, st>>>(
+        M, D, k, rest, Lk, dnext, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld);
     if (rest > 0) {
+      if (cudaEventRecord(ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess)
+        return check_launch("absorb fork");
+      diag_factor_kernel<<<1, 256, 0, side>>>(dnext, kT, M + (int64_t)off * D + (int64_t)k * kT, D, k + 1,
+                                              Lk + kT * kT, status);
+      if (cudaEventRecord(ev_join, side) != cudaSuccess) return check_launch("absorb join");
       s1 = absorb_step_update(D - off, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, rhs_cols,
                               M + (int64_t)off * D + off, D64, RHS + (int64_t)off * rhs_ld, rhs_ld, st);
       if (s1 != ISPA_OK) return s1;
+      if (cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess) return check_launch("absorb join");
     }
   }
   // dW = (L^-1)^T (L^-1 S): hi/lo of L^-1 S into M's storage, of L^-1 into the split area

@@ -199,7 +199,13 @@ ISPA_API size_t ispa_absorb_workspace_bytes(int64_t d_model);
  * bf16 W and d_model a multiple of 128 (>= 256) the products run on the tensor
  * cores in split precision (bf16 hi/lo pairs, about 2^-17 relative per
  * product) and the solves are carried through the factorisation; otherwise
- * (fp32 W, other sizes) the updates run on the CUDA cores in fp32.
+ * (fp32 W, other sizes) the updates run on the CUDA cores in fp32.  The
+ * tensor-core form factors each next diagonal block on an internal stream
+ * beside the current update (fork and join by events recorded on `stream`, so
+ * the call stays asynchronous and graph capture sees one fork/join per panel);
+ * that stream and its two events are created on the first such call in a host
+ * thread and CUDA context -- make that call before any stream capture -- and
+ * live until the process exits.
  * G, R fp32 [D, D] (G symmetric; only its lower triangle is read), W and w_new
  * [D, D] in w_dt, delta_w fp32 [D, D].  workspace: device buffer of at least
  * ispa_absorb_workspace_bytes(d_model) bytes, 256-byte aligned.  dev_status
