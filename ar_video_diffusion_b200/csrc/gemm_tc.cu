@@ -12,11 +12,14 @@
 //    partial sums are added into G, R with vector reductions in L2;
 //  * the output projection y = A W (stages 1 and 3 of the same section): A is
 //    K-major (token rows), W [D_in, D_out] is MN-major.
-// One CTA computes a 256 x BN tile as two 128-row halves that share every B
-// tile (two M=128 MMAs per K step), which halves the operand traffic per FLOP
-// against a 128-row tile: warp 0 issues TMA loads into an NST-deep ring,
-// warp 1 issues tcgen05.mma, warp 2 owns the 2*BN tensor-memory columns and
-// warps 4-11 drain the two accumulators (one row per thread).
+// One CTA computes either a 256 x BN tile as two 128-row halves that share
+// every B tile, or (the "wide" form) a 128 x 2BN tile as two BN-column halves
+// that share every A tile: two M=128 MMAs per K step either way, which halves
+// the operand traffic per FLOP against a single 128 x BN product.  The wide
+// form lets a 4680 x 1536 output be cut into exactly 148 tiles (128 x 384).
+// Warp 0 issues TMA loads into an NST-deep ring, warp 1 issues tcgen05.mma,
+// warp 2 owns the tensor-memory columns (two BN-column accumulators) and
+// warps 4-11 drain them (one row per thread, one accumulator per warpgroup).
 #include <cstring>
 
 #include "internal.h"
@@ -57,10 +60,13 @@ struct Params {
   const float* col_scale;
 };
 
-template <int BN, int NST>
+template <int BN, int NST, bool WIDE = false>
 struct Layout {
-  static constexpr int kABytes = kBM * kBK * 2;  // 32 KB
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kRows = WIDE ? 128 : kBM;  // output rows of a tile
+  static constexpr int kCols = WIDE ? 2 * BN : BN;  // output columns of a tile
+  static constexpr int kABytes = kRows * kBK * 2;
+  static constexpr int kBBytes = kCols * kBK * 2;
+  static constexpr int kTmemCols = 2 * BN <= 256 ? 256 : 512;  // a power of two
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBars = NST * kStage;
   static constexpr int kNumBars = 2 * NST + 2;  // full[NST], empty[NST], acc_full, teardown
@@ -77,17 +83,17 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // The body shared by the bf16 kernels and the e4m3 kernel (F8: both operands
 // K-major e4m3, kind::f8f6f4 MMAs with K = 32, the same 128-byte rows and
 // swizzle per stage as bf16, and a scaled bf16 epilogue through TMA).
-template <bool A_MN, bool B_MN, int BN, int NST, bool F8>
+template <bool A_MN, bool B_MN, int BN, int NST, bool F8, bool WIDE>
 __device__ __forceinline__ void gemm_body(const Params& p) {
-  using L = Layout<BN, NST>;
+  using L = Layout<BN, NST, WIDE>;
   static_assert(!F8 || (!A_MN && !B_MN), "e4m3 operands are K-major");
   constexpr int BK = F8 ? kBK8 : kBK;
-  const int n0g = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int n0g = blockIdx.x * L::kCols, m0 = blockIdx.y * L::kRows;
   const int half_n = n0g >= p.n_split ? 1 : 0;
   const int n0 = n0g - half_n * p.n_split;
   // whole-CTA early exit (before any barrier or tensor-memory use): a tile of
   // a lower-triangular output that lies strictly above the diagonal
-  if (half_n == 0 && p.lower_only0 && n0 > m0 + kBM - 1) return;
+  if (half_n == 0 && p.lower_only0 && n0 > m0 + L::kRows - 1) return;
   int k_begin = blockIdx.z * p.k_per_split;
   const int k_end = min(p.K, k_begin + p.k_per_split);
   if (p.a_upper) k_begin = max(k_begin, (m0 / BK) * BK);
@@ -116,7 +122,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     fence_barrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -143,15 +149,17 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
       mbar_arrive_expect_tx(&full[stage], L::kStage);
       if (A_MN) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_load_2d(sa + c * 8192, am, &full[stage], m0 + 64 * c, k0);
+        for (int c = 0; c < L::kRows / 64; ++c) tma_load_2d(sa + c * 8192, am, &full[stage], m0 + 64 * c, k0);
       } else {
-        tma_load_2d(sa, am, &full[stage], k0, m0);
+        tma_load_2d(sa, am, &full[stage], k0, m0);  // one box of kRows rows
       }
       if (B_MN) {
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * 8192, bm, &full[stage], n0 + 64 * c, k0);
+        for (int c = 0; c < L::kCols / 64; ++c) tma_load_2d(sb + c * 8192, bm, &full[stage], n0 + 64 * c, k0);
       } else {
-        tma_load_2d(sb, bm, &full[stage], k0, n0);
+#pragma unroll
+        for (int h = 0; h < L::kCols / BN; ++h)  // boxes of BN rows (a box is at most 256 rows)
+          tma_load_2d(sb + h * BN * 128, bm, &full[stage], k0, n0 + h * BN);
       }
     }
     if (kb < steps) {  // unwinding after a timeout
@@ -174,12 +182,16 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
       const uint32_t sb = sa + L::kABytes;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {  // 4 MMAs of 32 bytes of K (16 bf16 or 32 e4m3)
-        const uint64_t db = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024) : sdesc_sw128(sb + kk * 32, 16, 1024);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          // rows 128h..128h+127 of the A tile: MN-major blocks 2h, 2h+1 / K-major rows
-          const uint64_t da = A_MN ? sdesc_sw128(sa + h * 16384 + kk * 2048, 8192, 1024)
-                                   : sdesc_sw128(sa + h * 16384 + kk * 32, 16, 1024);
+          // tall tile: rows 128h..128h+127 of the A tile (MN-major blocks 2h,
+          // 2h+1 / K-major rows) against the whole B tile; wide tile: the
+          // whole A tile against columns BN h .. BN h + BN - 1 of the B tile
+          const int ah = WIDE ? 0 : h, bh = WIDE ? h : 0;
+          const uint64_t da = A_MN ? sdesc_sw128(sa + ah * 16384 + kk * 2048, 8192, 1024)
+                                   : sdesc_sw128(sa + ah * 16384 + kk * 32, 16, 1024);
+          const uint64_t db = B_MN ? sdesc_sw128(sb + bh * (BN / 64) * 8192 + kk * 2048, 8192, 1024)
+                                   : sdesc_sw128(sb + bh * BN * 128 + kk * 32, 16, 1024);
           if (F8)
             umma_ss_f8(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
           else
@@ -193,9 +205,10 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     mbar_wait_drain(teardown, 0, 100000000ull);
   } else if (warp >= 4) {
     // ----------------------------------------------------------- epilogue
-    const int h = (warp - 4) >> 2;
+    const int h = (warp - 4) >> 2;  // accumulator: row half (tall tile) or column half (wide tile)
     const int wq = warp & 3;
-    const int row0 = m0 + h * 128 + wq * 32;
+    const int row0 = m0 + (WIDE ? 0 : h * 128) + wq * 32;
+    const int col0 = n0 + (WIDE ? h * BN : 0);
     const int gm = row0 + lane;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag));
     if (ok && p.c_tma) {
@@ -219,10 +232,11 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
         if (F8) {
           // per-row and per-column dequantisation scales
           const float sa = gm < p.M ? __ldg(p.row_scale + gm) : 0.f;
-          const float4* sw4 = reinterpret_cast<const float4*>(p.col_scale + n0 + 32 * c);
+          const float4* sw4 = reinterpret_cast<const float4*>(p.col_scale + col0 + 32 * c);
+          const bool cols_in = col0 + 32 * c < p.n_cols[half_n];  // a ragged last tile reads no scale past N
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 w4 = __ldg(sw4 + j);
+            const float4 w4 = cols_in ? __ldg(sw4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             r[4 * j + 0] = __float_as_uint(__uint_as_float(r[4 * j + 0]) * (sa * w4.x));
             r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) * (sa * w4.y));
             r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) * (sa * w4.z));
@@ -255,7 +269,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const int gn = n0 + 32 * c;
+          const int gn = col0 + 32 * c;
           if (rows_in && gn < n_cols) {  // boxes are clipped at the matrix edge; skip wholly outside ones
             if (p.mode == kReduceF32)
               tma_reduce_add_2d(cm, buf, gn, row0);
@@ -276,7 +290,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
         uint32_t r[32];
         tmem_ld32(taddr + 32 * c, r);
         tmem_wait_ld();
-        const int gn = n0 + 32 * c;
+        const int gn = col0 + 32 * c;
         if (gm >= p.M || gn >= n_cols) continue;
         if (p.mode == kStoreBf16) {
           uint4* dst =
@@ -309,18 +323,18 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, 2 * BN);
+  if (warp == 2) tmem_dealloc(tmem, L::kTmemCols);
   if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
 }
 
-template <bool A_MN, bool B_MN, int BN, int NST>
+template <bool A_MN, bool B_MN, int BN, int NST, bool WIDE = false>
 __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_constant__ Params p) {
-  gemm_body<A_MN, B_MN, BN, NST, false>(p);
+  gemm_body<A_MN, B_MN, BN, NST, false, WIDE>(p);
 }
 
-template <int BN, int NST>
+template <int BN, int NST, bool WIDE = false>
 __global__ void __launch_bounds__(kThreads, 1) gemm_e4m3_kernel(const __grid_constant__ Params p) {
-  gemm_body<false, false, BN, NST, true>(p);
+  gemm_body<false, false, BN, NST, true, WIDE>(p);
 }
 
 // Output maps for the TMA epilogue: c[0] has inner0 columns, c[1] inner1, both
@@ -336,26 +350,60 @@ static bool set_out_maps(Params& p, bool f32, int64_t rows, int64_t ld, int64_t 
   return true;
 }
 
-template <int BN, int NST>
+template <int BN, int NST, bool WIDE = false>
 static ispa_status_t launch_e4m3(const Params& p, cudaStream_t stream) {
-  using L = Layout<BN, NST>;
-  auto kern = gemm_e4m3_kernel<BN, NST>;
+  using L = Layout<BN, NST, WIDE>;
+  auto kern = gemm_e4m3_kernel<BN, NST, WIDE>;
+  if (p.n_split < p.N && p.n_split % L::kCols) return unsupported("GEMM column ranges must start on a tile");
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
-  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM, 1);
+  dim3 grid((p.N + L::kCols - 1) / L::kCols, (p.M + L::kRows - 1) / L::kRows, 1);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
   return check_launch("gemm_e4m3_kernel");
 }
 
-template <bool A_MN, bool B_MN, int BN, int NST>
+template <bool A_MN, bool B_MN, int BN, int NST, bool WIDE = false>
 static ispa_status_t launch(const Params& p, int k_splits, cudaStream_t stream) {
-  using L = Layout<BN, NST>;
-  auto kern = gemm_bf16_kernel<A_MN, B_MN, BN, NST>;
+  using L = Layout<BN, NST, WIDE>;
+  auto kern = gemm_bf16_kernel<A_MN, B_MN, BN, NST, WIDE>;
+  if (p.n_split < p.N && p.n_split % L::kCols) return unsupported("GEMM column ranges must start on a tile");
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
-  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM, k_splits);
+  dim3 grid((p.N + L::kCols - 1) / L::kCols, (p.M + L::kRows - 1) / L::kRows, k_splits);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
   return check_launch("gemm_bf16_kernel");
+}
+
+// Output tile of a projection [M, N] (N a multiple of 128): 256 x 256,
+// 256 x 128 or the wide 128 x 384.  Each CTA holds one tile and one CTA fits
+// an SM, so the launch takes ceil(tiles / SMs) waves, each as long as one
+// tile; the shape with the least wave time (tile area over a relative
+// efficiency, measured on B200 at 4680 x 1536 and 4680 x 5120) wins.  A
+// wide tile may overhang the last columns (its loads read zeros there and its
+// stores are clipped).
+enum class ProjTile : int { kTall256, kTall128, kWide192 };
+
+static ProjTile projection_tile(int64_t M, int64_t N) {
+  struct Cand {
+    ProjTile t;
+    int64_t rows, cols;
+    double eff;
+  };
+  // time per tile area relative to 256 x 256, from B200 runs of one to
+  // six waves: the narrower tiles re-read more operand bytes per FLOP
+  const Cand cands[3] = {{ProjTile::kTall256, 256, 256, 1.0},
+                         {ProjTile::kWide192, 128, 384, 0.87},
+                         {ProjTile::kTall128, 256, 128, 0.75}};
+  const int64_t sms = num_sms();
+  ProjTile best = ProjTile::kTall128;
+  double best_cost = 0.0;
+  for (const Cand& c : cands) {
+    if (c.t == ProjTile::kTall256 && N % 256) continue;
+    const int64_t tiles = ((M + c.rows - 1) / c.rows) * ((N + c.cols - 1) / c.cols);
+    const double cost = (double)((tiles + sms - 1) / sms) * (double)(c.rows * c.cols) / c.eff;
+    if (best_cost == 0.0 || cost < best_cost) best = c.t, best_cost = cost;
+  }
+  return best;
 }
 
 }  // namespace gemm
@@ -481,7 +529,10 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_bf16_2d(&p.a_map[0], a, d_in, n_rows, a_stride * 2, 64, kBM)) return ISPA_ERR_CUDA;
+  if (d_out % 128) return unsupported("bf16 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);
+  const ProjTile t = projection_tile(n_rows, d_out);
+  if (!encode_map_bf16_2d(&p.a_map[0], a, d_in, n_rows, a_stride * 2, 64, t == ProjTile::kWide192 ? 128 : kBM))
+    return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&p.b_map[0][0], w, d_out, d_in, d_out * 2, 64, 64)) return ISPA_ERR_CUDA;
   p.b_map[1][0] = p.b_map[0][0];
   p.M = (int32_t)n_rows;
@@ -497,9 +548,11 @@ ispa_status_t project_bf16(const void* a, int64_t n_rows, int64_t d_in, int64_t 
   p.ldc = d_out;
   p.mode = kStoreBf16;
   if (!set_out_maps(p, false, n_rows, d_out, d_out, d_out)) return ISPA_ERR_CUDA;
-  if (d_out % 256 == 0) return launch<false, true, 256, 3>(p, 1, stream);
-  if (d_out % 128 == 0) return launch<false, true, 128, 4>(p, 1, stream);
-  return unsupported("bf16 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);
+  switch (t) {
+    case ProjTile::kWide192: return launch<false, true, 192, 3, true>(p, 1, stream);
+    case ProjTile::kTall256: return launch<false, true, 256, 3>(p, 1, stream);
+    default: return launch<false, true, 128, 4>(p, 1, stream);
+  }
 }
 
 // y[n_rows, d_out] (bf16) = diag(a_scale) qa[n_rows, d_in] qw_t[d_out, d_in]^T diag(w_scale):
@@ -510,8 +563,11 @@ ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_ro
   using namespace gemm;
   Params p;
   memset(&p, 0, sizeof(p));
-  if (!encode_map_u8_2d(&p.a_map[0], qa, d_in, n_rows, d_in, kBK8, kBM)) return ISPA_ERR_CUDA;
-  const int BN = d_out % 256 == 0 ? 256 : 128;
+  if (d_out % 128) return unsupported("e4m3 projection needs d_out to be a multiple of 128 (got %lld)", (long long)d_out);
+  const ProjTile t = projection_tile(n_rows, d_out);
+  const int BN = t == ProjTile::kWide192 ? 192 : t == ProjTile::kTall256 ? 256 : 128;
+  if (!encode_map_u8_2d(&p.a_map[0], qa, d_in, n_rows, d_in, kBK8, t == ProjTile::kWide192 ? 128 : kBM))
+    return ISPA_ERR_CUDA;
   if (!encode_map_u8_2d(&p.b_map[0][0], qw_t, d_in, d_out, d_in, kBK8, BN)) return ISPA_ERR_CUDA;
   p.b_map[1][0] = p.b_map[0][0];
   p.M = (int32_t)n_rows;
@@ -530,8 +586,11 @@ ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_ro
   p.col_scale = w_scale;
   if (!set_out_maps(p, false, n_rows, d_out, d_out, d_out)) return ISPA_ERR_CUDA;
   if (!p.c_tma) return unsupported("e4m3 projection needs a 16-byte aligned output");
-  if (BN == 256) return launch_e4m3<256, 3>(p, stream);
-  return launch_e4m3<128, 4>(p, stream);
+  switch (t) {
+    case ProjTile::kWide192: return launch_e4m3<192, 3, true>(p, stream);
+    case ProjTile::kTall256: return launch_e4m3<256, 3>(p, stream);
+    default: return launch_e4m3<128, 4>(p, stream);
+  }
 }
 
 }  // namespace ispa

@@ -296,7 +296,10 @@ def test_bounded_wait_times_out_and_gpu_stays_usable():
     assert x.sum().item() == 1000
 
 
-@pytest.mark.parametrize("n,din,dout", [(4680, 1536, 1536), (77, 128, 256)])
+# (4680, *, 1536) and (4680, *, 1280) take the 128 x 384 tile (the second
+# overhangs the last columns), (4680, *, 5120) the 256 x 256 tile and
+# (77, *, 256) the 256 x 128 tile on a 148-SM B200
+@pytest.mark.parametrize("n,din,dout", [(4680, 1536, 1536), (4680, 256, 1280), (4680, 64, 5120), (77, 128, 256)])
 def test_project_bf16_matches_oracle(n, din, dout):
     g = np.random.default_rng(n)
     A = synth.round_bf16(g.standard_normal((n, din)).astype(np.float32))

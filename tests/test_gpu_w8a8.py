@@ -89,8 +89,8 @@ def _check_projection(y, qa, sa, qw, sw):
     assert fro_rel(got, ref) <= 4e-3
 
 
-@pytest.mark.parametrize("n,d_in,d_out", [(4680, 1536, 1536), (300, 256, 384), (129, 128, 128), (1, 5120, 256),
-                                          (517, 48, 128)])
+@pytest.mark.parametrize("n,d_in,d_out", [(4680, 1536, 1536), (4680, 256, 1280), (300, 256, 384), (129, 128, 128),
+                                          (1, 5120, 256), (517, 48, 128)])
 def test_project_w8a8_matches_oracle(n, d_in, d_out):
     rng = np.random.default_rng(n + d_in + d_out)
     a = _bf16(rng, (n, d_in))
