@@ -12,7 +12,8 @@ namespace ispa {
 ispa_status_t dual_attention_bf16_db(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
                                      float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
                                      void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
-                                     int32_t* status, cudaStream_t stream);
+                                     int32_t* status, cudaStream_t stream, uint8_t* mx_codes = nullptr,
+                                     uint8_t* mx_exps = nullptr);
 ispa_status_t dual_attention_f32(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
                                  float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
                                  void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
@@ -46,6 +47,10 @@ ispa_status_t quantize_weight_e4m3(const void* w, int64_t K, int64_t N, uint8_t*
                                    cudaStream_t stream);
 ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_rows, int64_t d_in,
                            const uint8_t* qw_t, const float* w_scale, int64_t d_out, void* y, cudaStream_t stream);
+ispa_status_t mx_quantize_rows_e4m3(const void* x, int64_t n_rows, int64_t K, int64_t stride, uint8_t* q, uint8_t* e,
+                                    cudaStream_t stream);
+ispa_status_t project_mx(const uint8_t* qa, const uint8_t* ea, int64_t n_rows, int64_t d_in, const uint8_t* qw_t,
+                         const float* w_scale, int64_t d_out, void* y, cudaStream_t stream);
 
 static bool valid_dtype(ispa_dtype_t dt) { return dt == ISPA_DT_BF16 || dt == ISPA_DT_F32; }
 static int64_t elem_bytes(ispa_dtype_t dt) { return dt == ISPA_DT_BF16 ? 2 : 4; }
@@ -356,6 +361,60 @@ extern "C" ispa_status_t ispa_local_attention_project_w8a8(
   st = ispa_quantize_e4m3_rows(a_loc_out, n_q, D, D, dt, a_codes, a_scales, stream);
   if (st != ISPA_OK) return st;
   return ispa_project_w8a8(a_codes, a_scales, n_q, D, w_codes_t, w_scales, D, y, stream);
+}
+
+extern "C" ispa_status_t ispa_mx_quantize_e4m3_rows(const void* x, int64_t n_rows, int64_t k, int64_t row_stride,
+                                                    ispa_dtype_t dt, uint8_t* codes, uint8_t* exps, void* stream) {
+  if (dt != ISPA_DT_BF16) return unsupported("MX quantisation takes bf16 activations");
+  if (!x || !codes || !exps) return invalid("required pointer is NULL");
+  if (n_rows <= 0 || k <= 0) return invalid("sizes must be positive");
+  if (k % 32) return unsupported("MX quantisation needs k %% 32 == 0 (got %lld)", (long long)k);
+  if (row_stride < k) return invalid("row_stride < k");
+  if (!aligned16(x) || !aligned16(codes) || (row_stride * 2) % 16)
+    return invalid("x and codes must be 16-byte aligned (rows too)");
+  if (n_rows > INT32_MAX / 2 || k > 65536) return unsupported("problem too large");
+  return mx_quantize_rows_e4m3(x, n_rows, k, row_stride, codes, exps, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_project_mx(const uint8_t* a_codes, const uint8_t* a_exps, int64_t n_rows, int64_t d_in,
+                                         const uint8_t* w_codes_t, const float* w_scales, int64_t d_out, void* y,
+                                         void* stream) {
+  if (!a_codes || !a_exps || !w_codes_t || !w_scales || !y) return invalid("required pointer is NULL");
+  if (n_rows <= 0 || d_in <= 0 || d_out <= 0) return invalid("sizes must be positive");
+  if (!aligned16(a_codes) || !aligned4(a_exps) || !aligned16(w_codes_t) || !aligned16(w_scales) || !aligned16(y))
+    return invalid("codes, w_scales and y must be 16-byte aligned, a_exps 4-byte aligned");
+  if (n_rows > INT32_MAX / 2 || d_out > 65536) return unsupported("problem too large");
+  return project_mx(a_codes, a_exps, n_rows, d_in, w_codes_t, w_scales, d_out, y, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" ispa_status_t ispa_local_attention_project_mx(
+    const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim, ispa_dtype_t dt,
+    float softmax_scale, const ispa_kv_segment_t* local, int32_t n_local, const uint8_t* w_codes_t,
+    const float* w_scales, void* y, uint8_t* a_codes, uint8_t* a_exps, int32_t* dev_status, void* stream) {
+  if (dt != ISPA_DT_BF16) return unsupported("the MX L-layer path takes bf16 activations");
+  ispa_status_t st = check_attention_common(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale);
+  if (st != ISPA_OK) return st;
+  if (!w_codes_t || !w_scales || !y || !a_codes || !a_exps)
+    return invalid("w_codes_t, w_scales, y, a_codes and a_exps are required");
+  if (!aligned16(a_codes) || !aligned4(a_exps)) return invalid("a_codes must be 16-byte aligned, a_exps 4-byte");
+  const int64_t D = (int64_t)n_heads * head_dim;
+  if (D % 128) return unsupported("MX L-layer projection needs D %% 128 == 0");
+  ispa_kv_segment_t segs[ISPA_MAX_SEGMENTS];
+  int nl = 0, nh = 0;
+  int64_t lt = 0, ht = 0;
+  st = collect_segments(local, n_local, nullptr, 0, D, dt, segs, &nl, &nh, &lt, &ht);
+  if (st != ISPA_OK) return st;
+  if (lt == 0) return invalid("attention over an empty key set");
+  // the projection's limits are checked before anything is launched
+  if (D / 128 > 28) return unsupported("block-scaled projection needs D <= 3584 (got %lld)", (long long)D);
+  if (!aligned16(w_codes_t) || !aligned16(w_scales) || !aligned16(y))
+    return invalid("w_codes_t, w_scales and y must be 16-byte aligned");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt((float)head_dim);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = dual_attention_bf16_db(q, n_q, q_stride, n_heads, head_dim, scale, segs, nl, 0, nullptr, nullptr, nullptr,
+                              nullptr, nullptr, dev_status, s, a_codes, a_exps);
+  if (st != ISPA_OK) return st;
+  return project_mx(a_codes, a_exps, n_q, D, w_codes_t, w_scales, D, y, s);
 }
 
 // ------------------------------------------------------------ bookkeeping

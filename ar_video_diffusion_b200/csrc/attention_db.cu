@@ -84,6 +84,10 @@ struct Params {
   float* lse_full;
   int64_t out_stride;
   int32_t* status;
+  // single pass only: MX e4m3 codes [n_q, D] and exponent bytes [n_q, D / 32]
+  // of the bf16-rounded output (a_full may then be NULL)
+  uint8_t* mx_codes;
+  uint8_t* mx_exps;
 };
 
 template <int HD, int NST>
@@ -517,7 +521,24 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
       float x[32];
       load_o(r, c_first + kc, inv, x);
       if (!r.row_ok) continue;
-      store_bf16x32(p.a_full + base + 32 * kc, x);
+      if (p.a_full) store_bf16x32(p.a_full + base + 32 * kc, x);
+      if (p.mx_codes) {
+        // the block of the bf16 output, quantised with its own power-of-two scale
+        float xb[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const uint32_t u = pack_bf16x2(x[j], x[j + 1]);
+          xb[j] = __uint_as_float(u << 16);
+          xb[j + 1] = __uint_as_float(u & 0xFFFF0000u);
+        }
+        uint32_t c[8];
+        const uint32_t ebyte = mx_quantize32(xb, c);
+        const int64_t ch = (int64_t)head * HD + w * (HD / 2) + 32 * kc;  // first channel of the block
+        uint4* dst = reinterpret_cast<uint4*>(p.mx_codes + (int64_t)r.grow * p.out_stride + ch);
+        dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+        dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        p.mx_exps[(int64_t)r.grow * (p.out_stride / 32) + ch / 32] = (uint8_t)ebyte;
+      }
       if (dual) {
         store_bf16x32(p.a_loc + base + 32 * kc, x);
         if (p.a_delta) {
@@ -650,7 +671,7 @@ static ispa_status_t launch(Params& p, int n_heads, cudaStream_t stream) {
 ispa_status_t dual_attention_bf16_db(const void* q, int64_t n_q, int64_t q_stride, int32_t n_heads, int32_t head_dim,
                                      float scale, const ispa_kv_segment_t* segs, int n_local_seg, int n_hist_seg,
                                      void* a_loc, void* a_full, void* a_delta, float* lse_loc, float* lse_full,
-                                     int32_t* status, cudaStream_t stream) {
+                                     int32_t* status, cudaStream_t stream, uint8_t* mx_codes, uint8_t* mx_exps) {
   using namespace attn2;
   static_assert(sizeof(Params) <= 4096, "kernel parameter space");
   Params p;
@@ -687,6 +708,8 @@ ispa_status_t dual_attention_bf16_db(const void* q, int64_t n_q, int64_t q_strid
   p.lse_full = lse_full;
   p.out_stride = D;
   p.status = status;
+  p.mx_codes = mx_codes;
+  p.mx_exps = mx_exps;
   if (head_dim == 128) return launch<128, 3>(p, n_heads, stream);
   return launch<64, 6>(p, n_heads, stream);
 }

@@ -56,8 +56,10 @@ struct Params {
   int64_t ldc;
   int32_t mode;
   int32_t* status;
-  const float* row_scale;  // e4m3 inputs: y[i, j] = acc[i, j] * row_scale[i] * col_scale[j]
+  const float* row_scale;  // e4m3 inputs: y[i, j] = acc[i, j] * row_scale[i] * col_scale[j] (no row_scale: 1)
   const float* col_scale;
+  const uint8_t* a_exps;  // block-scaled A: ue8m0 exponent bytes [M, K / 32], exps_ld bytes per row
+  int32_t exps_ld;
 };
 
 template <int BN, int NST, bool WIDE = false>
@@ -69,7 +71,7 @@ struct Layout {
   static constexpr int kTmemCols = 2 * BN <= 256 ? 256 : 512;  // a power of two
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBars = NST * kStage;
-  static constexpr int kNumBars = 2 * NST + 2;  // full[NST], empty[NST], acc_full, teardown
+  static constexpr int kNumBars = 2 * NST + 3;  // full[NST], empty[NST], acc_full, teardown, sf_ready
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -80,13 +82,30 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-// The body shared by the bf16 kernels and the e4m3 kernel (F8: both operands
+// Tensor-memory columns of the block-scaled form (wide tile, BN = 192: the
+// accumulators take columns 0-383): unit B scales in 16 columns, then the A
+// scales, 4 columns per 128-element K stage.
+constexpr uint32_t kSfbCol = 384;
+constexpr uint32_t kSfaCol = 400;
+constexpr int kMxMaxStages = (512 - (int)kSfaCol) / 4;  // K <= 28 * 128 = 3584
+
+// The body shared by the bf16 kernels and the e4m3 kernels (F8: both operands
 // K-major e4m3, kind::f8f6f4 MMAs with K = 32, the same 128-byte rows and
 // swizzle per stage as bf16, and a scaled bf16 epilogue through TMA).
-template <bool A_MN, bool B_MN, int BN, int NST, bool F8, bool WIDE>
+//
+// MX (block-scaled A, wide tile only): the MMAs are kind::mxf8f6f4 with one
+// ue8m0 scale per 32 K-elements of each row of A and unit scales for B (the
+// per-column weight scale stays in the epilogue).  Before the first MMA,
+// warps 4-7 write every scale of the tile's 128 rows into tensor memory in
+// the layout the instruction reads for M = 128: the scale of row 32c + l for
+// the K block 4j + b sits in byte b of column kSfaCol + 4j + c, lane l, and is
+// repeated in the lanes l + 32, l + 64, l + 96 of the other three
+// sub-partitions.
+template <bool A_MN, bool B_MN, int BN, int NST, bool F8, bool WIDE, bool MX = false>
 __device__ __forceinline__ void gemm_body(const Params& p) {
   using L = Layout<BN, NST, WIDE>;
   static_assert(!F8 || (!A_MN && !B_MN), "e4m3 operands are K-major");
+  static_assert(!MX || (F8 && WIDE && BN == 192), "the block-scaled form uses the wide e4m3 tile");
   constexpr int BK = F8 ? kBK8 : kBK;
   const int n0g = blockIdx.x * L::kCols, m0 = blockIdx.y * L::kRows;
   const int half_n = n0g >= p.n_split ? 1 : 0;
@@ -107,6 +126,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
   uint64_t* empty = full + NST;
   uint64_t* acc_full = empty + NST;
   uint64_t* teardown = acc_full + 1;
+  uint64_t* sf_ready = teardown + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,6 +138,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     }
     mbar_init(acc_full, 1);
     mbar_init(teardown, 1);
+    mbar_init(sf_ready, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -129,6 +150,33 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  if (MX && warp >= 4 && warp < 8) {
+    // ------------------------------------------------- block scales (MX)
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t r[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[j] = 0x7F7F7F7Fu;  // 2^0 in every byte
+    tmem_st16(tmem + lanes + kSfbCol, r);
+#pragma unroll 1
+    for (int g = 0; g < (nk + 3) / 4; ++g) {  // 16 columns: 4 K stages x 4 row groups
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int j = 4 * g + t;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int row = m0 + 32 * c + lane;
+          r[4 * t + c] = (j < nk && row < p.M)
+                             ? __ldg(reinterpret_cast<const uint32_t*>(p.a_exps + (int64_t)row * p.exps_ld + 4 * j))
+                             : 0x7F7F7F7Fu;
+        }
+      }
+      tmem_st16(tmem + lanes + kSfaCol + 16 * g, r);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(sf_ready);
+  }
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA
@@ -168,10 +216,15 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
-    constexpr uint32_t kIdesc = F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, A_MN, B_MN);
+    constexpr uint32_t kIdesc =
+        MX ? idesc_mxf8_f32(128, BN) : F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, A_MN, B_MN);
     const uint32_t base = smem_u32(smem);
     bool ok = true;
-    for (int kb = 0; kb < steps; ++kb) {
+    if (MX) {
+      ok = mbar_wait(sf_ready, 0, abort_flag);
+      tc_fence_after();
+    }
+    for (int kb = 0; ok && kb < steps; ++kb) {
       const int stage = kb % NST;
       if (!mbar_wait(&full[stage], (kb / NST) & 1, abort_flag)) {
         ok = false;
@@ -192,7 +245,10 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
                                    : sdesc_sw128(sa + ah * 16384 + kk * 32, 16, 1024);
           const uint64_t db = B_MN ? sdesc_sw128(sb + bh * (BN / 64) * 8192 + kk * 2048, 8192, 1024)
                                    : sdesc_sw128(sb + bh * BN * 128 + kk * 32, 16, 1024);
-          if (F8)
+          if (MX)  // A scales of K stage kb, byte kk (k_begin is 0: the block-scaled form has no K split)
+            umma_mx(tmem + h * BN, da, db, kIdesc | ((uint32_t)kk << 29),
+                    (tmem + kSfaCol + 4 * kb) | ((uint32_t)kk << 30), tmem + kSfbCol, (kb > 0 || kk > 0) ? 1u : 0u);
+          else if (F8)
             umma_ss_f8(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
           else
             umma_ss(tmem + h * BN, da, db, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
@@ -231,7 +287,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
         tmem_wait_ld();
         if (F8) {
           // per-row and per-column dequantisation scales
-          const float sa = gm < p.M ? __ldg(p.row_scale + gm) : 0.f;
+          const float sa = !p.row_scale ? 1.f : gm < p.M ? __ldg(p.row_scale + gm) : 0.f;
           const float4* sw4 = reinterpret_cast<const float4*>(p.col_scale + col0 + 32 * c);
           const bool cols_in = col0 + 32 * c < p.n_cols[half_n];  // a ragged last tile reads no scale past N
 #pragma unroll
@@ -332,9 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_bf16_kernel(const __grid_con
   gemm_body<A_MN, B_MN, BN, NST, false, WIDE>(p);
 }
 
-template <int BN, int NST, bool WIDE = false>
+template <int BN, int NST, bool WIDE = false, bool MX = false>
 __global__ void __launch_bounds__(kThreads, 1) gemm_e4m3_kernel(const __grid_constant__ Params p) {
-  gemm_body<false, false, BN, NST, true, WIDE>(p);
+  gemm_body<false, false, BN, NST, true, WIDE, MX>(p);
 }
 
 // Output maps for the TMA epilogue: c[0] has inner0 columns, c[1] inner1, both
@@ -350,10 +406,10 @@ static bool set_out_maps(Params& p, bool f32, int64_t rows, int64_t ld, int64_t 
   return true;
 }
 
-template <int BN, int NST, bool WIDE = false>
+template <int BN, int NST, bool WIDE = false, bool MX = false>
 static ispa_status_t launch_e4m3(const Params& p, cudaStream_t stream) {
   using L = Layout<BN, NST, WIDE>;
-  auto kern = gemm_e4m3_kernel<BN, NST, WIDE>;
+  auto kern = gemm_e4m3_kernel<BN, NST, WIDE, MX>;
   if (p.n_split < p.N && p.n_split % L::kCols) return unsupported("GEMM column ranges must start on a tile");
   ispa_status_t st = set_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (st != ISPA_OK) return st;
@@ -591,6 +647,42 @@ ispa_status_t project_e4m3(const uint8_t* qa, const float* a_scale, int64_t n_ro
     case ProjTile::kTall256: return launch_e4m3<256, 3>(p, stream);
     default: return launch_e4m3<128, 4>(p, stream);
   }
+}
+
+// y[n_rows, d_out] (bf16) = block-scaled product of MX activation codes
+// qa [n_rows, d_in] with exponent bytes ea [n_rows, d_in / 32] (ue8m0) and the
+// per-channel weight codes qw_t [d_out, d_in] with w_scale [d_out]:
+// y[i, j] = w_scale[j] * sum_b 2^(ea[i, b] - 127) sum_{k in b} qa[i, k] qw[k, j].
+ispa_status_t project_mx(const uint8_t* qa, const uint8_t* ea, int64_t n_rows, int64_t d_in, const uint8_t* qw_t,
+                         const float* w_scale, int64_t d_out, void* y, cudaStream_t stream) {
+  using namespace gemm;
+  if (d_in % kBK8 || d_in / kBK8 > kMxMaxStages)
+    return unsupported("block-scaled projection needs d_in to be a multiple of 128 up to %d (got %lld)",
+                       kMxMaxStages * kBK8, (long long)d_in);
+  if (d_out % 128) return unsupported("block-scaled projection needs d_out %% 128 == 0 (got %lld)", (long long)d_out);
+  Params p;
+  memset(&p, 0, sizeof(p));
+  if (!encode_map_u8_2d(&p.a_map[0], qa, d_in, n_rows, d_in, kBK8, 128)) return ISPA_ERR_CUDA;
+  if (!encode_map_u8_2d(&p.b_map[0][0], qw_t, d_in, d_out, d_in, kBK8, 192)) return ISPA_ERR_CUDA;
+  p.b_map[1][0] = p.b_map[0][0];
+  p.M = (int32_t)n_rows;
+  p.N = (int32_t)d_out;
+  p.K = (int32_t)d_in;
+  p.n_split = (int32_t)d_out;
+  p.n_pairs = 1;
+  p.n_cols[0] = (int32_t)d_out;
+  p.k_per_split = (int32_t)d_in;
+  p.c[0] = y;
+  p.c[1] = y;
+  p.ldc = d_out;
+  p.mode = kStoreBf16;
+  p.row_scale = nullptr;
+  p.col_scale = w_scale;
+  p.a_exps = ea;
+  p.exps_ld = (int32_t)(d_in / 32);
+  if (!set_out_maps(p, false, n_rows, d_out, d_out, d_out)) return ISPA_ERR_CUDA;
+  if (!p.c_tma) return unsupported("block-scaled projection needs a 16-byte aligned output");
+  return launch_e4m3<192, 3, true, true>(p, stream);
 }
 
 }  // namespace ispa

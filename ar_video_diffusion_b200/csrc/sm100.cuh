@@ -301,6 +301,47 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Block-scaled e4m3 (MX) product: tcgen05.mma kind::mxf8f6f4 with one ue8m0
+// scale per 32 elements of K for each row of A and each column of B, read
+// from tensor memory.  The scale-factor byte within a 32-bit column is
+// selected by bits 29-30 (A) and 4-5 (B) of the instruction descriptor and
+// carried in the top two bits of the scale addresses too.
+__host__ __device__ constexpr uint32_t idesc_mxf8_f32(int M, int N) {
+  return (1u << 23)  // scale factors are ue8m0; A and B format fields 0 = e4m3, both K-major
+         | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+
+// MX quantisation of one block of 32 values that are exactly bf16: e is the
+// smallest integer with amax * 2^-e <= 448 (0 for an all-zero block, at least
+// -127); the codes are e4m3(x * 2^-e), round to nearest even (the scaling by
+// a power of two is exact).  Writing amax = m 2^E with m in [1, 2), e is
+// E - 8, plus one when m > 1.75 (448 = 1.75 * 2^8).  Returns the biased
+// exponent byte e + 127; the 32 codes go to c[0..7], 4 per word, in order.
+__device__ __forceinline__ uint32_t mx_quantize32(const float (&x)[32], uint32_t (&c)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(x[j]));
+  const uint32_t bits = __float_as_uint(amax);
+  const int ef = (int)(bits >> 23);
+  int e = ef == 0 ? (amax == 0.f ? 0 : -127) : ef - 135 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  e = max(e, -127);
+  const float s = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, a normal float for e in [-127, 121]
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    c[j] = (uint32_t)cvt_e4m3x2(x[4 * j] * s, x[4 * j + 1] * s) |
+           ((uint32_t)cvt_e4m3x2(x[4 * j + 2] * s, x[4 * j + 3] * s) << 16);
+  return (uint32_t)(e + 127);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
   return *reinterpret_cast<uint32_t*>(&v);

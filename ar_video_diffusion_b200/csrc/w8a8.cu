@@ -11,6 +11,9 @@
 //   * both divisions are IEEE fp32;
 //   * the weight codes are written transposed, [D_out, D_in], so both operands
 //     of the tensor-core product are K-major.
+// Block-scaled (MX) activation codes: one power-of-two scale per 32
+// consecutive elements of a row (see mx_quantize32), for the block-scaled
+// tensor-core product.
 // Both kernels are HBM-bound streams with 16-byte loads and stores.
 #include "internal.h"
 #include "sm100.cuh"
@@ -160,7 +163,47 @@ __global__ void __launch_bounds__(256) weight_codes_t_kernel(const __nv_bfloat16
   }
 }
 
+// MX codes of activation rows: one thread per block of 32 consecutive
+// elements of a row (64 bytes read as four 16-byte vectors, 32 code bytes
+// written as two, one exponent byte), consecutive threads on consecutive
+// blocks of a row, so every access of a warp is contiguous.
+__global__ void __launch_bounds__(256) mx_quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t n_rows,
+                                                               int K, int64_t stride, uint8_t* __restrict__ q,
+                                                               uint8_t* __restrict__ e) {
+  const int nb = K / 32;
+  const int64_t total = n_rows * nb;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / nb;
+    const int b = (int)(i - row * nb);
+    const uint4* src = reinterpret_cast<const uint4*>(x + row * stride + 32 * b);
+    float f[32];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      float g[8];
+      bf16x8(__ldg(src + v), g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[8 * v + j] = g[j];
+    }
+    uint32_t c[8];
+    e[i] = (uint8_t)mx_quantize32(f, c);
+    uint4* dst = reinterpret_cast<uint4*>(q + row * K + 32 * b);
+    dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+    dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+  }
+}
+
 }  // namespace w8a8
+
+ispa_status_t mx_quantize_rows_e4m3(const void* x, int64_t n_rows, int64_t K, int64_t stride, uint8_t* q, uint8_t* e,
+                                    cudaStream_t stream) {
+  const int64_t want = (n_rows * (K / 32) + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  const int blocks = (int)(want < cap ? want : cap);
+  if (blocks == 0) return ISPA_OK;
+  w8a8::mx_quantize_rows_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), n_rows, (int)K,
+                                                            stride, q, e);
+  return check_launch("mx_quantize_rows_kernel");
+}
 
 ispa_status_t quantize_rows_e4m3(const void* x, int64_t n_rows, int64_t K, int64_t stride, uint8_t* q, float* scale,
                                  cudaStream_t stream) {

@@ -33,7 +33,8 @@ EXPORTED = ("ispa_dual_attention", "ispa_lse_merge", "ispa_gram_accumulate", "is
             "ispa_layer_error_workspace_bytes", "ispa_layer_error", "ispa_select_layers", "ispa_absorb_workspace_bytes",
             "ispa_absorb_solve", "ispa_absorb_solve_noalloc", "ispa_project", "ispa_local_attention_project",
             "ispa_quantize_e4m3_rows", "ispa_quantize_e4m3_weight", "ispa_project_w8a8",
-            "ispa_local_attention_project_w8a8",
+            "ispa_local_attention_project_w8a8", "ispa_mx_quantize_e4m3_rows", "ispa_project_mx",
+            "ispa_local_attention_project_mx",
             "ispa_chunk_token_ranges", "ispa_kv_bytes", "ispa_selftest_wait_timeout", "ispa_status_string", "ispa_last_error",
             "ispa_version")
 
@@ -82,6 +83,10 @@ def lib() -> ctypes.CDLL:
             "ispa_project_w8a8": (i32, [vp, vp, i64, i64, vp, vp, i64, vp, vp]),
             "ispa_local_attention_project_w8a8": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp,
                                                         vp, vp, vp, vp, vp]),
+            "ispa_mx_quantize_e4m3_rows": (i32, [vp, i64, i64, i64, i32, vp, vp, vp]),
+            "ispa_project_mx": (i32, [vp, vp, i64, i64, vp, vp, i64, vp, vp]),
+            "ispa_local_attention_project_mx": (i32, [vp, i64, i64, i32, i32, i32, f32, seg_p, i32, vp, vp, vp,
+                                                      vp, vp, vp, vp]),
             "ispa_chunk_token_ranges": (i32, [i64, i64, i64, i64, c.POINTER(i64)]),
             "ispa_kv_bytes": (i64, [i64, i32, c.c_uint64, i32, i64, i64, i64, i32, i64]),
             "ispa_selftest_wait_timeout": (i32, [c.c_uint32, vp, vp]),
@@ -220,6 +225,23 @@ def ispa_local_attention_project_w8a8(q, n_q, q_stride, n_heads, head_dim, dt, s
     _check(lib().ispa_local_attention_project_w8a8(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local,
                                                    n_local, w_codes_t, w_scales, y, a_loc_out, a_codes, a_scales,
                                                    dev_status, stream), "ispa_local_attention_project_w8a8")
+
+
+def ispa_mx_quantize_e4m3_rows(x, n_rows, k, row_stride, dt, codes, exps, stream):
+    _check(lib().ispa_mx_quantize_e4m3_rows(x, n_rows, k, row_stride, dt, codes, exps, stream),
+           "ispa_mx_quantize_e4m3_rows")
+
+
+def ispa_project_mx(a_codes, a_exps, n_rows, d_in, w_codes_t, w_scales, d_out, y, stream):
+    _check(lib().ispa_project_mx(a_codes, a_exps, n_rows, d_in, w_codes_t, w_scales, d_out, y, stream),
+           "ispa_project_mx")
+
+
+def ispa_local_attention_project_mx(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local, n_local,
+                                    w_codes_t, w_scales, y, a_codes, a_exps, dev_status, stream):
+    _check(lib().ispa_local_attention_project_mx(q, n_q, q_stride, n_heads, head_dim, dt, softmax_scale, local,
+                                                 n_local, w_codes_t, w_scales, y, a_codes, a_exps, dev_status,
+                                                 stream), "ispa_local_attention_project_mx")
 
 
 def ispa_chunk_token_ranges(chunk: int, frame_tokens: int, chunk_frames: int, sink_frames: int = 1):
@@ -444,4 +466,52 @@ def local_attention_project_w8a8(q: torch.Tensor, local: Sequence[Tuple[torch.Te
                                       _dev(w_scales, "w_scales"), _dev(out["y"], "y"), _dev(out["a_loc"], "a_loc"),
                                       _dev(out["a_codes"], "a_codes"), _dev(out["a_scales"], "a_scales"),
                                       _dev(status, "status"), _stream(stream))
+    return out
+
+
+def mx_quantize_e4m3_rows(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                          exps: Optional[torch.Tensor] = None, stream=None):
+    """MX e4m3 codes (uint8 [n, k]) and block exponent bytes (uint8
+    [n, k / 32], ue8m0: e + 127) of bf16 x [n, k]."""
+    n, k = x.shape
+    if codes is None:
+        codes = torch.empty(n, k, dtype=torch.uint8, device=x.device)
+    if exps is None:
+        exps = torch.empty(n, k // 32, dtype=torch.uint8, device=x.device)
+    ispa_mx_quantize_e4m3_rows(_dev(x, "x"), n, k, _row_stride(x, "x"), _dtype_code(x), _dev(codes, "codes"),
+                               _dev(exps, "exps"), _stream(stream))
+    return codes, exps
+
+
+def project_mx(a_codes: torch.Tensor, a_exps: torch.Tensor, w_codes_t: torch.Tensor, w_scales: torch.Tensor,
+               y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 y [n, d_out] of the block-scaled projection of MX activation codes
+    by per-channel weight codes."""
+    n, d_in = a_codes.shape
+    d_out = w_codes_t.shape[0]
+    if y is None:
+        y = torch.empty(n, d_out, dtype=torch.bfloat16, device=a_codes.device)
+    ispa_project_mx(_dev(a_codes, "a_codes"), _dev(a_exps, "a_exps"), n, d_in, _dev(w_codes_t, "w_codes_t"),
+                    _dev(w_scales, "w_scales"), d_out, _dev(y, "y"), _stream(stream))
+    return y
+
+
+def local_attention_project_mx(q: torch.Tensor, local: Sequence[Tuple[torch.Tensor, torch.Tensor]],
+                               w_codes_t: torch.Tensor, w_scales: torch.Tensor, n_heads: int,
+                               softmax_scale: float = 0.0, out: Optional[dict] = None,
+                               status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """L-layer with the MX projection: local attention whose epilogue writes
+    MX codes of A_loc -> block-scaled product.  Returns {"y", "a_codes",
+    "a_exps"}."""
+    n_q, D = q.shape
+    if out is None:
+        dev = q.device
+        out = {"y": torch.empty(n_q, D, dtype=torch.bfloat16, device=dev),
+               "a_codes": torch.empty(n_q, D, dtype=torch.uint8, device=dev),
+               "a_exps": torch.empty(n_q, D // 32, dtype=torch.uint8, device=dev)}
+    ls, nl = _segments(local)
+    ispa_local_attention_project_mx(_dev(q, "q"), n_q, _row_stride(q, "q"), n_heads, D // n_heads,
+                                    _dtype_code(q), softmax_scale, ls, nl, _dev(w_codes_t, "w_codes_t"),
+                                    _dev(w_scales, "w_scales"), _dev(out["y"], "y"), _dev(out["a_codes"], "a_codes"),
+                                    _dev(out["a_exps"], "a_exps"), _dev(status, "status"), _stream(stream))
     return out

@@ -20,7 +20,9 @@ section 2):
     whole growing cache and project with W.  With ``precision="w8a8"`` the
     L-layers project with the post-training W8A8 reading of the same page's
     "Speedup" item: W_new quantised to e4m3 once, after the absorb, and each
-    chunk's A_loc quantised per token.
+    chunk's A_loc quantised per token; with ``precision="mx"`` the attention
+    epilogue writes A_loc as MX codes (one power-of-two scale per 32
+    channels) and the L-layer runs the block-scaled product.
 Chunk 0 holds the sink frame inside its own current chunk, so it has no
 separate sink and no history.  Every step runs in libispa's kernels; this
 module only owns the device buffers (torch tensors), the chunk schedule and the
@@ -57,8 +59,8 @@ class Rollout:
         ``rank_all``: rank every layer (eps of each) even for a fixed set."""
         if selection not in ("fixed", "instance"):
             raise ValueError("selection must be 'fixed' or 'instance'")
-        if precision not in ("bf16", "w8a8"):
-            raise ValueError("precision must be 'bf16' or 'w8a8'")
+        if precision not in ("bf16", "w8a8", "mx"):
+            raise ValueError("precision must be 'bf16', 'w8a8' or 'mx'")
         self.precision = precision
         self.w8: Dict[int, tuple] = {}  # L-layer -> (e4m3 codes of W_new, transposed; per-channel scales)
         self.w = w
@@ -113,6 +115,9 @@ class Rollout:
             self.w8_out = {"y": self.y, "a_loc": self.out["a_loc"],
                            "a_codes": torch.empty(n_q, D, dtype=torch.uint8, device=self.device),
                            "a_scales": torch.empty(n_q, dtype=torch.float32, device=self.device)}
+        elif precision == "mx":
+            self.w8_out = {"y": self.y, "a_codes": torch.empty(n_q, D, dtype=torch.uint8, device=self.device),
+                           "a_exps": torch.empty(n_q, D // 32, dtype=torch.uint8, device=self.device)}
         self.status = ispa.new_status(self.device)
         self.workspace = ispa.absorb_workspace(D, self.device)
         self.reports: List[ChunkReport] = []
@@ -202,7 +207,7 @@ class Rollout:
             k_small[:sink].copy_(self.k[l][:sink])
             v_small[:sink].copy_(self.v[l][:sink])
             self.k[l], self.v[l] = k_small, v_small
-        if self.precision == "w8a8":
+        if self.precision in ("w8a8", "mx"):
             for l in self.absorbed:
                 self.w8[l] = ispa.quantize_e4m3_weight(self.W_new[l])
         torch.cuda.synchronize(self.device)
@@ -229,6 +234,10 @@ class Rollout:
                     qwt, sw = self.w8[l]
                     ispa.local_attention_project_w8a8(self.q[l], local, qwt, sw, H, out=self.w8_out,
                                                       status=self.status)
+                elif self.precision == "mx":
+                    qwt, sw = self.w8[l]
+                    ispa.local_attention_project_mx(self.q[l], local, qwt, sw, H, out=self.w8_out,
+                                                    status=self.status)
                 else:
                     ispa.local_attention_project(self.q[l], local, self.W_new[l], H, y=self.y,
                                                  a_loc=self.out["a_loc"], status=self.status)

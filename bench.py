@@ -504,18 +504,20 @@ def run_rollout(device) -> dict:
     }
     del ro
     torch.cuda.empty_cache()
-    res["w8a8"] = run_rollout_w8a8(device, res)
+    res["w8a8"] = run_rollout_w8a8(device, res, "w8a8")
+    res["mx"] = run_rollout_w8a8(device, res, "mx")
     res["layer_selection"] = run_layer_selection(device)
     return res
 
 
-def run_rollout_w8a8(device, bf16_res: dict) -> dict:
+def run_rollout_w8a8(device, bf16_res: dict, precision: str) -> dict:
     """The same rollout with W8A8 L-layers (W_new quantised to e4m3 once after
-    the absorb, A_loc per token every chunk), post-transition chunks timed
-    the same way as the bf16 rollout's."""
+    the absorb; A_loc per token every chunk, or with precision "mx" as MX
+    codes from the attention epilogue), post-transition chunks timed the same
+    way as the bf16 rollout's."""
     from ar_video_diffusion_b200.rollout import Rollout
     w = synth.WORKLOADS["rollout"]
-    ro = Rollout(w, device=device, precision="w8a8")
+    ro = Rollout(w, device=device, precision=precision)
     reps = ro.run()
     post = [r for r in reps if r.phase == "post"]
     g_first = ro.chunk_graph_ms(w.warm_chunks)
@@ -524,7 +526,8 @@ def run_rollout_w8a8(device, bf16_res: dict) -> dict:
         raise RuntimeError("device status during the W8A8 rollout")
     del ro
     torch.cuda.empty_cache()
-    return {"workload": "the rollout above with W8A8 L-layers (e4m3 W_new per output channel, A_loc per token)",
+    form = "A_loc per token" if precision == "w8a8" else "A_loc as MX codes written by the attention epilogue"
+    return {"workload": f"the rollout above with W8A8 L-layers (e4m3 W_new per output channel, {form})",
             "post_chunk_ms_first": round(post[0].gpu_ms, 3), "post_chunk_ms_last": round(post[-1].gpu_ms, 3),
             "post_chunk_graph_ms_first": round(g_first, 3), "post_chunk_graph_ms_last": round(g_last, 3),
             "speedup_vs_bf16_graph_first": round(bf16_res["post_chunk_graph_ms_first"] / g_first, 4),
@@ -799,11 +802,38 @@ def _graph_ms(fn, device, iters) -> float:
     return e0.elapsed_time(e1) / (iters * COMP_REPS)
 
 
+def _graph_ms_flushed(fn, device, iters) -> float:
+    """Device time of one call of fn, captured once into a graph; before each
+    of the iters replays a 256 MB buffer is written, so no operand is left in
+    the 126 MB L2 by the previous replay.  Mean over the replays."""
+    side = torch.cuda.Stream(device)
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    fn()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        fn()
+    g.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+
+
 def w8a8_bench(ispa, w, device, peak_bf16: float, peak_hbm: float, iters=20) -> dict:
-    """The W8A8 variant of the post-transition L-layer (e4m3 projection with
-    per-token and per-output-channel scales) against the bf16 L-layer, both
-    timed as CUDA-graph replays on the same inputs.  The fp8 peak is the
-    measured bf16 peak times the nominal fp8 / bf16 ratio of 2."""
+    """The W8A8 variants of the post-transition L-layer against the bf16
+    L-layer on the same inputs: per-token (attention -> bf16 A_loc -> e4m3
+    codes -> e4m3 product) and MX (the attention epilogue writes e4m3 codes
+    with a power-of-two scale per 32 channels -> block-scaled product).  The
+    L-layers are timed with L2 flushed before every replay (their inputs,
+    52.8 MB, fit in L2); the single kernels as back-to-back graph replays.
+    The fp8 peak is the measured bf16 peak times the nominal fp8 / bf16 ratio
+    of 2."""
     H, D, n = w.n_heads, w.d_model, w.n_q
     x = synth.single_layer_inputs(w, 1)
 
@@ -820,12 +850,18 @@ def w8a8_bench(ispa, w, device, peak_bf16: float, peak_hbm: float, iters=20) -> 
     out8 = ispa.local_attention_project_w8a8(q, local, qwt, sw, H, status=status)
     ispa.local_attention_project(q, local, W, H, y=y16, a_loc=a16, status=status)
     qa, sa = ispa.quantize_e4m3_rows(a16)
+    outmx = ispa.local_attention_project_mx(q, local, qwt, sw, H, status=status)
+    mq, me = ispa.mx_quantize_e4m3_rows(a16)
     yp = torch.empty(n, D, dtype=torch.bfloat16, device=device)
     ms = {
-        "l_layer_w8a8": _graph_ms(lambda: ispa.local_attention_project_w8a8(q, local, qwt, sw, H, out=out8,
-                                                                            status=status), device, iters),
-        "l_layer_bf16": _graph_ms(lambda: ispa.local_attention_project(q, local, W, H, y=y16, a_loc=a16,
-                                                                       status=status), device, iters),
+        "l_layer_w8a8": _graph_ms_flushed(lambda: ispa.local_attention_project_w8a8(q, local, qwt, sw, H, out=out8,
+                                                                                    status=status), device, iters),
+        "l_layer_mx": _graph_ms_flushed(lambda: ispa.local_attention_project_mx(q, local, qwt, sw, H, out=outmx,
+                                                                                status=status), device, iters),
+        "l_layer_bf16": _graph_ms_flushed(lambda: ispa.local_attention_project(q, local, W, H, y=y16, a_loc=a16,
+                                                                               status=status), device, iters),
+        "project_mx": _graph_ms(lambda: ispa.project_mx(mq, me, qwt, sw, yp), device, iters),
+        "mx_quantize_rows": _graph_ms(lambda: ispa.mx_quantize_e4m3_rows(a16, mq, me), device, iters),
         "project_w8a8": _graph_ms(lambda: ispa.project_w8a8(qa, sa, qwt, sw, yp), device, iters),
         "project_bf16": _graph_ms(lambda: ispa.project(a16, W, yp), device, iters),
         "quantize_rows": _graph_ms(lambda: ispa.quantize_e4m3_rows(a16, qa, sa), device, iters),
@@ -838,12 +874,18 @@ def w8a8_bench(ispa, w, device, peak_bf16: float, peak_hbm: float, iters=20) -> 
     pk8 = 2.0 * peak_bf16
     q_bytes = n * D * 2 + n * D + n * 4
     diff = (out8["y"].float() - y16.float()).norm() / y16.float().norm()
+    diff_mx = (outmx["y"].float() - y16.float()).norm() / y16.float().norm()
     return {
         "workload": "wan1.3b L-layer: local attention (4680 queries, 6240 keys) + y = A_loc W_new, "
-                    "W8A8 = e4m3 codes, per-token and per-output-channel fp32 scales",
+                    "W8A8 = e4m3 codes; W_new per output channel, A_loc per token or (MX) per 32 channels",
+        "timing": "l_layer_*: L2 flushed before each replay; single kernels: back-to-back graph replays",
         "ms": {k: round(v, 4) for k, v in ms.items()},
         "project_w8a8_tflops": round(flops / (ms["project_w8a8"] * 1e-3) / 1e12, 1),
         "project_w8a8_frac_of_fp8_peak": round(flops / (ms["project_w8a8"] * 1e-3) / 1e12 / pk8, 4),
+        "project_mx_tflops": round(flops / (ms["project_mx"] * 1e-3) / 1e12, 1),
+        "project_mx_frac_of_fp8_peak": round(flops / (ms["project_mx"] * 1e-3) / 1e12 / pk8, 4),
+        "l_layer_mx_speedup_vs_bf16": round(ms["l_layer_bf16"] / ms["l_layer_mx"], 4),
+        "y_rel_diff_mx_vs_bf16": round(float(diff_mx), 5),
         "fp8_peak_tflops": round(pk8, 1),
         "quantize_rows_gbs": round(q_bytes / (ms["quantize_rows"] * 1e-3) / 1e9, 1),
         "quantize_rows_frac_of_hbm": round(q_bytes / (ms["quantize_rows"] * 1e-3) / 1e9 / peak_hbm, 4),

@@ -327,6 +327,55 @@ ISPA_API ispa_status_t ispa_local_attention_project_w8a8(const void* q, int64_t 
                                                          uint8_t* a_codes, float* a_scales, int32_t* dev_status,
                                                          void* stream);
 
+/* ------------------------------------------------------- W8A8, MX form --
+ * The same W8A8 projection with block-scaled (MX) activation codes, which
+ * the attention epilogue can write itself: a CTA there holds one head's
+ * channels of a row, so it can scale blocks of 32 consecutive channels but not
+ * a whole row.  Source as above (section 4, "Speedup"); this library's
+ * reading of the MX form:
+ *   - each block of 32 consecutive elements of an activation row has one
+ *     power-of-two scale 2^e, e the smallest integer with amax * 2^-e <= 448
+ *     (0 for an all-zero block, at least -127), stored as the ue8m0 byte
+ *     e + 127;
+ *   - code = e4m3(x * 2^-e), round to nearest even (the scaling is exact);
+ *     the activations quantised are the bf16 values;
+ *   - the weight keeps the per-output-channel codes and fp32 scales of
+ *     ispa_quantize_e4m3_weight;
+ *   - y[i, j] = s_w[j] * sum over blocks b of 2^(e[i, b])
+ *     * sum over k in b of dec(qa[i, k]) * dec(qw[k, j]), fp32 accumulation
+ *     (kind::mxf8f6f4 block-scaled tensor-core MMAs), bf16 output.
+ * All pointers are device pointers owned by the caller.  Nothing allocates;
+ * everything runs asynchronously on `stream`.
+ *
+ * ispa_mx_quantize_e4m3_rows:
+ *   - x [n_rows, k] bf16, row_stride elements apart;
+ *   - codes [n_rows, k] bytes, dense; exps [n_rows, k / 32] bytes, dense;
+ *   - k must be a multiple of 32; x, its rows and codes 16-byte aligned.
+ * ispa_project_mx:
+ *   - y [n_rows, d_out] bf16 from a_codes [n_rows, d_in], a_exps
+ *     [n_rows, d_in / 32], w_codes_t [d_out, d_in] and w_scales [d_out];
+ *   - d_in a multiple of 128 and at most 3584 (the scales of a 128-row tile
+ *     live in tensor memory beside its accumulators), d_out % 128 == 0;
+ *   - codes, w_scales and y 16-byte aligned, a_exps 4-byte aligned.
+ * ispa_local_attention_project_mx: the L-layer of ispa_local_attention_project
+ * with the MX projection.  The single-pass local attention writes the MX codes
+ * and exponents of A_loc (a_codes [n_q, D], a_exps [n_q, D / 32]) from its
+ * epilogue instead of bf16 A_loc, then the block-scaled product with the
+ * quantised W_new runs.  D = n_heads * head_dim as in ispa_project_mx.
+ * Errors as for the W8A8 calls above; nothing is launched on an error.
+ */
+ISPA_API ispa_status_t ispa_mx_quantize_e4m3_rows(const void* x, int64_t n_rows, int64_t k, int64_t row_stride,
+                                                  ispa_dtype_t dt, uint8_t* codes, uint8_t* exps, void* stream);
+ISPA_API ispa_status_t ispa_project_mx(const uint8_t* a_codes, const uint8_t* a_exps, int64_t n_rows, int64_t d_in,
+                                       const uint8_t* w_codes_t, const float* w_scales, int64_t d_out, void* y,
+                                       void* stream);
+ISPA_API ispa_status_t ispa_local_attention_project_mx(const void* q, int64_t n_q, int64_t q_stride,
+                                                       int32_t n_heads, int32_t head_dim, ispa_dtype_t dt,
+                                                       float softmax_scale, const ispa_kv_segment_t* local,
+                                                       int32_t n_local, const uint8_t* w_codes_t,
+                                                       const float* w_scales, void* y, uint8_t* a_codes,
+                                                       uint8_t* a_exps, int32_t* dev_status, void* stream);
+
 /* ------------------------------------------------------ host bookkeeping --
  * Streaming bookkeeping of [gist §2.1, §2.3], host-only and exact (integers).
  *

@@ -189,3 +189,32 @@ def project_mxfp8(a, w) -> np.ndarray:
     qa, ea = mx_quantize_rows(a)
     qw, ew = mx_quantize_cols(w)
     return mx_project_codes(qa, ea, qw, ew)
+
+
+# ---------------------------------------------------------------------------
+# MX activations against per-channel weights: the form the tensor-core
+# product takes when the attention epilogue writes the codes.  Activation
+# rows carry one power-of-two scale per 32-element block (mx_quantize_rows),
+# the weights the per-output-channel fp32 scale of quantize_cols (one scale
+# per column of a K-major weight code matrix, applied after the sum):
+#   y[i, j] = s_w[j] * sum over blocks b of 2^ea[i, b]
+#             * sum over k in b of dec(qa[i, k]) * dec(qw[k, j]).
+# The block exponents are stored biased by 127 (the ue8m0 byte) by the GPU
+# path; here they are plain integers.
+def mx_rows_project_codes(qa, ea, qw, sw) -> np.ndarray:
+    """y from MX activation codes and per-channel weight codes (fp64)."""
+    n, K = qa.shape
+    y = np.zeros((n, qw.shape[1]))
+    da, dw = e4m3_decode(qa), e4m3_decode(qw)
+    for b in range(K // MX_BLOCK):
+        ks = slice(b * MX_BLOCK, (b + 1) * MX_BLOCK)
+        y += np.ldexp(da[:, ks] @ dw[ks, :], np.asarray(ea)[:, b][:, None])
+    return y * np.asarray(sw, dtype=np.float64)[None, :]
+
+
+def project_mx_rows(a, w) -> np.ndarray:
+    """The projection of a [n, K] by w [K, N] with MX activation rows and
+    per-channel weight scales."""
+    qa, ea = mx_quantize_rows(a)
+    qw, sw = quantize_cols(w)
+    return mx_rows_project_codes(qa, ea, qw, sw)

@@ -99,9 +99,10 @@ def absorb_chain_sensitivity(w: synth.Workload, layers, seed: int = 0, rows_per_
     return out
 
 
-def w8a8_chain_sensitivity(draws: int = 3, n_rows: int = 48, seed: int = 1) -> list:
+def w8a8_chain_sensitivity(draws: int = 3, n_rows: int = 48, seed: int = 1, project=w8.project_w8a8) -> list:
     """W8A8 L-layer of the Wan-1.3B shapes on sampled rows: relative Frobenius
-    error and largest element error / max|y| of the e4m3 projection when A_loc
+    error and largest element error / max|y| of the e4m3 projection (the
+    per-token form, or with project=w8.project_mx_rows the MX form) when A_loc
     carries the GPU-like perturbation before its bf16 rounding."""
     w = synth.WORKLOADS["wan1.3b"]
     x = synth.single_layer_inputs(w, 1)
@@ -110,12 +111,12 @@ def w8a8_chain_sensitivity(draws: int = 3, n_rows: int = 48, seed: int = 1) -> l
     rows[-1] = w.n_q - 1
     a_ref, _ = orc.attention(x["q"][rows], np.concatenate([x["k_sink"], x["k_cur"]]),
                              np.concatenate([x["v_sink"], x["v_cur"]]), w.n_heads)
-    y_ref = w8.project_w8a8(synth.round_bf16(a_ref.astype(np.float32)), W)
+    y_ref = project(synth.round_bf16(a_ref.astype(np.float32)), W)
     rng = np.random.default_rng(seed)
     out = []
     for _ in range(draws):
         an = a_ref * (1 + NOISE * rng.standard_normal(a_ref.shape))
-        y = synth.round_bf16(w8.project_w8a8(synth.round_bf16(an.astype(np.float32)), W).astype(np.float32))
+        y = synth.round_bf16(project(synth.round_bf16(an.astype(np.float32)), W).astype(np.float32))
         out.append({"fro": float(np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref)),
                     "max": float(np.max(np.abs(y - y_ref)) / np.max(np.abs(y_ref)))})
     return out
@@ -128,8 +129,10 @@ def main():
     for r in absorb_chain_sensitivity(synth.WORKLOADS["rollout_small"], [0, 1, 2, 3]):
         print(f"rollout_small layer {r['layer']}: {r['rows']} rows, dW moves {r['dw_rel']:.2e}, "
               f"eps {r['eps']:.4f} moves {r['eps_rel']:.2e} (relative)")
-    for i, r in enumerate(w8a8_chain_sensitivity()):
-        print(f"W8A8 L-layer draw {i}: y relative Frobenius {r['fro']:.2e}, largest element {r['max']:.2e}")
+    for name, proj in (("per-token", w8.project_w8a8), ("MX", w8.project_mx_rows)):
+        for i, r in enumerate(w8a8_chain_sensitivity(project=proj)):
+            print(f"W8A8 ({name}) L-layer draw {i}: y relative Frobenius {r['fro']:.2e}, "
+                  f"largest element {r['max']:.2e}")
     if args.full:
         for r in absorb_chain_sensitivity(synth.WORKLOADS["rollout"], [0]):
             print(f"rollout (1.3B shapes) layer {r['layer']}: {r['rows']} rows, dW moves {r['dw_rel']:.2e}, "

@@ -19,8 +19,10 @@ def test_absorb_chain_bounds_cover_the_simulated_perturbation():
         assert 0 < r["eps_rel"] and MARGIN * r["eps_rel"] <= CHAIN_EPS_REL, r
 
 
-def test_w8a8_chain_bounds_cover_the_simulated_perturbation():
-    res = ct.w8a8_chain_sensitivity()
+@pytest.mark.parametrize("form", ["per-token", "mx"])
+def test_w8a8_chain_bounds_cover_the_simulated_perturbation(form):
+    from oracle import w8a8_oracle as w8
+    res = ct.w8a8_chain_sensitivity(project=w8.project_w8a8 if form == "per-token" else w8.project_mx_rows)
     for r in res:
         assert 0 < r["fro"] and MARGIN * r["fro"] <= CHAIN_W8A8_FRO, r
         assert 0 < r["max"] and MARGIN * r["max"] <= CHAIN_W8A8_MAX, r

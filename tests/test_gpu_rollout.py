@@ -193,19 +193,22 @@ def test_full_size_rollout_absorbed_layers_against_the_oracle_chain():
     assert other["mode"] == "F" and other["k_hist"].shape[0] == (w.warm_chunks * w.chunk_frames - 1) * w.frame_tokens
 
 
-def test_small_rollout_w8a8_l_layers_against_the_oracle_chain():
+@pytest.mark.parametrize("precision", ["w8a8", "mx"])
+def test_small_rollout_w8a8_l_layers_against_the_oracle_chain(precision):
     """The small rollout with W8A8 L-layers: after the absorb, W_new is
     quantised once (e4m3, per output channel) and every post-transition chunk
-    quantises A_loc per token before the e4m3 projection.  Expected values: the
-    oracle's own chain (its dW from its own dual stream over the warm-up rows),
-    then its W8A8 reading of y = A_loc W_new; bounds CHAIN_W8A8_FRO / _MAX
-    (tests/chain_tolerances.py)."""
+    quantises A_loc (per token, or per 32-channel block in the MX form written
+    by the attention epilogue) before the e4m3 projection.  Expected values:
+    the oracle's own chain (its dW from its own dual stream over the warm-up
+    rows), then its W8A8 reading of y = A_loc W_new; bounds CHAIN_W8A8_FRO /
+    _MAX (tests/chain_tolerances.py, which simulates both forms)."""
     from oracle import w8a8_oracle as w8
     from helpers import CHAIN_W8A8_FRO, CHAIN_W8A8_MAX
     w = synth.WORKLOADS["rollout_small"]
     absorbed = [0, 2]
     inputs = {}
-    ro = Rollout(w, absorbed=absorbed, on_layer=capture_inputs(w, inputs), precision="w8a8")
+    ro = Rollout(w, absorbed=absorbed, on_layer=capture_inputs(w, inputs), precision=precision)
+    project = w8.project_w8a8 if precision == "w8a8" else w8.project_mx_rows
     reports = ro.run()
     _check_bookkeeping(w, ro, reports, absorbed)
     W = {l: host(ro.W[l]) for l in range(w.n_layers)}
@@ -221,9 +224,9 @@ def test_small_rollout_w8a8_l_layers_against_the_oracle_chain():
             continue
         n_l += 1
         a, _ = orc.attention(x["q"], x["k_loc"], x["v_loc"], w.n_heads)
-        y_ref = w8.project_w8a8(synth.round_bf16(a.astype(np.float32)), W_new_ref[l])
+        y_ref = project(synth.round_bf16(a.astype(np.float32)), W_new_ref[l])
         err = fro_rel(x["y"], y_ref)
-        REPORT.append((f"small rollout W8A8 chain: y of layer {l} chunk {c} (relative Frobenius)", err, err))
+        REPORT.append((f"small rollout {precision} chain: y of layer {l} chunk {c} (relative Frobenius)", err, err))
         assert err <= CHAIN_W8A8_FRO, (l, c, err)
         assert np.max(np.abs(x["y"] - y_ref)) <= CHAIN_W8A8_MAX * np.max(np.abs(y_ref)), (l, c)
     assert n_l == len(absorbed) * w.post_chunks

@@ -158,3 +158,102 @@ def test_local_attention_project_w8a8_wan13b_sampled_rows():
     # the quantised weight is the oracle's, bit for bit
     qw_o, sw_o = w8.quantize_cols(W)
     assert np.array_equal(_u8(qwt), qw_o.T) and np.array_equal(_f32(sw), sw_o)
+
+
+# ---------------------------------------------------------------- MX form
+def _mx_rows_input(rng, n, k):
+    """bf16 rows whose 32-element blocks span many binades, with the edge
+    cases of the exponent rule: an all-zero block, a block whose largest
+    magnitude has mantissa exactly 1.75 (448 * 2^j: no carry), one just
+    above, and one of bf16 subnormals."""
+    x = _bf16(rng, (n, k)) * np.exp2(rng.integers(-20, 20, (n, k // 32))).repeat(32, 1).astype(np.float32)
+    x = synth.round_bf16(x.astype(np.float32))
+    if n > 4 and k >= 128:
+        x[0, 0:32] = 0.0
+        x[1, 32:64] = np.float32(0.5)
+        x[1, 40] = np.float32(-448.0 * 2.0 ** -5)
+        x[2, 64:96] = np.float32(0.25)
+        x[2, 70] = synth.round_bf16(np.array([448.0 * 2.0 ** -3 * (1 + 2.0 ** -7)], np.float32))[0]
+        x[3, 96:128] = np.float32(2.0 ** -130)
+    return x
+
+
+@pytest.mark.parametrize("n,k,pad", [(4680, 1536, 0), (300, 256, 32), (1, 32, 0), (77, 5120, 0)])
+def test_mx_quantize_rows_bit_exact(n, k, pad):
+    rng = np.random.default_rng(3 * n + k)
+    x = _mx_rows_input(rng, n, k)
+    xd = torch.zeros(n, k + pad, dtype=torch.bfloat16, device="cuda")
+    xd[:, :k] = dev(x, "bf16")
+    codes, exps = ispa.mx_quantize_e4m3_rows(xd[:, :k])
+    torch.cuda.synchronize()
+    qo, eo = w8.mx_quantize_rows(x)
+    assert np.array_equal(_u8(exps).astype(np.int64) - 127, eo)
+    assert np.array_equal(_u8(codes), qo)
+
+
+def _check_mx_projection(y, qa, ea, qw, sw):
+    ref = w8.mx_rows_project_codes(qa, ea, qw, sw)
+    mag = w8.mx_rows_project_codes(qa & 0x7F, ea, qw & 0x7F, sw)
+    got = host(y)
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -11 * mag + 1e-30
+    err = np.abs(got - ref)
+    assert np.all(err <= bound), float(np.max(err / bound))
+    assert fro_rel(got, ref) <= 4e-3
+
+
+# (4680, 1536, 1536): the wan1.3b L-layer; (517, 1536, 1280): ragged rows and
+# an overhanging last column tile; (1, 3584, 256): the longest K the tile's
+# scales fit; (129, 128, 128): one K stage
+@pytest.mark.parametrize("n,d_in,d_out", [(4680, 1536, 1536), (517, 1536, 1280), (1, 3584, 256), (129, 128, 128)])
+def test_project_mx_matches_oracle(n, d_in, d_out):
+    rng = np.random.default_rng(n + 3 * d_in + d_out)
+    a = _mx_rows_input(rng, n, d_in)
+    w = _bf16(rng, (d_in, d_out), 1.0 / np.sqrt(d_in))
+    qa, ea = w8.mx_quantize_rows(a)
+    qw, sw = w8.quantize_cols(w)
+    y = ispa.project_mx(torch.from_numpy(qa).cuda(), torch.from_numpy((ea + 127).astype(np.uint8)).cuda(),
+                        torch.from_numpy(np.ascontiguousarray(qw.T)).cuda(), torch.from_numpy(sw).cuda())
+    torch.cuda.synchronize()
+    _check_mx_projection(y, qa, ea, qw, sw)
+
+
+def test_project_mx_rejects_long_k_before_launch():
+    z = torch.zeros(16, 3712, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ispa.IspaError) as ei:
+        ispa.project_mx(z, torch.zeros(16, 116, dtype=torch.uint8, device="cuda"),
+                        torch.zeros(128, 3712, dtype=torch.uint8, device="cuda"),
+                        torch.ones(128, device="cuda"))
+    assert ei.value.code == 2
+
+
+def test_local_attention_project_mx_wan13b():
+    """The fused MX L-layer at the Wan-1.3B shapes (4680 chunk queries over
+    sink + current keys).  The attention epilogue quantises its bf16 output:
+    the plain single-pass attention of the same launch shape gives that bf16
+    A_loc bit for bit (attention parity against the oracle is tested
+    elsewhere), and the oracle's MX quantisation of it must equal the codes
+    and exponents the epilogue wrote.  y is the oracle's block-scaled product
+    of those codes with the oracle's weight codes, within the projection
+    bound."""
+    w = synth.WORKLOADS["wan1.3b"]
+    x = synth.single_layer_inputs(w, 1)
+    W = synth.weight(w, 0)
+    qwt, sw = ispa.quantize_e4m3_weight(dev(W, "bf16"))
+    status = ispa.new_status()
+    q = dev(x["q"], "bf16")
+    local = [(dev(x["k_sink"], "bf16"), dev(x["v_sink"], "bf16")), (dev(x["k_cur"], "bf16"), dev(x["v_cur"], "bf16"))]
+    out = ispa.local_attention_project_mx(q, local, qwt, sw, w.n_heads, status=status)
+    plain = ispa.dual_attention(q, local, [], w.n_heads, dual=False, status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "local_attention_project_mx")
+    a_bf16 = host(plain["a_full"])
+    qo, eo = w8.mx_quantize_rows(a_bf16)
+    assert np.array_equal(_u8(out["a_exps"]).astype(np.int64) - 127, eo)
+    assert np.array_equal(_u8(out["a_codes"]), qo)
+    qw_o, sw_o = w8.quantize_cols(W)
+    _check_mx_projection(out["y"], qo, eo, qw_o, sw_o)
+    # MX against the bf16 projection of the same A_loc: lossy, within e4m3 error
+    exact = a_bf16.astype(np.float64) @ W.astype(np.float64)
+    err = fro_rel(host(out["y"]), exact)
+    REPORT.append(("MX L-layer: y against the bf16 product (relative Frobenius)", err, err))
+    assert 1e-3 < err < 0.05

@@ -257,3 +257,46 @@ def test_mx_project_codes_brute_force_loops():
                 b = k // 32
                 acc += w8.e4m3_decode(qa[i, k]) * w8.e4m3_decode(qw[k, j]) * 2.0 ** (ea[i, b] + ew[b, j])
             assert got[i, j] == pytest.approx(acc, rel=1e-14, abs=1e-300)
+
+
+def test_mx_rows_project_codes_brute_force_loops():
+    rng = np.random.default_rng(36)
+    qa = rng.integers(0, 0x7E, (3, 96)).astype(np.uint8) | rng.choice([0, 0x80], (3, 96)).astype(np.uint8)
+    qw = rng.integers(0, 0x7E, (96, 4)).astype(np.uint8)
+    ea = rng.integers(-9, 9, (3, 3))
+    sw = rng.uniform(0.01, 2.0, 4)
+    got = w8.mx_rows_project_codes(qa, ea, qw, sw)
+    for i in range(3):
+        for j in range(4):
+            acc = 0.0
+            for k in range(96):
+                acc += w8.e4m3_decode(qa[i, k]) * w8.e4m3_decode(qw[k, j]) * 2.0 ** ea[i, k // 32]
+            assert got[i, j] == pytest.approx(acc * sw[j], rel=1e-14, abs=1e-300)
+
+
+def test_mx_rows_with_zero_exponents_is_the_per_token_product_with_unit_scales():
+    rng = np.random.default_rng(37)
+    qa = rng.integers(0, 0x7E, (5, 64)).astype(np.uint8)
+    qw = rng.integers(0, 0x7E, (64, 6)).astype(np.uint8) | rng.choice([0, 0x80], (64, 6)).astype(np.uint8)
+    sw = rng.uniform(0.5, 1.5, 6)
+    got = w8.mx_rows_project_codes(qa, np.zeros((5, 2), dtype=np.int64), qw, sw)
+    assert np.array_equal(got, w8.project_codes(qa, np.ones(5), qw, sw))
+
+
+def test_project_mx_rows_per_block_equivariance_and_accuracy():
+    """Scaling a 32-element block of a row by 2^k changes nothing but that
+    block's exponent, so the output is the same function of the unscaled
+    block; and the result is as close to the exact product as 3-bit
+    mantissas on both operands allow."""
+    rng = np.random.default_rng(38)
+    a = (rng.standard_normal((16, 128)) * np.exp2(rng.uniform(-6, 6, (16, 4))).repeat(32, 1)).astype(np.float32)
+    w = (rng.standard_normal((128, 24)) / 11).astype(np.float32)
+    qa, ea = w8.mx_quantize_rows(a)
+    a2 = a.copy()
+    a2[:, 64:96] *= 8.0
+    qa2, ea2 = w8.mx_quantize_rows(a2)
+    assert np.array_equal(qa2, qa) and np.array_equal(ea2[:, 2], ea[:, 2] + 3)
+    y = w8.project_mx_rows(a, w)
+    exact = a.astype(np.float64) @ w.astype(np.float64)
+    err = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert 1e-3 < err < 0.05
