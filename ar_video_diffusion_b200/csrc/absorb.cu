@@ -765,6 +765,9 @@ ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const voi
                                cudaStream_t stream);
 ispa_status_t gemm_hilo_w(int64_t M, int64_t K, const void* a_hi, const void* a_lo, const void* w, int64_t N,
                           float* c, int64_t ldc, cudaStream_t stream);
+ispa_status_t gemm_split3(int64_t M, int64_t N, int64_t K, const void* a_hi, const void* a_lo, int64_t lda,
+                          const void* b_hi, const void* b_lo, int64_t ldb, float* c, int64_t ldc,
+                          cudaStream_t stream);
 
 // One side stream and two events per host thread and CUDA context, created on
 // the first tensor-core solve there (make that first call before any stream
@@ -1008,7 +1011,100 @@ __global__ void frob_dot_kernel(const TX* __restrict__ x, const float* __restric
 
 }  // namespace simt
 
-size_t layer_error_workspace_bytes(int64_t D) { return (size_t)3 * D * D * sizeof(float); }
+// Tensor-core form (bf16 W, D % 128 == 0, D >= 256): the four products as
+// split-precision tcgen05 products, [P_R; P_E; P_G] = [R; sym(E); sym(G)] W
+// in one launch (W is exactly bf16: two operand pairs) and P_1 = sym(G) dW
+// (three pairs), then all six inner products in one pass.  Workspace:
+// P_R, P_E, P_G, P_1 (4 D^2 fp32), the bf16 hi / lo halves of the stacked
+// [R; sym(E); sym(G)] (2 x 3 D^2) and of dW (2 x D^2): 32 D^2 bytes.
+size_t layer_error_workspace_bytes(int64_t D) { return (size_t)32 * D * D; }
+
+// hi / lo bf16 halves of the rows of [R; sym(E); sym(G)] (3D x D): one 32 x 32
+// output tile per block, read through shared memory both as itself and
+// transposed, so the mirrored upper triangles are read with coalesced rows.
+__global__ void __launch_bounds__(256) split_stack_kernel(const float* __restrict__ R, const float* __restrict__ E,
+                                                          const float* __restrict__ G, int D,
+                                                          __nv_bfloat16* __restrict__ hi,
+                                                          __nv_bfloat16* __restrict__ lo) {
+  __shared__ float t[32][33], u[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;  // rows of the stack, columns
+  const int part = r0 / D, i0 = r0 - part * D;  // D % 32 == 0: a tile never straddles two parts
+  const float* M = part == 0 ? R : part == 1 ? E : G;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int y = ty; y < 32; y += 8) {
+    t[y][tx] = M[(int64_t)(i0 + y) * D + c0 + tx];
+    if (part > 0) u[y][tx] = M[(int64_t)(c0 + y) * D + i0 + tx];  // the mirrored tile, row by row
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int i = i0 + y, j = c0 + tx;
+    const float v = (part == 0 || i >= j) ? t[y][tx] : u[tx][y];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const int64_t e = (int64_t)(r0 + y) * D + j;
+    hi[e] = h;
+    lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// num += <dW, P_1> - 2 <dW, P_R> + <W, P_E>, den += <W, P_G> + 2 <W, P_R> + <W, P_E>
+// (fp64 accumulation, one pass over the six matrices)
+__global__ void __launch_bounds__(256) error_terms_kernel(const float* __restrict__ dW,
+                                                          const __nv_bfloat16* __restrict__ W,
+                                                          const float* __restrict__ P, int64_t n,
+                                                          double* __restrict__ num_den) {
+  __shared__ double part[2][8];
+  const float* PR = P;
+  const float* PE = P + n;
+  const float* PG = P + 2 * n;
+  const float* P1 = P + 3 * n;
+  double a_num = 0.0, a_den = 0.0;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const double d = dW[e], w = __bfloat162float(W[e]);
+    const double pr = PR[e], pe = PE[e];
+    a_num += d * (double)P1[e] - 2.0 * d * pr + w * pe;
+    a_den += w * (double)PG[e] + 2.0 * w * pr + w * pe;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a_num += __shfl_xor_sync(0xffffffffu, a_num, o);
+    a_den += __shfl_xor_sync(0xffffffffu, a_den, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    part[0][threadIdx.x >> 5] = a_num;
+    part[1][threadIdx.x >> 5] = a_den;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double x = 0.0, y = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) x += part[0][w], y += part[1][w];
+    atomicAdd(num_den, x);
+    atomicAdd(num_den + 1, y);
+  }
+}
+
+static ispa_status_t layer_error_tc(const float* G, const float* R, const float* E, const __nv_bfloat16* W,
+                                    const float* dW, int64_t D, uint8_t* ws, double* num_den, cudaStream_t st) {
+  const int64_t n = D * D;
+  float* P = reinterpret_cast<float*>(ws);  // P_R, P_E, P_G, P_1
+  __nv_bfloat16* s_hi = reinterpret_cast<__nv_bfloat16*>(ws + 16 * n);
+  __nv_bfloat16* s_lo = s_hi + 3 * n;
+  __nv_bfloat16* d_hi = s_lo + 3 * n;
+  __nv_bfloat16* d_lo = d_hi + n;
+  const int sms = num_sms();
+  if (cudaMemsetAsync(P, 0, 16 * (size_t)n, st) != cudaSuccess ||
+      cudaMemsetAsync(num_den, 0, 2 * sizeof(double), st) != cudaSuccess)
+    return check_launch("cudaMemsetAsync of the layer-error products");
+  split_stack_kernel<<<dim3((unsigned)(D / 32), (unsigned)(3 * D / 32)), 256, 0, st>>>(R, E, G, (int)D, s_hi, s_lo);
+  simt::split_bf16_kernel<<<sms * 4, 256, 0, st>>>(dW, d_hi, d_lo, n);
+  ispa_status_t s1 = check_launch("split_stack_kernel / split_bf16_kernel");
+  if (s1 != ISPA_OK) return s1;
+  s1 = gemm_hilo_w(3 * D, D, s_hi, s_lo, W, D, P, D, st);  // [R; E; G] W
+  if (s1 != ISPA_OK) return s1;
+  s1 = gemm_split3(D, D, D, s_hi + 2 * n, s_lo + 2 * n, D, d_hi, d_lo, D, P + 3 * n, D, st);  // G dW
+  if (s1 != ISPA_OK) return s1;
+  error_terms_kernel<<<sms * 2, 256, 0, st>>>(dW, W, P, n, num_den);
+  return check_launch("error_terms_kernel");
+}
 
 template <typename TW>
 static void layer_error_impl(const float* G, const float* R, const float* E, const TW* W, const float* dW, int D,
@@ -1039,6 +1135,9 @@ static void layer_error_impl(const float* G, const float* R, const float* E, con
 
 ispa_status_t layer_error_launch(const float* G, const float* R, const float* E, const void* W, ispa_dtype_t w_dt,
                                  const float* dW, int64_t D, void* workspace, double* num_den, cudaStream_t st) {
+  if (tc_eligible(w_dt, D))
+    return layer_error_tc(G, R, E, static_cast<const __nv_bfloat16*>(W), dW, D, static_cast<uint8_t*>(workspace),
+                          num_den, st);
   float* ws = static_cast<float*>(workspace);
   if (w_dt == ISPA_DT_BF16)
     layer_error_impl(G, R, E, static_cast<const __nv_bfloat16*>(W), dW, (int)D, ws, num_den, st);

@@ -781,6 +781,45 @@ ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const voi
   return launch<true, true, BN, 4>(p, (int)((k_blocks + per - 1) / per), stream);
 }
 
+// C[M, N] += A B for two fp32 matrices held as bf16 hi/lo pairs (A [M, K]
+// row-major with row stride lda, B [K, N] row-major with row stride ldb),
+// summed as hi(A) hi(B) + hi(A) lo(B) + lo(A) hi(B) in one accumulator; C fp32
+// (ldc), zeroed by the caller.  Two K halves per tile, reduced in L2.
+ispa_status_t gemm_split3(int64_t M, int64_t N, int64_t K, const void* a_hi, const void* a_lo, int64_t lda,
+                          const void* b_hi, const void* b_lo, int64_t ldb, float* c, int64_t ldc,
+                          cudaStream_t stream) {
+  using namespace gemm;
+  constexpr int BN = 128;
+  if (N % BN) return unsupported("split-precision product needs N %% 128 == 0");
+  Params p;
+  memset(&p, 0, sizeof(p));
+  CUtensorMap ah, al, bh, bl;
+  if (!encode_map_bf16_2d(&ah, a_hi, K, M, lda * 2, 64, kBM) || !encode_map_bf16_2d(&al, a_lo, K, M, lda * 2, 64, kBM))
+    return ISPA_ERR_CUDA;
+  if (!encode_map_bf16_2d(&bh, b_hi, N, K, ldb * 2, 64, 64) || !encode_map_bf16_2d(&bl, b_lo, N, K, ldb * 2, 64, 64))
+    return ISPA_ERR_CUDA;
+  p.a_map[0] = ah, p.a_map[1] = ah, p.a_map[2] = al;
+  p.b_map[0][0] = bh, p.b_map[0][1] = bl, p.b_map[0][2] = bh;
+  for (int q = 0; q < 3; ++q) p.b_map[1][q] = p.b_map[0][q];
+  p.n_pairs = 3;
+  p.c[0] = c;
+  p.c[1] = c;
+  p.ldc = ldc;
+  p.M = (int32_t)M;
+  p.N = (int32_t)N;
+  p.K = (int32_t)K;
+  p.n_split = (int32_t)N;
+  p.n_cols[0] = (int32_t)N;
+  p.mode = kReduceF32;
+  if (!encode_map_out_2d(&p.c_map[0], c, true, N, M, ldc * 4)) return ISPA_ERR_CUDA;
+  p.c_map[1] = p.c_map[0];
+  p.c_tma = 1;
+  const int64_t k_blocks = (K + kBK - 1) / kBK;
+  const int64_t per = (k_blocks + 1) / 2;
+  p.k_per_split = (int32_t)(per * kBK);
+  return launch<false, true, BN, 4>(p, (int)((k_blocks + per - 1) / per), stream);
+}
+
 // C[M, N] += (a_hi + a_lo) W, W exactly bf16 [K, N] row-major; a_hi / a_lo
 // bf16 [M, K] row-major; C fp32 (ldc), zeroed by the caller.  Two K halves
 // per tile, reduced in L2.

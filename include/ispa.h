@@ -158,7 +158,7 @@ ISPA_API ispa_status_t ispa_gram_accumulate(const void* a_loc, const void* a_del
 ISPA_API ispa_status_t ispa_sym_gram_accumulate(const void* x, int64_t n_rows, int64_t d_model, int64_t row_stride,
                                                 ispa_dtype_t dt, float* E, int32_t zero_first, void* stream);
 
-/* Bytes of device workspace ispa_layer_error needs for d_model (3 d^2 floats). */
+/* Bytes of device workspace ispa_layer_error needs for d_model (32 d^2). */
 ISPA_API size_t ispa_layer_error_workspace_bytes(int64_t d_model);
 
 /*
@@ -172,9 +172,12 @@ ISPA_API size_t ispa_layer_error_workspace_bytes(int64_t d_model);
  *   num_den[0] = <dW, G dW> - 2 <dW, R W> + <W, E W>,
  *   num_den[1] = <W, G W> + 2 <W, R W> + <W, E W>,
  * and eps = num_den[0] / num_den[1].  G, R, E, delta_w fp32 [D, D]; W [D, D]
- * in w_dt; num_den: two device doubles (8-byte aligned), overwritten.  fp32
- * products, fp64 sums.  workspace: at least ispa_layer_error_workspace_bytes
- * bytes, 16-byte aligned.  Asynchronous on `stream`.
+ * in w_dt; num_den: two device doubles (8-byte aligned), overwritten.  The
+ * products: with a bf16 W and D % 128 == 0, D >= 256, split-precision
+ * tensor-core products (each fp32 operand as a bf16 hi/lo pair, about 2^-17
+ * relative; W is exact), otherwise fp32 products on the CUDA cores; sums in
+ * fp64.  workspace: at least ispa_layer_error_workspace_bytes bytes, 16-byte
+ * aligned.  Asynchronous on `stream`.
  */
 ISPA_API ispa_status_t ispa_layer_error(const float* G, const float* R, const float* E, const void* W,
                                         ispa_dtype_t w_dt, const float* delta_w, int64_t d_model, void* workspace,

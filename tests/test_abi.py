@@ -133,7 +133,7 @@ def test_layer_selection_entry_points_reject_before_launch(L):
     assert L.ispa_layer_error(None, p, p, p, 0, p, 128, p, 1 << 20, p, None) == 1
     assert L.ispa_layer_error(p, p, p, p, 0, p, 128, p, 16, p, None) == 6
     assert L.ispa_layer_error(p, p, p, p, 9, p, 128, p, 1 << 20, p, None) == 2
-    assert ispa.ispa_layer_error_workspace_bytes(1536) == 3 * 1536 * 1536 * 4
+    assert ispa.ispa_layer_error_workspace_bytes(1536) == 32 * 1536 * 1536
     # symmetric statistics: bf16 needs d_model % 128 == 0; NULL E
     assert L.ispa_sym_gram_accumulate(p, 10, 96, 96, 0, p, 0, None) == 2
     assert L.ispa_sym_gram_accumulate(p, 10, 128, 128, 0, None, 0, None) == 1

@@ -46,7 +46,7 @@ def _activations(seed, n, D, dtype):
     return a_loc.astype(np.float64), d.astype(np.float64), W.astype(np.float64)
 
 
-@pytest.mark.parametrize("dtype,n,D", [("bf16", 4680, 1536), ("bf16", 900, 384), ("f32", 600, 128)])
+@pytest.mark.parametrize("dtype,n,D", [("bf16", 4680, 1536), ("bf16", 333, 512), ("bf16", 900, 384), ("f32", 600, 128)])
 def test_sym_gram_matches_oracle(dtype, n, D):
     _, d, _ = _activations(1, n, D, dtype)
     x = dev(d, dtype)
@@ -60,7 +60,9 @@ def test_sym_gram_matches_oracle(dtype, n, D):
     assert fro_rel(host(E)[lower], ref[lower]) < GRAM_REL
 
 
-@pytest.mark.parametrize("dtype,n,D", [("bf16", 4680, 1536), ("f32", 600, 128)])
+# bf16 with D % 128 == 0, D >= 256: split-precision tensor-core products;
+# fp32: the CUDA-core products
+@pytest.mark.parametrize("dtype,n,D", [("bf16", 4680, 1536), ("bf16", 700, 384), ("f32", 600, 128)])
 def test_layer_error_matches_oracle(dtype, n, D):
     a_loc, d, W = _activations(2, n, D, dtype)
     a_full = a_loc + d
