@@ -1031,9 +1031,11 @@ __global__ void __launch_bounds__(256) split_stack_kernel(const float* __restric
   const int part = r0 / D, i0 = r0 - part * D;  // D % 32 == 0: a tile never straddles two parts
   const float* M = part == 0 ? R : part == 1 ? E : G;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const bool need_t = part == 0 || i0 + 31 >= c0;  // some element on or below the diagonal
+  const bool need_u = part > 0 && i0 < c0 + 31;    // some element above it: read mirrored
   for (int y = ty; y < 32; y += 8) {
-    t[y][tx] = M[(int64_t)(i0 + y) * D + c0 + tx];
-    if (part > 0) u[y][tx] = M[(int64_t)(c0 + y) * D + i0 + tx];  // the mirrored tile, row by row
+    if (need_t) t[y][tx] = M[(int64_t)(i0 + y) * D + c0 + tx];
+    if (need_u) u[y][tx] = M[(int64_t)(c0 + y) * D + i0 + tx];  // the mirrored tile, row by row
   }
   __syncthreads();
   for (int y = ty; y < 32; y += 8) {
@@ -1058,11 +1060,24 @@ __global__ void __launch_bounds__(256) error_terms_kernel(const float* __restric
   const float* PG = P + 2 * n;
   const float* P1 = P + 3 * n;
   double a_num = 0.0, a_den = 0.0;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const double d = dW[e], w = __bfloat162float(W[e]);
-    const double pr = PR[e], pe = PE[e];
-    a_num += d * (double)P1[e] - 2.0 * d * pr + w * pe;
-    a_den += w * (double)PG[e] + 2.0 * w * pr + w * pe;
+  // four consecutive elements per step (n % 4 == 0): 16-byte loads, 8 bytes of W
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < n / 4; v += (int64_t)gridDim.x * blockDim.x) {
+    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dW) + v);
+    const float4 p1 = __ldg(reinterpret_cast<const float4*>(P1) + v);
+    const float4 pr = __ldg(reinterpret_cast<const float4*>(PR) + v);
+    const float4 pe = __ldg(reinterpret_cast<const float4*>(PE) + v);
+    const float4 pg = __ldg(reinterpret_cast<const float4*>(PG) + v);
+    const uint2 wb = __ldg(reinterpret_cast<const uint2*>(W) + v);
+    const float d[4] = {d4.x, d4.y, d4.z, d4.w}, q1[4] = {p1.x, p1.y, p1.z, p1.w};
+    const float qr[4] = {pr.x, pr.y, pr.z, pr.w}, qe[4] = {pe.x, pe.y, pe.z, pe.w}, qg[4] = {pg.x, pg.y, pg.z, pg.w};
+    const float w[4] = {__uint_as_float(wb.x << 16), __uint_as_float(wb.x & 0xFFFF0000u), __uint_as_float(wb.y << 16),
+                        __uint_as_float(wb.y & 0xFFFF0000u)};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double dj = d[j], wj = w[j], rj = qr[j], ej = qe[j];
+      a_num += dj * (double)q1[j] - 2.0 * dj * rj + wj * ej;
+      a_den += wj * (double)qg[j] + 2.0 * wj * rj + wj * ej;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -1102,7 +1117,7 @@ static ispa_status_t layer_error_tc(const float* G, const float* R, const float*
   if (s1 != ISPA_OK) return s1;
   s1 = gemm_split3(D, D, D, s_hi + 2 * n, s_lo + 2 * n, D, d_hi, d_lo, D, P + 3 * n, D, st);  // G dW
   if (s1 != ISPA_OK) return s1;
-  error_terms_kernel<<<sms * 2, 256, 0, st>>>(dW, W, P, n, num_den);
+  error_terms_kernel<<<sms * 8, 256, 0, st>>>(dW, W, P, n, num_den);
   return check_launch("error_terms_kernel");
 }
 
@@ -1135,7 +1150,8 @@ static void layer_error_impl(const float* G, const float* R, const float* E, con
 
 ispa_status_t layer_error_launch(const float* G, const float* R, const float* E, const void* W, ispa_dtype_t w_dt,
                                  const float* dW, int64_t D, void* workspace, double* num_den, cudaStream_t st) {
-  if (tc_eligible(w_dt, D))
+  // the tensor-core form reads W and dW through TMA and 16-byte vectors
+  if (tc_eligible(w_dt, D) && aligned16(W) && aligned16(dW) && aligned16(G) && aligned16(R) && aligned16(E))
     return layer_error_tc(G, R, E, static_cast<const __nv_bfloat16*>(W), dW, D, static_cast<uint8_t*>(workspace),
                           num_den, st);
   float* ws = static_cast<float*>(workspace);

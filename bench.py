@@ -429,10 +429,18 @@ def run_profile_case(op: str, reps: int, device):
         ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=True)
     if op == "merge":
         o_hist = ispa.dual_attention(q, [], hist, H, dual=False, status=status)
-    if op in ("project_w8a8", "quantize_rows"):
+    if op in ("project_w8a8", "quantize_rows", "project_mx", "local_mx"):
         a16 = ispa.dual_attention(q, local, hist, H, status=status)["a_loc"]
         qwt, sw = ispa.quantize_e4m3_weight(W)
         qa, sa = ispa.quantize_e4m3_rows(a16)
+        mq, me = ispa.mx_quantize_e4m3_rows(a16)
+    if op == "layer_error":
+        out = ispa.dual_attention(q, local, hist, H, status=status)
+        G, R, E = (torch.empty(D, D, device=device) for _ in range(3))
+        ispa.gram_accumulate(out["a_loc"], out["a_delta"], G, R, zero_first=True)
+        ispa.sym_gram_accumulate(out["a_delta"], E, zero_first=True)
+        dW, _ = ispa.absorb_solve(G, R, W, status=status)
+        ws = torch.empty(ispa.ispa_layer_error_workspace_bytes(D), dtype=torch.uint8, device=device)
     if op == "dual":
         out = {"a_loc": torch.empty(n, D, dtype=torch.bfloat16, device=device),
                "a_full": torch.empty(n, D, dtype=torch.bfloat16, device=device),
@@ -458,6 +466,12 @@ def run_profile_case(op: str, reps: int, device):
             ispa.project_w8a8(qa, sa, qwt, sw)
         elif op == "quantize_rows":
             ispa.quantize_e4m3_rows(a16, qa, sa)
+        elif op == "project_mx":
+            ispa.project_mx(mq, me, qwt, sw)
+        elif op == "local_mx":
+            ispa.local_attention_project_mx(q, local, qwt, sw, H, status=status)
+        elif op == "layer_error":
+            ispa.layer_error(G, R, E, W, dW, workspace=ws)
     torch.cuda.synchronize(device)
     if int(status[0].item()) != 0:
         raise RuntimeError(f"device status {int(status[0].item())}")
@@ -1056,7 +1070,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rollout", action="store_true", help="skip the 30-layer streaming rollout")
     ap.add_argument("--profile", choices=["dual", "full", "local", "gram", "project", "merge", "absorb",
-                                          "project_w8a8", "quantize_rows"],
+                                          "project_w8a8", "quantize_rows", "project_mx", "local_mx",
+                                          "layer_error"],
                     help="run only this op --steps times on the wan1.3b shapes (for ncu captures), no timing")
     args = ap.parse_args()
     if args.warmup < 3:
