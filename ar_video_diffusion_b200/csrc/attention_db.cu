@@ -353,38 +353,36 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
   // this warpgroup's partial row sum l, relative to the maximum m_l it last used
   float m_l = -INFINITY, l = 0.f, lse_loc2 = 0.f;
 
-  // local result: O / l written as A_loc (warpgroup w writes channels
-  // [w HD/2, (w + 1) HD/2)), LSE_loc by warpgroup 0; then a fresh accumulation
+  // local result: O / l written as A_loc and LSE_loc, then a fresh
+  // accumulation.  One warpgroup does it: the one that does not own tile
+  // n_loc (the first history tile), so that the other hands over its partial
+  // sums and goes straight on to that tile's scores while the local result is
+  // read out; the product of tile n_loc waits for the checkpoint (ck_done).
+  const int ck_wg = (n_loc + 1) & 1;
   auto checkpoint = [&]() -> bool {
-    if (!all(mbar_wait(B.ck_ready(), 0, abort_flag))) return false;  // PV of the last local tile complete
-    tc_fence_after();
-    float mf, lt;
-    if (w == 1) {
+    if (w != ck_wg) {
       xck[r.row] = m_l;
       xck[kBM + r.row] = l;
       mbar_arrive(B.xsum(0));
-      if (!all(mbar_wait(B.xsum(1), 0, abort_flag))) return false;
-      mf = xck[r.row];
-      lt = xck[kBM + r.row];
-    } else {
-      if (!all(mbar_wait(B.xsum(0), 0, abort_flag))) return false;
-      const float2 c = combine(m_l, l, xck[r.row], xck[kBM + r.row]);
-      mf = c.x;
-      lt = c.y;
-      xck[r.row] = mf;
-      xck[kBM + r.row] = lt;
-      mbar_arrive(B.xsum(1));
+      m_l = -INFINITY;
+      l = 0.f;
+      return true;
     }
-    const float inv = 1.0f / lt;
-    __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD + w * (HD / 2);
+    if (!all(mbar_wait(B.ck_ready(), 0, abort_flag))) return false;  // PV of the last local tile complete
+    tc_fence_after();
+    if (!all(mbar_wait(B.xsum(0), 0, abort_flag))) return false;
+    const float2 c = combine(m_l, l, xck[r.row], xck[kBM + r.row]);
+    const float inv = 1.0f / c.y;
+    __nv_bfloat16* dst = p.a_loc + (int64_t)r.grow * p.out_stride + head * HD;
 #pragma unroll 1
-    for (int kc = 0; kc < HD / 64; ++kc) {
+    for (int kc = 0; kc < HD / 32; ++kc) {
       float x[32];
-      load_o(r, w * (HD / 64) + kc, inv, x);
+      load_o(r, kc, inv, x);
       if (r.row_ok) store_bf16x32(dst + 32 * kc, x);
     }
-    lse_loc2 = mf + log2f(lt);
-    if (w == 0 && r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
+    lse_loc2 = c.x + log2f(c.y);
+    xck[r.row] = lse_loc2;  // for the other warpgroup's final fusion (read after xsum(2))
+    if (r.row_ok && p.lse_loc) p.lse_loc[(int64_t)head * p.n_q + r.grow] = lse_loc2 * kLn2;
     tc_fence_before();
     __syncwarp();
     if (r.lane == 0) mbar_arrive(B.ck_done());
@@ -509,6 +507,7 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
   mbar_arrive(B.xsum(2));
   if (!all(mbar_wait(B.xsum(2), 0, abort_flag))) return;
   const float2 cmb = combine(xfin[r.row], xfin[kBM + r.row], xfin[2 * kBM + r.row], xfin[3 * kBM + r.row]);
+  if (ck && w != ck_wg) lse_loc2 = xck[r.row];  // published by the checkpoint warpgroup
   const float inv = 1.0f / cmb.y;
   const float lse2 = cmb.x + log2f(cmb.y);
   const int64_t li = (int64_t)head * p.n_q + r.grow;
@@ -555,8 +554,8 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
     }
     return;
   }
-  // fuse the history result with the checkpointed local result (this
-  // warpgroup wrote the same channels of A_loc itself)
+  // fuse the history result with the checkpointed local result (A_loc was
+  // written by the checkpoint warpgroup before its xsum(2) arrival)
   const float mx = fmaxf(lse_loc2, lse2);
   const float lse_full2 = mx + log2f(exp2f(lse_loc2 - mx) + exp2f(lse2 - mx));
   const float wgt = exp2f(lse2 - lse_full2);
@@ -608,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
     }
     for (int i = 0; i < 4; ++i) mbar_init(B.mref_full(i), 32);  // the 32 rows of one warp
     mbar_init(B.ck_ready(), 1);
-    mbar_init(B.ck_done(), 8);
+    mbar_init(B.ck_done(), 4);  // the four warps of the checkpoint warpgroup
     mbar_init(B.fin_ready(), 1);
     mbar_init(B.xsum(0), 128);
     mbar_init(B.xsum(1), 128);
