@@ -99,11 +99,12 @@ def replica_tflops(flop_per_step: float, steps: int, world: int, t_max_ms: float
 
 def absorb_launches(D: int) -> int:
     """Kernel launches of one tensor-core absorb solve (bf16 W, D % 128 == 0):
-    split of R, [0 | I] fill, S = R W, trace, shift, one panel kernel per
-    64-wide panel, one update product per panel but the last, the split of
-    [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new."""
+    split of R, [0 | I] fill, S = R W, trace, shift and the first diagonal
+    factorisation; per 64-wide panel its application, and for every panel but
+    the last the next diagonal factorisation (side stream) and the update
+    product; the split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new."""
     nb = D // 64
-    return 5 + nb + (nb - 1) + 3
+    return 6 + nb + 2 * (nb - 1) + 3
 
 
 def cores() -> int:

@@ -31,10 +31,13 @@ def test_solve_flops_and_launch_count():
     assert bench.solve_flops(D) == pytest.approx(D ** 3 / 3 + 2 * D ** 3 + 2 * D ** 3)
     assert bench.solve_flops(D) == pytest.approx(15.7e9, rel=3e-3)
     nb = D // 64
-    # tensor-core form: split of R, [0 | I] fill, S = R W, trace, shift;
-    # nb panel kernels (each factoring its diagonal block) and nb-1 update
-    # products; the split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new
-    assert bench.absorb_launches(D) == 5 + nb + (nb - 1) + 3 == 55
+    # tensor-core form: split of R, [0 | I] fill, S = R W, trace, shift, the
+    # first diagonal factorisation; nb panel applications, nb-1 further
+    # diagonal factorisations (one panel ahead) and nb-1 update products; the
+    # split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new (an ncu launch
+    # list shows 24 diag_factor_kernel and 24 panel_apply_kernel launches per
+    # D = 1536 solve).
+    assert bench.absorb_launches(D) == 6 + nb + 2 * (nb - 1) + 3 == 79
 
 
 def test_chunk_rooflines_are_the_tensor_time_of_their_contractions():
