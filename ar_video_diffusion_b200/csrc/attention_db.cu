@@ -36,10 +36,10 @@
 // warpgroup of tile j once PV(j-1) has completed and before it hands P(j)
 // over, so every product lands on the right scale.  Each warpgroup keeps its
 // own partial row sum, brought to the current maximum when it next uses it.
-// Dual mode: once PV of the last local tile has completed, both warpgroups
-// normalise O (each writes half of the channels of A_loc) and LSE_loc is
-// written; the first history product then restarts O and the maximum chain
-// restarts.  The epilogue fuses the history result with A_loc (logaddexp of
+// Dual mode: once PV of the last local tile has completed, the warpgroup that
+// does not own the first history tile normalises O into A_loc and writes
+// LSE_loc while the other goes on with that tile; the first history product
+// then restarts O and the maximum chain restarts.  The epilogue fuses the history result with A_loc (logaddexp of
 // the two LSEs).  Single-pass mode runs one softmax over every tile.
 #include <cstring>
 
@@ -56,9 +56,11 @@ constexpr int kMaxSeg = ISPA_MAX_SEGMENTS;
 constexpr float kRescaleLog2 = 16.0f;  // lazy rescale threshold (log2)
 constexpr float kLn2 = 0.69314718055994530942f;
 // tensor-memory column map
-constexpr int kNS = 3;          // S buffers: tile j uses buffer j mod 3 at kTmS + 128 (j mod 3)
+constexpr int kNS = 3;          // S buffers: tile j uses buffer j mod kNS at kTmS + kBN (j mod kNS)
 constexpr uint32_t kTmS = 0;
-constexpr uint32_t kTmO = 384;  // the O accumulator (head_dim columns)
+constexpr uint32_t kTmO = kNS * kBN;  // the O accumulator (head_dim columns)
+static_assert(kTmO + 128 <= 512, "tensor-memory budget");
+static_assert(kBN % 32 == 0 && kBN <= 128, "key tile");
 // bit j set: column pair j (mod 8) of a score row takes 2^x from the FMA-pipe
 // polynomial (exp2_fma2) instead of the special-function unit
 constexpr uint32_t kEmuPairs = 0x00u;
@@ -92,15 +94,17 @@ struct Params {
 
 template <int HD, int NST>
 struct Layout {
+  static constexpr int kQBytes = kBM * HD * 2;     // the Q tile
+  static constexpr int kQBox = kBM * 128;          // kBM rows x 64 bf16 (one swizzle column block)
   static constexpr int kTileBytes = kBN * HD * 2;  // one K or V tile
-  static constexpr int kBoxBytes = kBN * 128;      // 128 rows x 64 bf16 (one swizzle column block)
+  static constexpr int kBoxBytes = kBN * 128;      // kBN rows x 64 bf16
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kK = kQ + kQBytes;
   static constexpr int kV = kK + NST * kTileBytes;
   static constexpr int kXs = kV + NST * kTileBytes;  // local checkpoint exchange: (m, l) per row
   static constexpr int kMref = kXs + 2 * kBM * 4;     // the shared running maximum, one float per row
   static constexpr int kBars = kMref + kBM * 4;
-  // kv_full, kv_empty, v_full, v_empty [NST]; q_full; s_full, p_full, pv_done [3]; mref_full[4];
+  // kv_full, kv_empty, v_full, v_empty [NST]; q_full; s_full, p_full, pv_done [kNS]; mref_full[4];
   // ck_ready, ck_done, fin_ready; xsum[3]; teardown[2]
   static constexpr int kNumBars = 4 * NST + 1 + 3 * kNS + 4 + 3 + 3 + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;
@@ -158,10 +162,10 @@ __device__ void producer(const Params& p, uint8_t* smem, bool v_side, uint64_t* 
   using L = Layout<HD, NST>;
   if (!v_side) {
     tma_prefetch_desc(&p.q_map);
-    mbar_arrive_expect_tx(q_full, L::kTileBytes);
+    mbar_arrive_expect_tx(q_full, L::kQBytes);
 #pragma unroll
     for (int c = 0; c < HD / 64; ++c)
-      tma_load_2d(smem + L::kQ + c * L::kBoxBytes, &p.q_map, q_full, head * HD + 64 * c, q0);
+      tma_load_2d(smem + L::kQ + c * L::kQBox, &p.q_map, q_full, head * HD + 64 * c, q0);
   }
   uint8_t* ring = smem + (v_side ? L::kV : L::kK);
   const CUtensorMap* maps = v_side ? p.v_map : p.k_map;
@@ -203,16 +207,18 @@ struct Bars {
   __device__ __forceinline__ uint64_t* v_full(int i) const { return base + 2 * NST + i; }
   __device__ __forceinline__ uint64_t* v_empty(int i) const { return base + 3 * NST + i; }
   __device__ __forceinline__ uint64_t* q_full() const { return base + 4 * NST; }
-  __device__ __forceinline__ uint64_t* s_full(int b) const { return base + 4 * NST + 1 + b; }     // per S buffer
-  __device__ __forceinline__ uint64_t* p_full(int b) const { return base + 4 * NST + 4 + b; }
-  __device__ __forceinline__ uint64_t* pv_done(int b) const { return base + 4 * NST + 7 + b; }
-  __device__ __forceinline__ uint64_t* mref_full(int q) const { return base + 4 * NST + 10 + q; }  // per warp quarter
-  __device__ __forceinline__ uint64_t* ck_ready() const { return base + 4 * NST + 14; }
-  __device__ __forceinline__ uint64_t* ck_done() const { return base + 4 * NST + 15; }
-  __device__ __forceinline__ uint64_t* fin_ready() const { return base + 4 * NST + 16; }
-  __device__ __forceinline__ uint64_t* xsum(int k) const { return base + 4 * NST + 17 + k; }
-  __device__ __forceinline__ uint64_t* teardown(int w) const { return base + 4 * NST + 20 + w; }  // per issuer
-  static constexpr int kCount = 4 * NST + 22;
+  static constexpr int kS = 4 * NST + 1;  // the per-S-buffer barriers start here
+  static constexpr int kR = kS + 3 * kNS;  // and the rest here
+  __device__ __forceinline__ uint64_t* s_full(int b) const { return base + kS + b; }  // per S buffer
+  __device__ __forceinline__ uint64_t* p_full(int b) const { return base + kS + kNS + b; }
+  __device__ __forceinline__ uint64_t* pv_done(int b) const { return base + kS + 2 * kNS + b; }
+  __device__ __forceinline__ uint64_t* mref_full(int q) const { return base + kR + q; }  // per warp quarter
+  __device__ __forceinline__ uint64_t* ck_ready() const { return base + kR + 4; }
+  __device__ __forceinline__ uint64_t* ck_done() const { return base + kR + 5; }
+  __device__ __forceinline__ uint64_t* fin_ready() const { return base + kR + 6; }
+  __device__ __forceinline__ uint64_t* xsum(int k) const { return base + kR + 7 + k; }
+  __device__ __forceinline__ uint64_t* teardown(int w) const { return base + kR + 10 + w; }  // per issuer
+  static constexpr int kCount = kR + 12;
 };
 
 // Two issuing warps, each converged with one elected lane issuing:
@@ -240,11 +246,13 @@ __device__ void s_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, vol
     if (!(ok = wait(B.kv_full(stage), (j / NST) & 1))) break;
     tc_fence_after();
     const uint32_t kb = sK + stage * L::kTileBytes;
-    const uint32_t d = tmem + kTmS + b * 128;
+    const uint32_t d = tmem + kTmS + b * kBN;
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-      umma_ss_warp(d, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdescQK,
+      // 16 head-dim elements (32 bytes) of every row, in the column block kk / 4
+      const uint32_t offq = (kk >> 2) * L::kQBox + (kk & 3) * 32;
+      const uint32_t offk = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+      umma_ss_warp(d, sdesc_sw128(sQ + offq, 16, 1024), sdesc_sw128(kb + offk, 16, 1024), kIdescQK,
                    kk > 0 ? 1u : 0u);
     }
     umma_commit_warp(B.s_full(b));
@@ -276,15 +284,15 @@ __device__ void pv_issuer(const Params& p, uint8_t* smem, const Bars<NST>& B, vo
     if (first_hist && !wait(B.ck_done(), 0)) break;
     const int stage = i % NST;
     const uint32_t vb = sV + stage * L::kTileBytes;
-    const uint32_t pb = tmem + kTmS + b * 128;
+    const uint32_t pb = tmem + kTmS + b * kBN;
     if (!wait(B.v_full(stage), (i / NST) & 1)) break;
     // p_full[b] completes once per use of buffer b; its next phase needs
     // S(i + 3), which waits for PV(i), so the parity is unambiguous
     if (!wait(B.p_full(b), (i / kNS) & 1)) break;
     tc_fence_after();
-    // O += P V: P (bf16, 128 keys) in the first 64 columns of S buffer b
+    // O += P V: P (bf16, kBN keys) in the first kBN / 2 columns of S buffer b
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
+    for (int kk = 0; kk < kBN / 16; ++kk)
       umma_ts_warp(tmem + kTmO, pb + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBoxBytes, 1024), kIdescPV,
                    (kk > 0 || !fresh) ? 1u : 0u);
     umma_commit_warp(B.v_empty(stage));
@@ -413,15 +421,16 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
     for (int q = 0; q < kMaxSeg; ++q)
       if (i == p.seg_last_tile[q]) valid = p.seg_last_valid[q];
 
-    // the whole 128-key row of S in registers
-    const uint32_t sbuf = r.lane_base + kTmS + b * 128;
-    uint32_t s[4][32];
+    // the whole kBN-key row of S in registers
+    constexpr int NC = kBN / 32;
+    const uint32_t sbuf = r.lane_base + kTmS + b * kBN;
+    uint32_t s[NC][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, s[c]);
+    for (int c = 0; c < NC; ++c) tmem_ld32(sbuf + 32 * c, s[c]);
     tmem_wait_ld();
     if (valid < kBN) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (c * 32 + j >= valid) s[c][j] = __float_as_uint(-INFINITY);
@@ -429,16 +438,20 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
     // tile maximum (scaled, log2 domain; -inf if every key is masked)
     float m_tile;
     {
-      float mc[8];
+      constexpr int NG = kBN / 16;  // groups of 16 scores, reduced independently
+      float mc[NG];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < NG; ++q) {
         const uint32_t* v = &s[q >> 1][(q & 1) * 16];
         mc[q] = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
 #pragma unroll
         for (int j = 1; j < 8; ++j) mc[q] = fmax3(mc[q], __uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
       }
-      const float a = fmax3(mc[0], mc[1], mc[2]), bb = fmax3(mc[3], mc[4], mc[5]), c = fmaxf(mc[6], mc[7]);
-      m_tile = fmax3(a, bb, c) * sl2;
+      float m = mc[0];
+#pragma unroll
+      for (int q = 1; q + 1 < NG; q += 2) m = fmax3(m, mc[q], mc[q + 1]);
+      if (NG % 2 == 0) m = fmaxf(m, mc[NG - 1]);
+      m_tile = m * sl2;
     }
     const bool fin_prev = m_prev != -INFINITY;
     const bool grow = __any_sync(0xffffffffu, fin_prev && m_tile > m_prev + kRescaleLog2);
@@ -446,15 +459,15 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
     mref[r.row] = m_i;
     mbar_arrive(B.mref_full(r.quarter));
 
-    // P = 2^(s * scale_log2 - m) as bf16 into the first 64 columns of the S
-    // buffer (whose values are all in registers by now); the sum of P
+    // P = 2^(s * scale_log2 - m) as bf16 into the first kBN / 2 columns of
+    // the S buffer (whose values are all in registers by now); the sum of P
     float psum;
     {
       const float m = m_i == -INFINITY ? 0.f : m_i;
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
-      float2 sum2[4];
+      float2 sum2[NC];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < NC; ++c) {
         sum2[c] = make_float2(0.f, 0.f);
         uint32_t pk[16];
 #pragma unroll
@@ -467,7 +480,9 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
         }
         tmem_st16(sbuf + 16 * c, pk);
       }
-      const float2 st2 = fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3]));
+      float2 st2 = sum2[0];
+#pragma unroll
+      for (int c = 1; c < NC; ++c) st2 = fadd2(st2, sum2[c]);
       psum = st2.x + st2.y;
     }
     if (l > 0.f && m_i != m_l) l *= ex2(m_l - m_i);
