@@ -67,7 +67,9 @@ struct Layout {
   static constexpr int kRows = WIDE ? 128 : kBM;  // output rows of a tile
   static constexpr int kCols = WIDE ? 2 * BN : BN;  // output columns of a tile
   static constexpr int kABytes = kRows * kBK * 2;
-  static constexpr int kBBytes = kCols * kBK * 2;
+  // B is loaded in 64-column boxes (MN-major) or kCols-row boxes (K-major):
+  // a tile width that is not a multiple of 64 still lands whole boxes
+  static constexpr int kBBytes = (kCols + 63) / 64 * 64 * kBK * 2;
   static constexpr int kTmemCols = 2 * BN <= 256 ? 256 : 512;  // a power of two
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBars = NST * kStage;
@@ -203,7 +205,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
       }
       if (B_MN) {
 #pragma unroll
-        for (int c = 0; c < L::kCols / 64; ++c) tma_load_2d(sb + c * 8192, bm, &full[stage], n0 + 64 * c, k0);
+        for (int c = 0; c < (L::kCols + 63) / 64; ++c) tma_load_2d(sb + c * 8192, bm, &full[stage], n0 + 64 * c, k0);
       } else {
 #pragma unroll
         for (int h = 0; h < L::kCols / BN; ++h)  // boxes of BN rows (a box is at most 256 rows)
@@ -464,6 +466,68 @@ static ProjTile projection_tile(int64_t M, int64_t N) {
 
 }  // namespace gemm
 
+namespace gemm {
+
+// Tile width and token split of the statistics [G | R] (with_r) or E.  The
+// row tile is 256 (two M=128 halves); the column tile BN is 256, 224 or 128
+// (D % 128 == 0 is required).  Tiles: those of G that touch its lower
+// triangle, plus all of R.  The token range of every tile is split in
+// `splits` parts so that the launch fills one wave of SMs where it can
+// (at least 8 K steps per part), and the plan with the least time per SM --
+// waves x tile width x K steps per part -- wins.  The 224-wide tile (69
+// tiles x 2 parts = 138 CTAs at D = 1536 instead of 57 x 2 = 114) is taken
+// only for short parts (at most 64 K steps): measured on B200, it saves 10 %
+// over 4680 rows, but over long token ranges, where the wave streams its
+// operands from L2 at 11-13 TB/s, its more numerous CTAs and the unused
+// quarter of its last B box cost more than the narrower tile saves (93600
+// rows: 511 against 490 us).
+// G's column range is padded to whole tiles (g_cols) so that R's starts on a
+// tile; the padding columns are clipped by the output maps.
+struct StatPlan {
+  int BN;
+  int64_t g_cols;
+  int32_t k_per_split;
+  int splits;
+};
+
+static StatPlan statistics_plan(int64_t D, int64_t n_rows, bool with_r) {
+  const int64_t sms = num_sms();
+  const int64_t k_blocks = (n_rows + kBK - 1) / kBK;
+  const int widths[3] = {256, 224, 128};
+  const double eff[3] = {1.0, 1.0, 0.9};  // per-area rate of each width, relative to 256
+  StatPlan best{128, 0, 0, 1};
+  double best_cost = -1.0;
+  for (int w = 0; w < 3; ++w) {
+    const int BN = widths[w];
+    if (BN == 256 && D % 256) continue;
+    const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = (D + BN - 1) / BN;
+    int64_t tiles = with_r ? m_tiles * n_tiles : 0;
+    for (int64_t i = 0; i < m_tiles; ++i)
+      for (int64_t j = 0; j < n_tiles; ++j) tiles += (j * BN <= i * kBM + kBM - 1) ? 1 : 0;
+    int64_t splits = sms / tiles;
+    if (splits > k_blocks / 8) splits = k_blocks / 8;
+    if (splits < 1) splits = 1;
+    const int64_t per = (k_blocks + splits - 1) / splits;
+    if (BN == 224 && per > 64) continue;
+    splits = (k_blocks + per - 1) / per;
+    const int64_t waves = (tiles * splits + sms - 1) / sms;
+    const double cost = (double)waves * BN * per / eff[w];
+    if (best_cost < 0.0 || cost < best_cost) {
+      best = {BN, n_tiles * BN, (int32_t)(per * kBK), (int)splits};
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+static ispa_status_t launch_statistics(const Params& p, const StatPlan& sp, cudaStream_t stream) {
+  if (sp.BN == 256) return launch<true, true, 256, 3>(p, sp.splits, stream);
+  if (sp.BN == 224) return launch<true, true, 224, 3>(p, sp.splits, stream);
+  return launch<true, true, 128, 4>(p, sp.splits, stream);
+}
+
+}  // namespace gemm
+
 // [G | R] (+)= A_loc^T [A_loc | delta]  (bf16 inputs, fp32 outputs).  Only the
 // lower triangle of G (and all of R) is produced; the K range (rows) is split
 // across CTAs so that the launch fills the GPU, and the partial products are
@@ -493,22 +557,11 @@ ispa_status_t gram_bf16(const void* a_loc, const void* a_delta, int64_t n_rows, 
   p.ldc = D;
   p.mode = kReduceF32;
   if (!set_out_maps(p, true, D, D, D, D)) return ISPA_ERR_CUDA;
-  const int BN = D % 256 == 0 ? 256 : 128;
-  const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
-  int64_t tiles = m_tiles * n_tiles;  // R
-  for (int64_t i = 0; i < m_tiles; ++i)
-    for (int64_t j = 0; j < n_tiles; ++j) tiles += (j * BN <= i * kBM + kBM - 1) ? 1 : 0;  // lower part of G
-  const int64_t k_blocks = (n_rows + kBK - 1) / kBK;
-  const int sms = num_sms();
-  // one CTA per SM: the largest split count that still fits in one wave
-  int64_t splits = sms / tiles;
-  if (splits > k_blocks / 8) splits = k_blocks / 8;  // keep at least 8 K steps per CTA
-  if (splits < 1) splits = 1;
-  const int64_t blocks_per_split = (k_blocks + splits - 1) / splits;
-  p.k_per_split = (int32_t)(blocks_per_split * kBK);
-  splits = (k_blocks + blocks_per_split - 1) / blocks_per_split;
-  if (BN == 256) return launch<true, true, 256, 3>(p, (int)splits, stream);
-  return launch<true, true, 128, 4>(p, (int)splits, stream);
+  const StatPlan sp = statistics_plan(D, n_rows, true);
+  p.n_split = (int32_t)sp.g_cols;  // the R range starts on a whole tile
+  p.N = p.n_split + (int32_t)D;
+  p.k_per_split = sp.k_per_split;
+  return launch_statistics(p, sp, stream);
 }
 
 // E (+)= X^T X (bf16 input, fp32 output): the lower triangle of a symmetric
@@ -537,20 +590,11 @@ ispa_status_t sym_gram_bf16(const void* x, int64_t n_rows, int64_t D, int64_t ro
   p.ldc = D;
   p.mode = kReduceF32;
   if (!set_out_maps(p, true, D, D, D, D)) return ISPA_ERR_CUDA;
-  const int BN = D % 256 == 0 ? 256 : 128;
-  const int64_t m_tiles = (D + kBM - 1) / kBM, n_tiles = D / BN;
-  int64_t tiles = 0;
-  for (int64_t i = 0; i < m_tiles; ++i)
-    for (int64_t j = 0; j < n_tiles; ++j) tiles += (j * BN <= i * kBM + kBM - 1) ? 1 : 0;
-  const int64_t k_blocks = (n_rows + kBK - 1) / kBK;
-  int64_t splits = num_sms() / tiles;
-  if (splits > k_blocks / 8) splits = k_blocks / 8;
-  if (splits < 1) splits = 1;
-  const int64_t blocks_per_split = (k_blocks + splits - 1) / splits;
-  p.k_per_split = (int32_t)(blocks_per_split * kBK);
-  splits = (k_blocks + blocks_per_split - 1) / blocks_per_split;
-  if (BN == 256) return launch<true, true, 256, 3>(p, (int)splits, stream);
-  return launch<true, true, 128, 4>(p, (int)splits, stream);
+  const StatPlan sp = statistics_plan(D, n_rows, false);
+  p.n_split = (int32_t)sp.g_cols;
+  p.N = (int32_t)sp.g_cols;
+  p.k_per_split = sp.k_per_split;
+  return launch_statistics(p, sp, stream);
 }
 
 // C[M, N] (= | +=) A[M, K] W[K, N]: bf16 row-major A and W, fp32 C (ldc).
