@@ -98,7 +98,7 @@ constexpr int kMxMaxStages = (512 - (int)kSfaCol) / 4;  // K <= 28 * 128 = 3584
 // MX (block-scaled A, wide tile only): the MMAs are kind::mxf8f6f4 with one
 // ue8m0 scale per 32 K-elements of each row of A and unit scales for B (the
 // per-column weight scale stays in the epilogue).  Before the first MMA,
-// warps 4-7 write every scale of the tile's 128 rows into tensor memory in
+// warps 4-11 write every scale of the tile's 128 rows into tensor memory in
 // the layout the instruction reads for M = 128: the scale of row 32c + l for
 // the K block 4j + b sits in byte b of column kSfaCol + 4j + c, lane l, and is
 // repeated in the lanes l + 32, l + 64, l + 96 of the other three
@@ -140,7 +140,7 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
     }
     mbar_init(acc_full, 1);
     mbar_init(teardown, 1);
-    mbar_init(sf_ready, 128);
+    mbar_init(sf_ready, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -153,15 +153,20 @@ __device__ __forceinline__ void gemm_body(const Params& p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (MX && warp >= 4 && warp < 8) {
+  if (MX && warp >= 4) {
     // ------------------------------------------------- block scales (MX)
+    // both epilogue warpgroups take turns over the 16-column groups (a warp
+    // reaches the lanes of its own sub-partition, warp mod 4)
+    const int wg = (warp - 4) >> 2;
     const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t r[16];
+    if (wg == 0) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) r[j] = 0x7F7F7F7Fu;  // 2^0 in every byte
-    tmem_st16(tmem + lanes + kSfbCol, r);
+      for (int j = 0; j < 16; ++j) r[j] = 0x7F7F7F7Fu;  // 2^0 in every byte
+      tmem_st16(tmem + lanes + kSfbCol, r);
+    }
 #pragma unroll 1
-    for (int g = 0; g < (nk + 3) / 4; ++g) {  // 16 columns: 4 K stages x 4 row groups
+    for (int g = wg; g < (nk + 3) / 4; g += 2) {  // 16 columns: 4 K stages x 4 row groups
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int j = 4 * g + t;
