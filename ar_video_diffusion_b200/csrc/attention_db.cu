@@ -624,9 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
     mbar_init(B.ck_ready(), 1);
     mbar_init(B.ck_done(), 4);  // the four warps of the checkpoint warpgroup
     mbar_init(B.fin_ready(), 1);
-    mbar_init(B.xsum(0), 128);
-    mbar_init(B.xsum(1), 128);
-    mbar_init(B.xsum(2), 256);
+    mbar_init(B.xsum(0), 128);  // the partial sums handed to the checkpoint warpgroup
+    mbar_init(B.xsum(2), 256);  // the final (m, l) exchange; xsum(1) is unused
     mbar_init(B.teardown(0), 1);
     mbar_init(B.teardown(1), 1);
     *abort_flag = 0;
