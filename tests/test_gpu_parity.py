@@ -208,10 +208,10 @@ def test_lse_merge_rows_with_both_branches_empty():
         assert np.all(got["a_full"][np.ix_(r, range(h * d, (h + 1) * d))] == 0.0)
 
 
-# (1, 256): one row; (130, 512): ragged rows over several tiles; D % 256 != 0
-# takes the 256 x 128 tiles
-@pytest.mark.parametrize("n_rows,D", [(4680, 1536), (300, 256), (1, 256), (130, 512), (5000, 768), (1, 128),
-                                      (129, 384)])
+# (1, 256): one row; (130, 512): ragged rows over several 224-wide tiles
+# (the last overhangs D); (1000, 640): a width the 256-wide tile cannot take
+@pytest.mark.parametrize("n_rows,D", [(4680, 1536), (300, 256), (1, 256), (130, 512), (5000, 768), (1000, 640),
+                                      (1, 128), (129, 384)])
 def test_gram_bf16_matches_oracle(n_rows, D):
     g = np.random.default_rng(n_rows + D)
     A = synth.round_bf16((g.standard_normal((n_rows, D)) * 0.3).astype(np.float32))

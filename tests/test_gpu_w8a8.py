@@ -257,3 +257,28 @@ def test_local_attention_project_mx_wan13b():
     err = fro_rel(host(out["y"]), exact)
     REPORT.append(("MX L-layer: y against the bf16 product (relative Frobenius)", err, err))
     assert 1e-3 < err < 0.05
+
+
+def test_local_attention_project_mx_head_dim_64_ragged():
+    """The MX epilogue with head_dim 64 (one 32-channel block per warpgroup
+    and row), 4 heads, a ragged last query tile and ragged key segments:
+    codes and exponents bit-exact against the oracle's MX quantisation of the
+    plain pass's bf16 output, y within the projection bound."""
+    H, d, n_q = 4, 64, 300
+    c = synth.random_case(77, n_q, H, d, [100, 333])
+    q = dev(c["q"], "bf16")
+    local = [(dev(k, "bf16"), dev(v, "bf16")) for k, v in c["segments"]]
+    rng = np.random.default_rng(78)
+    W = _bf16(rng, (H * d, H * d), 1.0 / np.sqrt(H * d))
+    qwt, sw = ispa.quantize_e4m3_weight(dev(W, "bf16"))
+    status = ispa.new_status()
+    out = ispa.local_attention_project_mx(q, local, qwt, sw, H, status=status)
+    plain = ispa.dual_attention(q, local, [], H, dual=False, status=status)
+    torch.cuda.synchronize()
+    ispa.raise_on_status(status, "local_attention_project_mx")
+    qo, eo = w8.mx_quantize_rows(host(plain["a_full"]))
+    assert np.array_equal(_u8(out["a_exps"]).astype(np.int64) - 127, eo)
+    assert np.array_equal(_u8(out["a_codes"]), qo)
+    qw_o, sw_o = w8.quantize_cols(W)
+    _check_mx_projection(out["y"], qo, eo, qw_o, sw_o)
+
