@@ -663,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, 512);
-  if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
+  if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status, *abort_flag);
 }
 
 template <int HD, int NST>

@@ -65,9 +65,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// A wait gives up only when BOTH its time limit has passed on %globaltimer
+// and it has polled at least this many times, so that a jump of the global
+// timer alone cannot end a wait that is still making progress.
+constexpr uint32_t kMinPolls = 1u << 20;
+constexpr uint32_t kMinPollsDrain = 1u << 16;
+
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (and sets *abort_flag) once the time limit passes or another thread
-// of the CTA has already given up.
+// of the CTA has already given up.  The flag records which barrier gave up:
+// 0x40000000 | its shared-memory address | parity << 29.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -75,19 +82,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
+      if (it >= kMinPolls && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = (int)(0x40000000u | ((parity & 1u) << 29) | (smem_u32(bar) & 0x1FFFFFFFu));
         return false;
       }
     }
   }
 }
 
-// Bounded wait used during unwinding: never looks at the abort flag.
+// After a bounded wait gave up: the status word gets ISPA_ERR_TIMEOUT and,
+// from the CTA that set it first, which barrier it was (detail word).
+__device__ __forceinline__ void report_timeout(int32_t* status, int abort_flag) {
+  if (status && atomicCAS(status, 0, (int32_t)ISPA_ERR_TIMEOUT) == 0) status[1] = abort_flag;
+}
+
+// Bounded wait used during unwinding and before tensor memory is released:
+// never looks at the abort flag.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+    if (it >= kMinPollsDrain && globaltimer_ns() - t0 > limit_ns) return false;
   }
   return true;
 }

@@ -307,7 +307,7 @@ class Rollout:
             torch.cuda.synchronize(self.device)
             code = int(self.status[0].item())
             if code != 0:
-                raise ispa.IspaError(code, f"rollout chunk {c}", "device status")
+                raise ispa.IspaError(code, f"rollout chunk {c}", f"device status detail {int(self.status[1].item())}")
             self.reports.append(ChunkReport(c, "warmup" if c < self.w.warm_chunks else "post",
                                             e0.elapsed_time(e1), self.kv_bytes(c), self.kv_bytes(c, all_f=True)))
         return self.reports
