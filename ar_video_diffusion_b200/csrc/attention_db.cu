@@ -407,12 +407,16 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, const Bar
       if (!(ok = checkpoint())) break;
     }
     // the maximum tile i - 1 used (none at the start of an accumulation),
-    // read before the scores occupy the registers
+    // read before the scores occupy the registers.  Every tile's publication
+    // is one phase of mref_full, in tile order, so even the first history
+    // tile, which does not use it, waits for tile i - 1's publication before
+    // making its own (it would otherwise complete that phase in its place and
+    // leave a stale maximum in mref for the tile after it)
     const bool first_acc = i == 0 || (ck && i == n_loc);
     float m_prev = -INFINITY;
-    if (!first_acc) {
+    if (i > 0) {
       if (!(ok = all(mbar_wait(B.mref_full(r.quarter), (i - 1) & 1, abort_flag)))) break;
-      m_prev = mref[r.row];
+      if (!first_acc) m_prev = mref[r.row];
     }
     if (!(ok = all(mbar_wait(B.s_full(b), (i / kNS) & 1, abort_flag)))) break;
     tc_fence_after();
@@ -663,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, 512);
-  if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status, *abort_flag);
+  if (threadIdx.x == 0 && *abort_flag) report_status(p.status, ISPA_ERR_TIMEOUT);
 }
 
 template <int HD, int NST>
