@@ -75,3 +75,28 @@ def test_statistics_and_solve_reproducible_within_summation_rounding():
         assert fro_rel(g, res[0][0]) <= 1e-5
         assert fro_rel(r, res[0][1]) <= 1e-5
         assert fro_rel(d, res[0][2]) <= 1e-4
+
+
+def test_dual_attention_repeated_against_the_oracle():
+    """The local checkpoint hands over to the history between two tiles of
+    different warpgroups; the row maximum each tile publishes must stay in
+    tile order across that hand-over (a mixed-up publication once left a
+    stale maximum in place and gave a wrong A_full while A_loc and the LSEs
+    stayed right).  Every one of several runs is checked against the
+    oracle, not only against the others."""
+    from oracle import ispa_oracle as orc
+    from helpers import ATTN_MAX_REL, max_rel
+    for seed, segs_n in ((41, [128, 600, 1000, 333]), (42, [1, 700, 129, 900]), (43, [256, 256, 640])):
+        c = synth.random_case(seed, n_q=600, n_heads=3, head_dim=128, seg_tokens=segs_n)
+        n_loc = 2
+        ref = orc.dual_stream(c["q"], c["segments"][:n_loc], c["segments"][n_loc:], 3)
+        q = dev(c["q"], "bf16")
+        segs = [(dev(k, "bf16"), dev(v, "bf16")) for k, v in c["segments"]]
+        status = ispa.new_status()
+        for _ in range(5):
+            out = ispa.dual_attention(q, segs[:n_loc], segs[n_loc:], 3, status=status)
+            torch.cuda.synchronize()
+            assert max_rel(host(out["a_loc"]), ref["a_loc"]) <= ATTN_MAX_REL, seed
+            assert max_rel(host(out["a_full"]), ref["a_full"]) <= ATTN_MAX_REL, seed
+            assert max_rel(host(out["a_delta"]), ref["a_full"] - ref["a_loc"]) <= ATTN_MAX_REL, seed
+        ispa.raise_on_status(status, "dual attention")
