@@ -13,7 +13,10 @@
 //      is factored (and its factor inverted) by one CTA, the panel below and
 //      the panel's rows of the right-hand sides are multiplied by that
 //      inverse, and one split-precision tensor-core product updates the
-//      trailing lower triangle and the remaining right-hand-side rows;
+//      trailing lower triangle from the second column block on and the
+//      remaining right-hand-side rows; the first trailing column block is
+//      updated by the next diagonal step itself, so the chain of diagonal
+//      steps runs on a second stream beside the panels and products;
 //   4. dW = (L^-1)^T (L^-1 S), one split-precision tensor-core product;
 //   5. W_new = W + dW, rounded to W's dtype.
 // Compact form (every other case, and the no-allocation entry point): the
@@ -391,10 +394,12 @@ __global__ void wnew_kernel(const TW* __restrict__ W, const float* __restrict__ 
 // per product), with the right-hand sides carried through the factorisation:
 //   RHS = [S | I] (D x 2D) with S = R W;
 //   for each 64-wide panel k (right-looking):
-//     factor the diagonal block and invert its factor (one CTA);
+//     factor the diagonal block and invert its factor (one CTA), after
+//     applying panel k - 1 to column block k (the other CTAs of that step);
 //     L21 = A21 L_kk^-T for the rows below, and Y_k = L_kk^-1 RHS_k for the
 //     panel's rows of the right-hand sides (final rows of L^-1 S and L^-1);
-//     one tensor-core update [M22 | RHS_2] -= L21 [L21^T | Y_k];
+//     one tensor-core update [M22 | RHS_2] -= L21 [L21^T | Y_k], without
+//     M22's first column block;
 //   after the last panel RHS = [L^-1 S | L^-1], and
 //   dW = (L^-1)^T (L^-1 S) = (G + lambda I)^-1 S is one tensor-core product
 //   whose A operand (L^-1)^T is upper triangular.
@@ -569,71 +574,115 @@ __device__ __forceinline__ void split_store16(const float (&v)[16], float sign, 
   l4[1] = make_uint4(l[4], l[5], l[6], l[7]);
 }
 
-// Factorisation of diagonal block k (one CTA): the block is Dsrc (row stride
-// ld_src) minus Lrow Lrow^T when Lrow (the 64 x 64 block of L to its left in
-// the same block row, row stride D) is given -- the last trailing update,
-// applied here so that the factorisation of block k + 1 can run beside the
-// update product of panel k; the inverse of its Cholesky factor goes to
-// Linv (64 x 64 row-major).  A bad pivot records ISPA_ERR_NOT_SPD and its row.
-__global__ void __launch_bounds__(256) diag_factor_kernel(const float* __restrict__ Dsrc, int64_t ld_src,
-                                                          const float* __restrict__ Lrow, int D, int k,
-                                                          float* __restrict__ Linv, int32_t* status) {
+// 64 x 64 block of a row-major fp32 matrix (row stride ld) into shared memory
+__device__ __forceinline__ void load_block64(float (*S)[kT + 1], const float* __restrict__ src, int64_t ld) {
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = threadIdx.x + 256 * q;
+    v[q] = src[(int64_t)(e >> 6) * ld + (e & 63)];
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e = threadIdx.x + 256 * q;
+    S[e >> 6][e & 63] = v[q];
+  }
+}
+
+// Step k of the chain of diagonal blocks (grid nb - k CTAs; k = 0: one CTA).
+// It finishes the update of column block k by panel k - 1 and factors the
+// diagonal block, reading only column blocks k - 1 and k of M, which the
+// update products of panels <= k - 2 and step k - 1 have completed:
+//   every CTA forms L_{k,k-1} = A_{k,k-1} L_{k-1}^-T (L_{k-1}^-1 from step k - 1);
+//   CTA r > 0 forms L_{k+r,k-1} = A_{k+r,k-1} L_{k-1}^-T and writes
+//     A_{k+r,k} - L_{k+r,k-1} L_{k,k-1}^T back to M;
+//   CTA 0 factors A_kk - L_{k,k-1} L_{k,k-1}^T and writes the inverse of its
+//     Cholesky factor to Linv_k (64 x 64 row-major, at Linv + 64 * 64 k).
+// The tensor-core update of panel k - 1 leaves column block k alone, so this
+// runs beside that panel's own kernels and product.  A bad pivot records
+// ISPA_ERR_NOT_SPD and its row.
+__global__ void __launch_bounds__(256) diag_step_kernel(float* M, int D, int k, float* __restrict__ Linv,
+                                                        int32_t* status) {
   __shared__ float A[kT][kT + 1];
   __shared__ float X[kT][kT + 1];
   __shared__ float T[32][33];
   __shared__ __align__(16) float Ls[32][32];
   __shared__ float rinv[32];
   __shared__ int bad;
-  const int tid = threadIdx.x;
-  float dg[16], lr[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q;
-    dg[q] = Dsrc[(int64_t)(e >> 6) * ld_src + (e & 63)];
-    lr[q] = Lrow ? Lrow[(int64_t)(e >> 6) * D + (e & 63)] : 0.f;
-  }
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q;
-    A[e >> 6][e & 63] = dg[q];
-    X[e >> 6][e & 63] = lr[q];
-  }
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int r = blockIdx.x;
+  const int64_t ld = D;
+  auto block = [&](int bi, int bj) { return M + (int64_t)bi * kT * ld + (int64_t)bj * kT; };
   if (tid == 0) bad = -1;
-  __syncthreads();
-  if (Lrow) {  // A -= Lrow Lrow^T
-    float acc[4][4];
-    mm64(X, X, false, true, acc);
+  if (k == 0) {
+    load_block64(A, block(0, 0), ld);
     __syncthreads();
-    const int tx = tid & 15, ty = tid >> 4;
+  } else {
+    load_block64(A, block(k, k - 1), ld);
+    load_block64(X, Linv + (int64_t)(k - 1) * kT * kT, kT);
+    __syncthreads();
+    float lk[4][4], lr[4][4];
+    mm64(A, X, false, true, lk);  // L_{k,k-1}
+    if (r > 0) {
+      __syncthreads();
+      load_block64(A, block(k + r, k - 1), ld);
+      __syncthreads();
+      mm64(A, X, false, true, lr);  // L_{k+r,k-1}
+    }
+    float* tgt = block(k + r, k);
+    float tv[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] -= acc[a][b];
+      for (int b = 0; b < 4; ++b) tv[a][b] = tgt[(int64_t)(ty + 16 * a) * ld + tx + 16 * b];
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        X[ty + 16 * a][tx + 16 * b] = lk[a][b];
+        A[ty + 16 * a][tx + 16 * b] = r > 0 ? lr[a][b] : lk[a][b];
+      }
+    __syncthreads();
+    float acc[4][4];
+    mm64(A, X, false, true, acc);  // L_{k+r,k-1} L_{k,k-1}^T
+    __syncthreads();
+    if (r > 0) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tgt[(int64_t)(ty + 16 * a) * ld + tx + 16 * b] = tv[a][b] - acc[a][b];
+      return;
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] = tv[a][b] - acc[a][b];
     __syncthreads();
   }
   factor_diag64(A, X, T, Ls, rinv, &bad, k * kT);
   if (tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
   }
+  float* out = Linv + (int64_t)k * kT * kT;
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const int e = tid + 256 * q;
-    Linv[e] = X[e >> 6][e & 63];
+    out[e] = X[e >> 6][e & 63];
   }
 }
 
-// Panel k with L_kk^-1 given (Linv, from diag_factor_kernel):
+// Panel k with L_kk^-1 given (Linv, from diag_step_kernel):
 //   blocks [0, rest): one 64-row block r below the diagonal,
-//     L_rk = A_rk L_kk^-T, written back to M, plus its split operands: -hi/-lo
-//     as K-major [rows, 64] (a_hi, a_lo, local row index) and hi/lo
-//     transposed as [64, ld_t] (lt_hi, lt_lo); block 0 (row block k + 1)
-//     also copies the diagonal block (k + 1, k + 1), as the earlier updates
-//     left it, to dnext before the update product of this panel changes it;
+//     L_rk = A_rk L_kk^-T as split operands only: -hi/-lo as K-major
+//     [rows, 64] (a_hi, a_lo, local row index) and hi/lo transposed as
+//     [64, ld_t] (lt_hi, lt_lo); M is only read (step k + 1 of the diagonal
+//     chain reads the same A_rk beside this kernel);
 //   blocks [rest, rest + ncb): one 64-column block of the panel's
 //     right-hand-side rows, Y = L_kk^-1 RHS_k, written back to RHS, plus hi/lo
 //     [64, ld_y] (y_hi, y_lo).
-__global__ void __launch_bounds__(256) panel_apply_kernel(float* M, int D, int k, int rest, const float* __restrict__ Linv,
-                                                          float* __restrict__ dnext, float* RHS, int64_t rhs_ld,
+__global__ void __launch_bounds__(256) panel_apply_kernel(const float* M, int D, int k, int rest,
+                                                          const float* __restrict__ Linv, float* RHS, int64_t rhs_ld,
                                                           int rhs_cols, __nv_bfloat16* a_hi, __nv_bfloat16* a_lo,
                                                           __nv_bfloat16* lt_hi, __nv_bfloat16* lt_lo, int64_t ld_t,
                                                           __nv_bfloat16* y_hi, __nv_bfloat16* y_lo, int64_t ld_y) {
@@ -651,17 +700,6 @@ __global__ void __launch_bounds__(256) panel_apply_kernel(float* M, int D, int k
     const int e = tid + 256 * q, i = e >> 6, j = e & 63;
     pre[q] = own[(int64_t)i * own_ld + j];
     li[q] = Linv[e];
-  }
-  if (row_block && blockIdx.x == 0) {  // the next diagonal block, before this panel's update reaches it
-    const float* dsrc = M + (int64_t)(k + 1) * kT * D + (int64_t)(k + 1) * kT;
-    float dv[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const int e = tid + 256 * q;
-      dv[q] = dsrc[(int64_t)(e >> 6) * D + (e & 63)];
-    }
-#pragma unroll
-    for (int q = 0; q < 16; ++q) dnext[tid + 256 * q] = dv[q];
   }
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
@@ -690,10 +728,6 @@ __global__ void __launch_bounds__(256) panel_apply_kernel(float* M, int D, int k
   for (int e = 0; e < 16; ++e) v[e] = A[ri][c16 + e];
   if (row_block) {
     const int64_t row0 = (int64_t)blockIdx.x * kT;  // local row of the trailing block
-    float4* dst = reinterpret_cast<float4*>(M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)ri * D +
-                                            (int64_t)k * kT + c16);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     split_store16(v, -1.f, a_hi + (row0 + ri) * 64 + c16, a_lo + (row0 + ri) * 64 + c16);
     // L21^T: row ri of the transpose is column ri of the block
 #pragma unroll
@@ -747,19 +781,18 @@ __global__ void split_rhs_kernel(const float* __restrict__ RHS, int D, __nv_bflo
 }  // namespace simt
 
 // workspace of the tensor-core form: M (4 D^2) | RHS (8 D^2) | split area (4 D^2) |
-// Linv (256 D) | A hi/lo (256 D) | L21^T hi/lo (256 D) | Y_k hi/lo (512 D) | lambda (256) |
-// next diagonal block (16 KB)
+// Linv (256 D) | A hi/lo (256 D) | L21^T hi/lo (256 D) | Y_k hi/lo (512 D) | lambda (256)
 static bool tc_eligible(ispa_dtype_t w_dt, int64_t D) { return w_dt == ISPA_DT_BF16 && D % 128 == 0 && D >= 256; }
-static size_t tc_workspace_bytes(int64_t D) { return (size_t)(16 * D * D + 1280 * D + 256 + 64 * 64 * 4); }
+static size_t tc_workspace_bytes(int64_t D) { return (size_t)(16 * D * D + 1280 * D + 256); }
 static size_t compact_workspace_bytes(int64_t D) { return (size_t)(4 * D * D + 256 * D + 256); }
 
 size_t absorb_workspace_bytes(int64_t D) { return D % 128 == 0 && D >= 256 ? tc_workspace_bytes(D) : compact_workspace_bytes(D); }
 size_t absorb_compact_workspace_bytes(int64_t D) { return compact_workspace_bytes(D); }
 
-ispa_status_t absorb_step_update(int64_t rows, const void* a_hi, const void* a_lo, const void* lt_hi,
-                                 const void* lt_lo, int64_t lt_ld, const void* y_hi, const void* y_lo, int64_t y_ld,
-                                 int64_t rhs_cols, float* m_sub, int64_t m_ld, float* rhs_sub, int64_t rhs_ld,
-                                 cudaStream_t stream);
+ispa_status_t absorb_step_update(int64_t rows, int64_t m_col0, const void* a_hi, const void* a_lo,
+                                 const void* lt_hi, const void* lt_lo, int64_t lt_ld, const void* y_hi,
+                                 const void* y_lo, int64_t y_ld, int64_t rhs_cols, float* m_sub, int64_t m_ld,
+                                 float* rhs_sub, int64_t rhs_ld, cudaStream_t stream);
 ispa_status_t gemm_split3_xt_y(int64_t D, int64_t N, const void* x_hi, const void* x_lo, int64_t x_ld,
                                const void* y_hi, const void* y_lo, int64_t y_ld, float* c, int64_t ldc,
                                cudaStream_t stream);
@@ -833,7 +866,6 @@ static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_
   __nv_bfloat16* y_lo = y_hi + 128 * D64;
   double* lam = reinterpret_cast<double*>(ws + 16 * D64 * D64 + 1280 * D64);
   float* Linv = reinterpret_cast<float*>(ws + 16 * D64 * D64);
-  float* dnext = reinterpret_cast<float*>(ws + 16 * D64 * D64 + 1280 * D64 + 256);
   const int sms = num_sms();
   const int64_t rhs_ld = 2 * D64;
   cudaStream_t side = nullptr;
@@ -850,26 +882,34 @@ static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_
   if (s1 != ISPA_OK) return s1;
   trace_lambda_kernel<<<1, 256, 0, st>>>(G, D, lam_abs, lam_rel, lam);
   shift_kernel<<<sms * 4, 256, 0, st>>>(G, M, D, lam);
-  // the first diagonal block; each later one is factored on the side stream
-  // while the previous panel's update product runs (one-panel look-ahead)
-  diag_factor_kernel<<<1, 256, 0, st>>>(M, D64, nullptr, D, 0, Linv, status);
+  // The chain of diagonal steps runs on the side stream: step k + 1 needs
+  // step k and the update product of panel k - 1 only, so it runs beside
+  // panel k's kernel and product on the main stream, which need step k (and
+  // the product of panel k - 1, earlier on the same stream).  Host order
+  // keeps one event per direction: ev_join marks the latest diagonal step,
+  // ev_fork the latest update product, each waited on before it is recorded
+  // again.
+  diag_step_kernel<<<1, 256, 0, st>>>(M, D, 0, Linv, status);
+  if (nb > 1 && (cudaEventRecord(ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess))
+    return check_launch("absorb fork");
   for (int k = 0; k < nb; ++k) {
     const int rest = nb - k - 1;
     const int off = (k + 1) * kT;
     const int rhs_cols = D + off;  // nonzero columns of the panel's rows of [L^-1 S | L^-1]
-    float* Lk = Linv + (int64_t)k * kT * kT;
+    if (k > 0 && cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess) return check_launch("absorb join");
     panel_apply_kernel<<<rest + (rhs_cols + kT - 1) / kT, 256, 0, st>>>(
-        M, D, k, rest, Lk, dnext, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld);
+        M, D, k, rest, Linv + (int64_t)k * kT * kT, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi,
+        y_lo, rhs_ld);
     if (rest > 0) {
-      if (cudaEventRecord(ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess)
-        return check_launch("absorb fork");
-      diag_factor_kernel<<<1, 256, 0, side>>>(dnext, kT, M + (int64_t)off * D + (int64_t)k * kT, D, k + 1,
-                                              Lk + kT * kT, status);
+      diag_step_kernel<<<rest, 256, 0, side>>>(M, D, k + 1, Linv, status);
       if (cudaEventRecord(ev_join, side) != cudaSuccess) return check_launch("absorb join");
-      s1 = absorb_step_update(D - off, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, rhs_cols,
+      // trailing columns from block k + 2: step k + 1 updates block k + 1
+      s1 = absorb_step_update(D - off, kT, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, rhs_cols,
                               M + (int64_t)off * D + off, D64, RHS + (int64_t)off * rhs_ld, rhs_ld, st);
       if (s1 != ISPA_OK) return s1;
-      if (cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess) return check_launch("absorb join");
+      if (rest > 1 &&
+          (cudaEventRecord(ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess))
+        return check_launch("absorb fork");
     }
   }
   // dW = (L^-1)^T (L^-1 S): hi/lo of L^-1 S into M's storage, of L^-1 into the split area

@@ -746,24 +746,30 @@ namespace ispa {
 
 // One trailing update of the blocked Cholesky with its right-hand sides
 // (panel width 64, rows and columns from `off`):
-//   M[off:, off:] (lower tiles) += A  [L^T]      A = -L21 (rows x 64),
-//   RHS[off:, :rhs_cols]        += A  Y_k        Y_k (64 x rhs_cols),
+//   M[off:, off + m_col0:] (lower tiles) += A  [L^T](:, m_col0:)   A = -L21 (rows x 64),
+//   RHS[off:, :rhs_cols]                 += A  Y_k                 Y_k (64 x rhs_cols),
 // A given as K-major hi/lo [rows, 64]; L21^T as MN-major hi/lo [64, rows]
 // with row stride lt_ld; Y_k as MN-major hi/lo [64, rhs_cols] with row stride
 // y_ld.  M has row stride D, RHS row stride rhs_ld (fp32, reduced in L2).
-ispa_status_t absorb_step_update(int64_t rows, const void* a_hi, const void* a_lo, const void* lt_hi,
-                                 const void* lt_lo, int64_t lt_ld, const void* y_hi, const void* y_lo, int64_t y_ld,
-                                 int64_t rhs_cols, float* m_sub, int64_t m_ld, float* rhs_sub, int64_t rhs_ld,
-                                 cudaStream_t stream) {
+// m_col0 (a multiple of 64) leaves the first trailing columns to the caller.
+ispa_status_t absorb_step_update(int64_t rows, int64_t m_col0, const void* a_hi, const void* a_lo,
+                                 const void* lt_hi, const void* lt_lo, int64_t lt_ld, const void* y_hi,
+                                 const void* y_lo, int64_t y_ld, int64_t rhs_cols, float* m_sub, int64_t m_ld,
+                                 float* rhs_sub, int64_t rhs_ld, cudaStream_t stream) {
   using namespace gemm;
   constexpr int BN = 128;
+  if (m_col0 < 0 || m_col0 > rows || m_col0 % 64) return unsupported("absorb update: first trailing column");
+  const int64_t m_cols = rows - m_col0;  // trailing columns this product updates
   Params p;
   memset(&p, 0, sizeof(p));
   CUtensorMap ah, al, bh0, bl0, bh1, bl1;
   if (!encode_map_bf16_2d(&ah, a_hi, 64, rows, 128, 64, kBM) || !encode_map_bf16_2d(&al, a_lo, 64, rows, 128, 64, kBM))
     return ISPA_ERR_CUDA;
-  if (!encode_map_bf16_2d(&bh0, lt_hi, rows, 64, lt_ld * 2, 64, 64) ||
-      !encode_map_bf16_2d(&bl0, lt_lo, rows, 64, lt_ld * 2, 64, 64))
+  // with no trailing column left the first range is empty and its maps are
+  // never read: they are encoded over the whole block so that they are valid
+  const int64_t b0 = m_cols > 0 ? m_col0 : 0, nb0 = m_cols > 0 ? m_cols : rows;
+  if (!encode_map_bf16_2d(&bh0, static_cast<const __nv_bfloat16*>(lt_hi) + b0, nb0, 64, lt_ld * 2, 64, 64) ||
+      !encode_map_bf16_2d(&bl0, static_cast<const __nv_bfloat16*>(lt_lo) + b0, nb0, 64, lt_ld * 2, 64, 64))
     return ISPA_ERR_CUDA;
   if (!encode_map_bf16_2d(&bh1, y_hi, rhs_cols, 64, y_ld * 2, 64, 64) ||
       !encode_map_bf16_2d(&bl1, y_lo, rhs_cols, 64, y_ld * 2, 64, 64))
@@ -772,19 +778,21 @@ ispa_status_t absorb_step_update(int64_t rows, const void* a_hi, const void* a_l
   p.b_map[0][0] = bh0, p.b_map[0][1] = bl0, p.b_map[0][2] = bh0;
   p.b_map[1][0] = bh1, p.b_map[1][1] = bl1, p.b_map[1][2] = bh1;
   p.n_pairs = 3;
-  if (!encode_map_out_2d(&p.c_map[0], m_sub, true, rows, rows, m_ld * 4) ||
+  if (!encode_map_out_2d(&p.c_map[0], m_sub + b0, true, nb0, rows, m_ld * 4) ||
       !encode_map_out_2d(&p.c_map[1], rhs_sub, true, rhs_cols, rows, rhs_ld * 4))
     return ISPA_ERR_CUDA;
   p.c_tma = 1;
-  p.c[0] = m_sub;
+  p.c[0] = m_sub + b0;
   p.c[1] = rhs_sub;
   p.M = (int32_t)rows;
   p.K = 64;
   p.k_per_split = 64;
-  p.n_split = (int32_t)((rows + BN - 1) / BN * BN);  // range 0 padded to whole tiles
+  p.n_split = (int32_t)((m_cols + BN - 1) / BN * BN);  // range 0 padded to whole tiles
   p.N = p.n_split + (int32_t)rhs_cols;
-  p.n_cols[0] = (int32_t)rows;
+  p.n_cols[0] = (int32_t)m_cols;
   p.n_cols[1] = (int32_t)rhs_cols;
+  // tiles wholly above the diagonal are skipped; the column shift only makes
+  // the test keep a few more tiles than the triangle needs
   p.lower_only0 = 1;
   p.mode = kReduceF32;
   return launch<false, true, BN, 4>(p, 1, stream);

@@ -101,7 +101,7 @@ def absorb_launches(D: int) -> int:
     """Kernel launches of one tensor-core absorb solve (bf16 W, D % 128 == 0):
     split of R, [0 | I] fill, S = R W, trace, shift and the first diagonal
     factorisation; per 64-wide panel its application, and for every panel but
-    the last the next diagonal factorisation (side stream) and the update
+    the last the next diagonal step (side stream) and the update
     product; the split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new."""
     nb = D // 64
     return 6 + nb + 2 * (nb - 1) + 3
