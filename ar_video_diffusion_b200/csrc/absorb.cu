@@ -322,6 +322,55 @@ __device__ __forceinline__ void mm64(const float (*Ps)[kT + 1], const float (*Qs
   }
 }
 
+// 64 x 64 operands stored with the contraction index first (row stride
+// kLdv, rows 16-byte aligned): acc[a][b] = sum_t P[t][4 ty + a] Q[t][4 tx + b].
+// Per t a warp reads one 16-byte vector of P (two addresses, one wavefront)
+// and sixteen of Q (256 contiguous bytes, two wavefronts), against eight
+// scalar wavefronts in mm64.
+constexpr int kLdv = kT + 4;
+__device__ __forceinline__ void mm64v(const float (*P)[kLdv], const float (*Q)[kLdv], float (&acc)[4][4]) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+#pragma unroll 8
+  for (int t = 0; t < kT; ++t) {
+    const float4 pv = *reinterpret_cast<const float4*>(&P[t][4 * ty]);
+    const float4 qv = *reinterpret_cast<const float4*>(&Q[t][4 * tx]);
+    const float pa[4] = {pv.x, pv.y, pv.z, pv.w}, qb[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(pa[a], qb[b], acc[a][b]);
+  }
+}
+
+// 64 x 64 block of a row-major fp32 matrix (row stride ld, 16-byte aligned
+// rows) into shared memory as it is (S[i][j] = G[i][j]) or transposed
+// (S[j][i] = G[i][j]; consecutive threads take consecutive rows, so the
+// scalar stores hit distinct banks)
+__device__ __forceinline__ void load_n64(float (*S)[kLdv], const float* __restrict__ G, int64_t ld) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = threadIdx.x + 256 * q, i = e >> 4, j = (e & 15) * 4;
+    *reinterpret_cast<float4*>(&S[i][j]) = *reinterpret_cast<const float4*>(G + (int64_t)i * ld + j);
+  }
+}
+__device__ __forceinline__ void load_t64(float (*S)[kLdv], const float* __restrict__ G, int64_t ld) {
+  float4 v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = threadIdx.x + 256 * q, i = e & 63, j = (e >> 6) * 4;
+    v[q] = *reinterpret_cast<const float4*>(G + (int64_t)i * ld + j);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = threadIdx.x + 256 * q, i = e & 63, j = (e >> 6) * 4;
+    S[j][i] = v[q].x, S[j + 1][i] = v[q].y, S[j + 2][i] = v[q].z, S[j + 3][i] = v[q].w;
+  }
+}
+
 // Panel below diagonal block k: M[r, k] <- M[r, k] Linv_k^T, one 64-row block per CTA.
 __global__ void __launch_bounds__(256) panel_kernel(float* M, int D, int k, const float* __restrict__ Linv) {
   __shared__ float Li[kT][kT + 1];
@@ -452,25 +501,30 @@ __device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], fl
   }
 }
 
-// Column `lane` of X = L^-1 for the 32 x 32 lower-triangular L whose columns
-// chol32_rot left shifted in Ls (rinv: reciprocals of its diagonal), by one
-// warp: column-oriented forward elimination with the right-hand side rotated
-// in registers; X[m][lane] written with row stride ldx.
-__device__ __forceinline__ void inv32_rot(const float (*Ls)[32], const float* rinv, float* X, int ldx, int lane) {
-  float b[32];
+// Forward elimination x = L^-1 b for the 32 x 32 lower-triangular L whose
+// columns chol32_rot left shifted in Ls (rinv: reciprocals of its diagonal),
+// by one warp with one right-hand side per lane, rotated in registers
+// (b[0] is the current row); x[m] goes to out[m * s_m + lane * s_l].  The
+// column for step m + 1 is loaded while step m runs, so a step's chain is
+// one multiply and one multiply-add.
+__device__ __forceinline__ void trsv32_rot(const float (*Ls)[32], const float* rinv, float (&b)[32], float* out,
+                                           int s_m, int s_l, int lane) {
+  float4 nx[8];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
+  for (int q = 0; q < 8; ++q) nx[q] = reinterpret_cast<const float4*>(Ls[0])[q];
+  float rn = rinv[0];
 #pragma unroll 1
   for (int m = 0; m < 32; ++m) {
-    const float4* col = reinterpret_cast<const float4*>(Ls[m]);
     float lr[32];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 v = col[q];
-      lr[4 * q] = v.x, lr[4 * q + 1] = v.y, lr[4 * q + 2] = v.z, lr[4 * q + 3] = v.w;
-    }
-    const float x = b[0] * rinv[m];
-    X[m * ldx + lane] = x;
+    for (int q = 0; q < 8; ++q) lr[4 * q] = nx[q].x, lr[4 * q + 1] = nx[q].y, lr[4 * q + 2] = nx[q].z, lr[4 * q + 3] = nx[q].w;
+    const float rm = rn;
+    const float4* nxt = reinterpret_cast<const float4*>(Ls[(m + 1) & 31]);  // wraps harmlessly after the last
+#pragma unroll
+    for (int q = 0; q < 8; ++q) nx[q] = nxt[q];
+    rn = rinv[(m + 1) & 31];
+    const float x = b[0] * rm;
+    out[m * s_m + lane * s_l] = x;
 #pragma unroll
     for (int c = 1; c < 32; ++c) b[c - 1] = b[c] - lr[c] * x;
     b[31] = 0.f;
@@ -479,10 +533,14 @@ __device__ __forceinline__ void inv32_rot(const float (*Ls)[32], const float* ri
 
 // Cholesky factor of the 64 x 64 block in A (shared, row stride 65; lower
 // triangle used) and the inverse X of that factor (shared, row stride 65),
-// by the 256 threads of a CTA: L11 = chol(A11) and X11 by warp 0,
-// L21 = A21 X11^T, A22 - L21 L21^T, L22 = chol(.) and X22 by warp 0,
-// X21 = -X22 (L21 X11).  T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned;
-// rinv: 32 floats.
+// by the 256 threads of a CTA:
+//   L11 = chol(A11) by warp 0;
+//   then at once X11 = L11^-1 (warp 0) and L21 = A21 L11^-T (warp 1, a row
+//   of A21 per lane, solved in place);
+//   A22 - L21 L21^T (all);
+//   then at once L22 = chol(.) (warp 0) and T = L21 X11 (warps 4-7);
+//   X22 = L22^-1 (warp 0); X21 = -X22 T (all).
+// T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned; rinv: 32 floats.
 __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], float (*Ls)[32], float* rinv,
                               int* bad, int base) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -493,24 +551,17 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
     const int e = tid + 256 * q;
     X[e >> 5][32 + (e & 31)] = 0.f;
   }
-  if (warp == 0) {
-    chol32_rot(&A[0][0], 65, Ls, rinv, lane, base, bad);
-    __syncwarp();
-    inv32_rot(Ls, rinv, &X[0][0], 65, lane);
-  }
+  if (warp == 0) chol32_rot(&A[0][0], 65, Ls, rinv, lane, base, bad);
   __syncthreads();
-  float acc[4];
+  if (warp < 2) {
+    float b[32];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {  // L21 = A21 X11^T
-    const int j = pj + 8 * b;
-    float v = 0.f;
-#pragma unroll 8
-    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * X[j][m];
-    acc[b] = v;
+    for (int c = 0; c < 32; ++c) b[c] = warp == 0 ? (c == lane ? 1.f : 0.f) : A[32 + lane][c];
+    if (warp == 0)
+      trsv32_rot(Ls, rinv, b, &X[0][0], 65, 1, lane);  // column `lane` of X11
+    else
+      trsv32_rot(Ls, rinv, b, &A[32][0], 1, 65, lane);  // row `lane` of L21
   }
-  __syncthreads();
-#pragma unroll
-  for (int b = 0; b < 4; ++b) A[32 + pi][pj + 8 * b] = acc[b];
   __syncthreads();
 #pragma unroll
   for (int b = 0; b < 4; ++b) {  // A22 -= L21 L21^T
@@ -524,16 +575,23 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
   if (warp == 0) {
     chol32_rot(&A[32][32], 65, Ls, rinv, lane, base + 32, bad);
     __syncwarp();
-    inv32_rot(Ls, rinv, &X[32][32], 65, lane);
-  }
-  __syncthreads();
+    float b[32];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {  // T = L21 X11
-    const int j = pj + 8 * b;
-    float v = 0.f;
-#pragma unroll 8
-    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * X[m][j];
-    T[pi][j] = v;
+    for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
+    trsv32_rot(Ls, rinv, b, &X[32][32], 65, 1, lane);
+  } else if (warp >= 4) {  // T = L21 X11: 128 threads, row ti, columns tj + 4 b
+    const int ti = (tid - 128) >> 2, tj = tid & 3;
+    float v[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) v[b] = 0.f;
+#pragma unroll 4
+    for (int m = 0; m < 32; ++m) {
+      const float a = A[32 + ti][m];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) v[b] = fmaf(a, X[m][tj + 4 * b], v[b]);
+    }
+#pragma unroll
+    for (int b = 0; b < 8; ++b) T[ti][tj + 4 * b] = v[b];
   }
   __syncthreads();
 #pragma unroll
@@ -603,61 +661,70 @@ __device__ __forceinline__ void load_block64(float (*S)[kT + 1], const float* __
 // ISPA_ERR_NOT_SPD and its row.
 __global__ void __launch_bounds__(256) diag_step_kernel(float* M, int D, int k, float* __restrict__ Linv,
                                                         int32_t* status) {
-  __shared__ float A[kT][kT + 1];
-  __shared__ float X[kT][kT + 1];
+  // the products' operands, contraction index first; then the block to
+  // factor (A) and its inverse factor (X), row stride 65, in the same storage
+  __shared__ __align__(16) float U[kT][kLdv];
+  __shared__ __align__(16) float V[kT][kLdv];
   __shared__ float T[32][33];
   __shared__ __align__(16) float Ls[32][32];
   __shared__ float rinv[32];
   __shared__ int bad;
+  auto A = reinterpret_cast<float (*)[kT + 1]>(&U[0][0]);
+  auto X = reinterpret_cast<float (*)[kT + 1]>(&V[0][0]);
+  // the next step may be resident early: it waits below for this grid's end
+  asm volatile("griddepcontrol.launch_dependents;");
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int r = blockIdx.x;
   const int64_t ld = D;
   auto block = [&](int bi, int bj) { return M + (int64_t)bi * kT * ld + (int64_t)bj * kT; };
   if (tid == 0) bad = -1;
+  // every read of M and Linv follows the completion of the previous step
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (k == 0) {
     load_block64(A, block(0, 0), ld);
     __syncthreads();
   } else {
-    load_block64(A, block(k, k - 1), ld);
-    load_block64(X, Linv + (int64_t)(k - 1) * kT * kT, kT);
+    load_t64(U, block(k, k - 1), ld);                   // U[t][i] = A_{k,k-1}[i][t]
+    load_t64(V, Linv + (int64_t)(k - 1) * kT * kT, kT);  // V[t][j] = L_{k-1}^-1[j][t]
     __syncthreads();
     float lk[4][4], lr[4][4];
-    mm64(A, X, false, true, lk);  // L_{k,k-1}
+    mm64v(U, V, lk);  // L_{k,k-1}
     if (r > 0) {
       __syncthreads();
-      load_block64(A, block(k + r, k - 1), ld);
+      load_t64(U, block(k + r, k - 1), ld);
       __syncthreads();
-      mm64(A, X, false, true, lr);  // L_{k+r,k-1}
+      mm64v(U, V, lr);  // L_{k+r,k-1}
     }
     float* tgt = block(k + r, k);
-    float tv[4][4];
+    float4 tv[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) tv[a][b] = tgt[(int64_t)(ty + 16 * a) * ld + tx + 16 * b];
+    for (int a = 0; a < 4; ++a) tv[a] = *reinterpret_cast<const float4*>(tgt + (int64_t)(4 * ty + a) * ld + 4 * tx);
     __syncthreads();
+    // U[t][i] = L_{k+r,k-1}[i][t], V[t][j] = L_{k,k-1}[j][t]
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        X[ty + 16 * a][tx + 16 * b] = lk[a][b];
-        A[ty + 16 * a][tx + 16 * b] = r > 0 ? lr[a][b] : lk[a][b];
-      }
+    for (int b = 0; b < 4; ++b) {
+      const float(&w)[4][4] = r > 0 ? lr : lk;
+      *reinterpret_cast<float4*>(&U[4 * tx + b][4 * ty]) = make_float4(w[0][b], w[1][b], w[2][b], w[3][b]);
+      *reinterpret_cast<float4*>(&V[4 * tx + b][4 * ty]) = make_float4(lk[0][b], lk[1][b], lk[2][b], lk[3][b]);
+    }
     __syncthreads();
     float acc[4][4];
-    mm64(A, X, false, true, acc);  // L_{k+r,k-1} L_{k,k-1}^T
+    mm64v(U, V, acc);  // L_{k+r,k-1} L_{k,k-1}^T
     __syncthreads();
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      tv[a].x -= acc[a][0], tv[a].y -= acc[a][1], tv[a].z -= acc[a][2], tv[a].w -= acc[a][3];
+    }
     if (r > 0) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) tgt[(int64_t)(ty + 16 * a) * ld + tx + 16 * b] = tv[a][b] - acc[a][b];
+      for (int a = 0; a < 4; ++a) *reinterpret_cast<float4*>(tgt + (int64_t)(4 * ty + a) * ld + 4 * tx) = tv[a];
       return;
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] = tv[a][b] - acc[a][b];
+    for (int a = 0; a < 4; ++a) {
+      float* row = &A[4 * ty + a][4 * tx];
+      row[0] = tv[a].x, row[1] = tv[a].y, row[2] = tv[a].z, row[3] = tv[a].w;
+    }
     __syncthreads();
   }
   factor_diag64(A, X, T, Ls, rinv, &bad, k * kT);
@@ -686,41 +753,35 @@ __global__ void __launch_bounds__(256) panel_apply_kernel(const float* M, int D,
                                                           int rhs_cols, __nv_bfloat16* a_hi, __nv_bfloat16* a_lo,
                                                           __nv_bfloat16* lt_hi, __nv_bfloat16* lt_lo, int64_t ld_t,
                                                           __nv_bfloat16* y_hi, __nv_bfloat16* y_lo, int64_t ld_y) {
-  __shared__ float A[kT][kT + 1];  // this CTA's block, then its result
-  __shared__ float X[kT][kT + 1];  // L_kk^-1
+  // operands with the contraction index first; the result then goes through
+  // the storage of the first, row stride 65
+  __shared__ __align__(16) float U[kT][kLdv];  // this CTA's block
+  __shared__ __align__(16) float V[kT][kLdv];  // V[t][j] = L_kk^-1[j][t]
+  auto A = reinterpret_cast<float (*)[kT + 1]>(&U[0][0]);
   const int tid = threadIdx.x;
   const bool row_block = (int)blockIdx.x < rest;
   const int c0 = row_block ? 0 : ((int)blockIdx.x - rest) * kT;
   const float* own = row_block ? M + (int64_t)(k + 1 + blockIdx.x) * kT * D + (int64_t)k * kT
                                : RHS + (int64_t)k * kT * rhs_ld + c0;
-  const int64_t own_ld = row_block ? D : rhs_ld;
-  float pre[16], li[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q, i = e >> 6, j = e & 63;
-    pre[q] = own[(int64_t)i * own_ld + j];
-    li[q] = Linv[e];
-  }
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e = tid + 256 * q;
-    A[e >> 6][e & 63] = pre[q];
-    X[e >> 6][e & 63] = li[q];
-  }
+  load_t64(V, Linv, kT);
+  if (row_block)
+    load_t64(U, own, D);  // U[t][i] = A_rk[i][t]
+  else
+    load_n64(U, own, rhs_ld);  // U[t][j] = RHS_k[t][j]
   __syncthreads();
   const int tx = tid & 15, ty = tid >> 4;
   float acc[4][4];
   if (row_block)
-    mm64(A, X, false, true, acc);  // A_rk L_kk^-T
+    mm64v(U, V, acc);  // A_rk L_kk^-T
   else
-    mm64(X, A, false, false, acc);  // L_kk^-1 RHS_k
+    mm64v(V, U, acc);  // L_kk^-1 RHS_k
   __syncthreads();
   // the 64 x 64 result through shared memory, so that every global store
   // below is a 16-byte vector of one row
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) A[ty + 16 * a][tx + 16 * b] = acc[a][b];
+    for (int b = 0; b < 4; ++b) A[4 * ty + a][4 * tx + b] = acc[a][b];
   __syncthreads();
   const int ri = tid >> 2, c16 = (tid & 3) * 16;  // this thread: row (or column) ri, 16 values from c16
   float v[16];
@@ -901,7 +962,19 @@ static ispa_status_t absorb_solve_tc(const float* G, const float* R, const __nv_
         M, D, k, rest, Linv + (int64_t)k * kT * kT, RHS, rhs_ld, rhs_cols, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi,
         y_lo, rhs_ld);
     if (rest > 0) {
-      diag_step_kernel<<<rest, 256, 0, side>>>(M, D, k + 1, Linv, status);
+      // programmatic launch: the step's CTAs may become resident while the
+      // previous step runs (the kernel waits for its end before any read)
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)rest);
+      cfg.blockDim = dim3(256);
+      cfg.stream = side;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, diag_step_kernel, M, D, k + 1, Linv, status) != cudaSuccess)
+        return check_launch("absorb diagonal step");
       if (cudaEventRecord(ev_join, side) != cudaSuccess) return check_launch("absorb join");
       // trailing columns from block k + 2: step k + 1 updates block k + 1
       s1 = absorb_step_update(D - off, kT, a_hi, a_lo, lt_hi, lt_lo, D64, y_hi, y_lo, rhs_ld, rhs_cols,
