@@ -32,11 +32,10 @@ def test_solve_flops_and_launch_count():
     assert bench.solve_flops(D) == pytest.approx(15.7e9, rel=3e-3)
     nb = D // 64
     # tensor-core form: split of R, [0 | I] fill, S = R W, trace, shift, the
-    # first diagonal factorisation; nb panel applications, nb-1 further
-    # diagonal factorisations (one panel ahead) and nb-1 update products; the
-    # split of [L^-1 S | L^-1], dW = (L^-1)^T (L^-1 S), W_new (an ncu launch
-    # list shows 24 diag_factor_kernel and 24 panel_apply_kernel launches per
-    # D = 1536 solve).
+    # first diagonal step; nb panel applications, nb-1 further diagonal steps
+    # (side stream) and nb-1 update products; the split of [L^-1 S | L^-1],
+    # dW = (L^-1)^T (L^-1 S), W_new (an ncu launch list shows 24
+    # diag_step_kernel and 24 panel_apply_kernel launches per D = 1536 solve).
     assert bench.absorb_launches(D) == 6 + nb + 2 * (nb - 1) + 3 == 79
 
 
