@@ -6,7 +6,8 @@
 * The statistics (G, R, E) split the token range across CTAs and add the
   partial sums into the outputs with L2 reductions, whose order is not fixed,
   so they are reproducible only up to fp32 rounding of the summation order;
-  the absorb solve consumes them (its own kernels are order-fixed).  Three runs
+  the absorb solve consumes them, and its last product (dW) splits its K
+  range the same way.  Three runs
   must agree within a bound far below the oracle tolerances: 1e-5 relative
   (Frobenius) for G, R and 1e-4 for dW, which amplifies the statistics'
   rounding by cond(G + lambda I) (hundreds here)."""
