@@ -478,7 +478,8 @@ __device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], fl
       if (lane == 0 && *bad < 0) *bad = base + j;
       d = 1.f;
     }
-    const float r = rsqrtf(d);
+    float r;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));  // d > 0 and finite here
     const float l = lane == j ? d * r : (lane > j ? a[0] * r : 0.f);
     // the next pivot: lane j + 1's entry (j + 1, j + 1) less its own l squared
     const float dn = __shfl_sync(0xffffffffu, a[1] - l * l, (j + 1) & 31);
@@ -508,7 +509,7 @@ __device__ __forceinline__ void chol32_rot(float* A, int ld, float (*Ls)[32], fl
 // column for step m + 1 is loaded while step m runs, so a step's chain is
 // one multiply and one multiply-add.
 __device__ __forceinline__ void trsv32_rot(const float (*Ls)[32], const float* rinv, float (&b)[32], float* out,
-                                           int s_m, int s_l, int lane) {
+                                           int s_m, int s_l, int lane, float* out_t = nullptr, int t_ld = 0) {
   float4 nx[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) nx[q] = reinterpret_cast<const float4*>(Ls[0])[q];
@@ -525,6 +526,7 @@ __device__ __forceinline__ void trsv32_rot(const float (*Ls)[32], const float* r
     rn = rinv[(m + 1) & 31];
     const float x = b[0] * rm;
     out[m * s_m + lane * s_l] = x;
+    if (out_t) out_t[m * t_ld + lane] = x;  // the same value, x[m] of lane at [m][lane]
 #pragma unroll
     for (int c = 1; c < 32; ++c) b[c - 1] = b[c] - lr[c] * x;
     b[31] = 0.f;
@@ -536,16 +538,18 @@ __device__ __forceinline__ void trsv32_rot(const float (*Ls)[32], const float* r
 // by the 256 threads of a CTA:
 //   L11 = chol(A11) by warp 0;
 //   then at once X11 = L11^-1 (warp 0) and L21 = A21 L11^-T (warp 1, a row
-//   of A21 per lane, solved in place);
-//   A22 - L21 L21^T (all);
-//   then at once L22 = chol(.) (warp 0) and T = L21 X11 (warps 4-7);
+//   of A21 per lane, solved in place and also stored transposed in Lt);
+//   A22 - L21 L21^T (all, from Lt);
+//   then at once L22 = chol(.) (warp 0) and T = L21 X11 (warps 1, 2, 3 and
+//   5, which leave warp 0's scheduler to it);
 //   X22 = L22^-1 (warp 0); X21 = -X22 T (all).
-// T: 32 x 33 scratch; Ls: 32 x 32, 16-byte aligned; rinv: 32 floats.
-__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], float (*Ls)[32], float* rinv,
-                              int* bad, int base) {
+// The 32 x 32 products read two-element vectors of an operand stored with
+// the contraction index first.  T, Lt: 32 x 36 scratch (8-byte aligned
+// rows); Ls: 32 x 32, 16-byte aligned; rinv: 32 floats.
+__device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[36], float (*Lt)[36], float (*Ls)[32],
+                              float* rinv, int* bad, int base) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // element (i, j) of a 32 x 32 product: i = tid / 8, j = tid % 8 + 8 b
-  const int pi = tid >> 3, pj = tid & 7;
+  const int ti = tid >> 4, tj = tid & 15;  // a 2 x 2 block of a 32 x 32 product
 #pragma unroll
   for (int q = 0; q < 4; ++q) {  // the upper right quarter of X is zero
     const int e = tid + 256 * q;
@@ -560,16 +564,22 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
     if (warp == 0)
       trsv32_rot(Ls, rinv, b, &X[0][0], 65, 1, lane);  // column `lane` of X11
     else
-      trsv32_rot(Ls, rinv, b, &A[32][0], 1, 65, lane);  // row `lane` of L21
+      trsv32_rot(Ls, rinv, b, &A[32][0], 1, 65, lane, &Lt[0][0], 36);  // row `lane` of L21
   }
   __syncthreads();
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {  // A22 -= L21 L21^T
-    const int j = pj + 8 * b;
-    float v = 0.f;
+  {  // A22 -= L21 L21^T: rows 2 ti + a, columns 2 tj + c
+    float v[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll 8
-    for (int m = 0; m < 32; ++m) v += A[32 + pi][m] * A[32 + j][m];
-    A[32 + pi][32 + j] -= v;
+    for (int m = 0; m < 32; ++m) {
+      const float2 p = *reinterpret_cast<const float2*>(&Lt[m][2 * ti]);
+      const float2 q = *reinterpret_cast<const float2*>(&Lt[m][2 * tj]);
+      v[0][0] = fmaf(p.x, q.x, v[0][0]), v[0][1] = fmaf(p.x, q.y, v[0][1]);
+      v[1][0] = fmaf(p.y, q.x, v[1][0]), v[1][1] = fmaf(p.y, q.y, v[1][1]);
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) A[32 + 2 * ti + a][32 + 2 * tj + c] -= v[a][c];
   }
   __syncthreads();
   if (warp == 0) {
@@ -579,28 +589,40 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[33], fl
 #pragma unroll
     for (int c = 0; c < 32; ++c) b[c] = c == lane ? 1.f : 0.f;
     trsv32_rot(Ls, rinv, b, &X[32][32], 65, 1, lane);
-  } else if (warp >= 4) {  // T = L21 X11: 128 threads, row ti, columns tj + 4 b
-    const int ti = (tid - 128) >> 2, tj = tid & 3;
-    float v[8];
-#pragma unroll
-    for (int b = 0; b < 8; ++b) v[b] = 0.f;
+  } else if (warp <= 3 || warp == 5) {  // T = L21 X11: 128 threads, rows 2 ui + a, columns uj + 4 c
+    const int u = (warp <= 3 ? warp - 1 : 3) * 32 + lane;
+    const int ui = u >> 3, uj = u & 7;  // ui < 16
+    float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll 4
     for (int m = 0; m < 32; ++m) {
-      const float a = A[32 + ti][m];
+      const float2 p = *reinterpret_cast<const float2*>(&Lt[m][2 * ui]);
 #pragma unroll
-      for (int b = 0; b < 8; ++b) v[b] = fmaf(a, X[m][tj + 4 * b], v[b]);
+      for (int c = 0; c < 4; ++c) {
+        const float x = X[m][uj + 8 * c];
+        v[0][c] = fmaf(p.x, x, v[0][c]);
+        v[1][c] = fmaf(p.y, x, v[1][c]);
+      }
     }
 #pragma unroll
-    for (int b = 0; b < 8; ++b) T[ti][tj + 4 * b] = v[b];
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) T[2 * ui + a][uj + 8 * c] = v[a][c];
   }
   __syncthreads();
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {  // X21 = -X22 T
-    const int j = pj + 8 * b;
-    float v = 0.f;
+  {  // X21 = -X22 T: rows ti and ti + 16, columns 2 tj + c
+    float v[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll 8
-    for (int m = 0; m < 32; ++m) v += X[32 + pi][32 + m] * T[m][j];
-    X[32 + pi][j] = -v;
+    for (int m = 0; m < 32; ++m) {
+      const float x0 = X[32 + ti][32 + m], x1 = X[48 + ti][32 + m];
+      const float2 t = *reinterpret_cast<const float2*>(&T[m][2 * tj]);
+      v[0][0] = fmaf(x0, t.x, v[0][0]), v[0][1] = fmaf(x0, t.y, v[0][1]);
+      v[1][0] = fmaf(x1, t.x, v[1][0]), v[1][1] = fmaf(x1, t.y, v[1][1]);
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      X[32 + ti][2 * tj + c] = -v[0][c];
+      X[48 + ti][2 * tj + c] = -v[1][c];
+    }
   }
   __syncthreads();
 }
@@ -665,7 +687,8 @@ __global__ void __launch_bounds__(256) diag_step_kernel(float* M, int D, int k, 
   // factor (A) and its inverse factor (X), row stride 65, in the same storage
   __shared__ __align__(16) float U[kT][kLdv];
   __shared__ __align__(16) float V[kT][kLdv];
-  __shared__ float T[32][33];
+  __shared__ __align__(16) float T[32][36];
+  __shared__ __align__(16) float Lt[32][36];
   __shared__ __align__(16) float Ls[32][32];
   __shared__ float rinv[32];
   __shared__ int bad;
@@ -727,7 +750,7 @@ __global__ void __launch_bounds__(256) diag_step_kernel(float* M, int D, int k, 
     }
     __syncthreads();
   }
-  factor_diag64(A, X, T, Ls, rinv, &bad, k * kT);
+  factor_diag64(A, X, T, Lt, Ls, rinv, &bad, k * kT);
   if (tid == 0 && bad >= 0 && status) {
     if (atomicCAS(status, 0, (int32_t)ISPA_ERR_NOT_SPD) == 0) status[1] = bad;
   }
