@@ -627,12 +627,6 @@ __device__ void factor_diag64(float (*A)[65], float (*X)[65], float (*T)[36], fl
   __syncthreads();
 }
 
-__device__ __forceinline__ void split_store(float v, __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t i) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  hi[i] = h;
-  lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
-}
-
 // 16 consecutive values (times `sign`) as bf16 hi and lo halves, two 16-byte
 // stores each (hi and lo 32-byte aligned)
 __device__ __forceinline__ void split_store16(const float (&v)[16], float sign, __nv_bfloat16* hi,
