@@ -203,9 +203,11 @@ ISPA_API size_t ispa_absorb_workspace_bytes(int64_t d_model);
  * cores in split precision (bf16 hi/lo pairs, about 2^-17 relative per
  * product) and the solves are carried through the factorisation; otherwise
  * (fp32 W, other sizes) the updates run on the CUDA cores in fp32.  The
- * tensor-core form factors each next diagonal block on an internal stream
- * beside the current update (fork and join by events recorded on `stream`, so
- * the call stays asynchronous and graph capture sees one fork/join per panel);
+ * tensor-core form runs its chain of diagonal factorisations on an internal
+ * stream beside the panel applications and update products (joined by events
+ * recorded on `stream`, so the call stays asynchronous and graph capture sees
+ * one exchange of events per panel; each diagonal step is launched with
+ * programmatic stream serialisation behind the one before it);
  * that stream and its two events are created on the first such call in a host
  * thread and CUDA context -- make that call before any stream capture -- and
  * live until the process exits.
